@@ -1,0 +1,313 @@
+"""Pins for the CPU oracle: each test checks the oracle against something other
+than itself -- a hand-computed fixture, an algebraic identity the pages state,
+a brute-force sum, a closed form or a library routine on a special case.
+CPU only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import serq_oracle as O
+from w4a4_rank_gemm_b200 import synth
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "quantizer_cases.json")))
+F32 = np.float32
+
+
+# --------------------------------------------------------------------------
+# Quantizer, packing, smoothing and ranking against hand-computed fixtures
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("case", GOLD["quantize"], ids=lambda c: c["why"][:20])
+def test_quantizer_golden(case):
+    x = np.array([case["x"]], dtype=F32)
+    q, s = O.quantize_act(x, case["bits"])
+    assert q[0].tolist() == case["codes"]
+    assert float(s[0]) == pytest.approx(case["scale"], rel=1e-7, abs=0)
+
+
+@pytest.mark.parametrize("case", GOLD["pack_int4"], ids=lambda c: c["why"])
+def test_pack_golden(case):
+    b = O.pack_int4_rows(np.array([case["codes"]], dtype=np.int8))
+    assert int(b[0, 0]) == case["byte"]
+    assert O.unpack_int4_rows(b)[0].tolist() == case["codes"]
+
+
+def test_pack_roundtrip_all_codes():
+    codes = np.array([[a, b] for a in range(-8, 8) for b in range(-8, 8)], dtype=np.int8)
+    assert np.array_equal(O.unpack_int4_rows(O.pack_int4_rows(codes)), codes)
+
+
+def test_smooth_scales_golden():
+    g = GOLD["smooth"]
+    s = O.smooth_scales(np.array(g["X_calib"], F32), np.array(g["W"], F32))
+    assert s.tolist() == g["s"]
+
+
+def test_smooth_scales_group_uses_max_over_weights():
+    rng = np.random.default_rng(0)
+    Xc = rng.standard_normal((8, 6)).astype(F32)
+    W1 = rng.standard_normal((6, 5)).astype(F32)
+    W2 = (3 * rng.standard_normal((6, 7))).astype(F32)
+    s = O.smooth_scales(Xc, [W1, W2])
+    amax_w = np.maximum(np.abs(W1).max(1), np.abs(W2).max(1)).astype(np.float64)
+    ref = np.sqrt(np.abs(Xc).max(0).astype(np.float64)) / np.sqrt(amax_w)
+    np.testing.assert_allclose(s, ref, rtol=3e-7)
+
+
+def test_saliency_golden():
+    g = GOLD["saliency"]
+    assert O.saliency_perm(np.array(g["s"], F32)).tolist() == g["perm"]
+
+
+def test_quantizer_extremes_and_range():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((64, 100)).astype(F32)
+    for bits in (4, 8):
+        Q = O.QMAX[bits]
+        q, s = O.quantize_act(x, bits)
+        assert q.min() >= -Q and q.max() <= Q
+        i = np.argmax(np.abs(x), axis=1)
+        assert np.all(np.abs(q[np.arange(64), i]) == Q)       # +-amax -> +-Q
+        # round-to-nearest: error at most half a step (plus fp32 slack)
+        err = np.abs(q * s[:, None].astype(np.float64) - x)
+        assert np.all(err <= 0.5 * s[:, None] * (1 + 1e-5) + 1e-12)
+
+
+# --------------------------------------------------------------------------
+# Flattening and permutation identities ([radio]: X diag(s^-1) P^-1 P diag(s) W
+# = XW; [notes] key design 3: permutation costs nothing)
+# --------------------------------------------------------------------------
+def _layer(seed=0, M=24, K=96, N=40):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((M, K)).astype(F32)
+    X[:, [3, 17, 50]] *= 40
+    W = (0.02 * rng.standard_normal((K, N))).astype(F32)
+    return X, W
+
+
+def test_flatten_permute_identity():
+    X, W = _layer()
+    s = O.smooth_scales(X, W)
+    pi = O.saliency_perm(s)
+    y = O.flatten_permute(X, s, pi, False).astype(np.float64) @ O.fold_weight(W, s, pi).astype(np.float64)
+    ref = X.astype(np.float64) @ W.astype(np.float64)
+    assert np.max(np.abs(y - ref)) <= 1e-5 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_permutation_invariance(seed):
+    X, W = _layer(seed)
+    s = O.smooth_scales(X, W)
+    perm = np.random.default_rng(seed).permutation(X.shape[1]).astype(np.int32)
+    y1 = O.flatten_permute(X, s, perm, False).astype(np.float64) @ O.fold_weight(W, s, perm).astype(np.float64)
+    y2 = O.flatten_permute(X, s, O.saliency_perm(s), False).astype(np.float64) @ \
+        O.fold_weight(W, s, O.saliency_perm(s)).astype(np.float64)
+    assert np.max(np.abs(y1 - y2)) <= 1e-5 * np.max(np.abs(y1))
+
+
+def test_saliency_puts_outlier_channels_first():
+    X, W = _layer()
+    s = O.smooth_scales(X, W)
+    pi = O.saliency_perm(s)
+    assert set(pi[:3].tolist()) == {3, 17, 50}
+    assert np.all(np.diff(s[pi].astype(np.float64)) <= 0)
+
+
+# --------------------------------------------------------------------------
+# Compensator ([notes] core idea: R = W~_s - Q(W~_s))
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("r", [1, 8, 32])
+def test_compensator_reconstructs_salient_rows(r):
+    X, W = _layer(4)
+    L = O.prepare(W, X, r)
+    deq = L.q_w.astype(np.float64) * L.s_w.astype(np.float64)[None, :]
+    recon = deq[:r] + L.R.astype(np.float64)
+    target = L.W_hat[:r].astype(np.float64)
+    # exact up to two fp32 roundings: of code*scale and of the subtraction
+    bound = 2.0 ** -24 * (np.abs(deq[:r]) + np.abs(target - deq[:r]))
+    assert np.all(np.abs(recon - target) <= bound)
+    # and far better than the main path alone
+    assert np.abs(recon - target).max() < 1e-3 * np.abs(target - deq[:r]).max()
+    assert L.R.shape == (r, W.shape[1])       # R is r x d_out
+    # rows past r are untouched by the compensator
+    assert L.q_r.shape == (r, W.shape[1])
+
+
+def test_compensator_is_not_a_separate_quantization():
+    # A plausible mistake is R = W~_s - Q_sep(W~_s) with W~_s quantized on its
+    # own (scale from the r rows only); that does not cancel the main error.
+    X, W = _layer(5)
+    r = 8
+    L = O.prepare(W, X, r)
+    q_sep, s_sep = O.quantize_weight(L.W_hat[:r])
+    R_wrong = L.W_hat[:r] - q_sep * s_sep[None, :]
+    assert not np.allclose(R_wrong, L.R)
+    eff = L.q_w[:r] * L.s_w.astype(np.float64) + L.R
+    assert np.allclose(eff, L.W_hat[:r], atol=1e-7)
+
+
+# --------------------------------------------------------------------------
+# Integer GEMM and epilogue
+# --------------------------------------------------------------------------
+def test_int_matmul_bruteforce():
+    rng = np.random.default_rng(6)
+    a = rng.integers(-7, 8, size=(5, 13)).astype(np.int8)
+    b = rng.integers(-7, 8, size=(13, 4)).astype(np.int8)
+    got = O.int_matmul(a, b)
+    for m in range(5):
+        for n in range(4):
+            assert got[m, n] == sum(int(a[m, k]) * int(b[k, n]) for k in range(13))
+
+
+def test_int_matmul_large_is_exact():
+    # W4A8 worst case: |acc| <= 127 * 7 * K stays exact
+    K = 14336
+    a = np.full((2, K), 127, np.int8); a[1] = -127
+    b = np.full((K, 3), 7, np.int8)
+    got = O.int_matmul(a, b)
+    assert got[0, 0] == 127 * 7 * K and got[1, 2] == -127 * 7 * K
+
+
+def test_linear_equals_dequantize_then_matmul():
+    X, W = _layer(7, M=9, K=64, N=24)
+    r = 16
+    L = O.prepare(W, X, r)
+    xh = O.flatten_permute(X, L.s, L.pi, False)
+    y, xq, sx, acc0, acc1 = O.linear(xh, L, 4)
+    # brute-force definition: Y[m,n] = sum_k deqX[m,k] * Weff[k,n]
+    deqx = xq.astype(np.float64) * sx.astype(np.float64)[:, None]
+    Weff = O.dequant_weight(L, True)
+    ref = np.zeros((9, 24))
+    for m in range(9):
+        for n in range(24):
+            ref[m, n] = math.fsum(deqx[m, k] * Weff[k, n] for k in range(64))
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+    # residual uses only the first r code columns
+    assert np.array_equal(acc1, O.int_matmul(xq[:, :r], L.q_r))
+
+
+def test_w4a8_integer_activations_exact():
+    rng = np.random.default_rng(8)
+    xi = rng.integers(-127, 128, size=(4, 32)).astype(F32)
+    xi[:, 0] = 127
+    q, s = O.quantize_act(xi, 8)
+    assert np.array_equal(q.astype(F32), xi) and np.all(s == 1)
+
+
+def test_r0_reduces_to_smoothquant_rtn():
+    X, W = _layer(9)
+    L = O.prepare(W, X, 0)
+    xh = O.flatten_permute(X, L.s, L.pi, False)
+    y = O.linear(xh, L, 4)[0]
+    # textbook fake-quant matmul: per-token and per-channel RTN in fp64
+    qx, sx = O.quantize_act(xh, 4)
+    qw, sw = O.quantize_weight(L.W_hat, 4)
+    ref = (qx * sx[:, None].astype(np.float64)) @ (qw * sw[None, :].astype(np.float64))
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_r_equals_k_unquantized_leaves_only_activation_error():
+    X, W = _layer(10, K=64)
+    K = 64
+    L = O.prepare(W, X, K)
+    xh = O.flatten_permute(X, L.s, L.pi, False)
+    qx, sx = O.quantize_act(xh, 4)
+    deqx = qx * sx[:, None].astype(np.float64)
+    Weff = L.q_w * L.s_w.astype(np.float64)[None, :] + L.R.astype(np.float64)
+    np.testing.assert_allclose(Weff, L.W_hat, rtol=0, atol=1e-6 * np.abs(L.W_hat).max())
+    y = deqx @ Weff
+    np.testing.assert_allclose(y, deqx @ L.W_hat.astype(np.float64), rtol=1e-5, atol=1e-6)
+
+
+def test_rank_trend_on_outlier_data():
+    """Statistical (the rank ablation's trend: error falls as r grows)."""
+    wl = synth.custom_layer(64, 512, 256, 0, act_dtype="f32", seed=11, n_outliers=8)
+    X, W = wl.inputs["x"].X, wl.projections[0].W
+    ref = X.astype(np.float64) @ W.astype(np.float64)
+    errs = []
+    for r in (0, 16, 128):
+        L = O.prepare(W, wl.inputs["x"].X_calib, r)
+        y = O.linear(O.flatten_permute(X, L.s, L.pi, False), L, 4)[0]
+        errs.append(np.linalg.norm(y - ref) / np.linalg.norm(ref))
+    assert errs[0] > errs[1] > errs[2]
+
+
+# --------------------------------------------------------------------------
+# fp32 exponential and SiLU (Cody-Waite + Taylor) against libm in fp64
+# --------------------------------------------------------------------------
+def test_exp_f32_accuracy():
+    x = np.concatenate([np.linspace(-87.9, 87.9, 200001, dtype=F32),
+                        np.array([0, -0.0, 1e-8, -1e-8, 0.3465, -0.3466, 1, -1], F32)])
+    got = O.exp_f32(x).astype(np.float64)
+    ref = np.exp(x.astype(np.float64))
+    ulp = np.spacing(ref.astype(F32)).astype(np.float64)
+    assert np.max(np.abs(got - ref) / ulp) <= 4.0
+    assert O.exp_f32(np.array([0.0], F32))[0] == 1.0
+
+
+def test_exp_f32_saturation():
+    assert np.isinf(O.exp_f32(np.array([89.0, 200.0], F32))).all()
+    assert (O.exp_f32(np.array([-89.0, -1e4], F32)) == 0).all()
+
+
+def test_silu_mul_against_fp64():
+    rng = np.random.default_rng(12)
+    g = (4 * rng.standard_normal(5000)).astype(F32)
+    u = rng.standard_normal(5000).astype(F32)
+    got = O.silu_mul_f32(g, u).astype(np.float64)
+    gd = g.astype(np.float64)
+    ref = gd / (1 + np.exp(-gd)) * u.astype(np.float64)
+    assert np.max(np.abs(got - ref) / np.maximum(np.abs(ref), 1e-30)) <= 1e-6
+    # saturation: large negative gate -> exactly zero; large positive -> g*u
+    assert O.silu_mul_f32(np.array([-100.0], F32), np.array([3.0], F32))[0] == 0
+    assert O.silu_mul_f32(np.array([100.0], F32), np.array([3.0], F32))[0] == 300.0
+
+
+# --------------------------------------------------------------------------
+# MLP-block permutation propagation ([notes] key design 3)
+# --------------------------------------------------------------------------
+def _silu64(x):
+    return x / (1 + np.exp(-x))
+
+
+def test_mlp_fold_is_exact_without_quantization():
+    rng = np.random.default_rng(13)
+    M, K, F = 8, 32, 48
+    X = rng.standard_normal((M, K)).astype(F32)
+    Wg = (0.1 * rng.standard_normal((K, F))).astype(F32)
+    Wu = (0.1 * rng.standard_normal((K, F))).astype(F32)
+    Wd = (0.1 * rng.standard_normal((F, K))).astype(F32)
+    Hc = (_silu64(X.astype(np.float64) @ Wg) * (X.astype(np.float64) @ Wu)).astype(F32)
+    s4 = O.smooth_scales(Hc, Wd)
+    pi4 = O.saliency_perm(s4)
+    Wg_f = O.fold_output_columns(Wg, pi4, None)
+    Wu_f = O.fold_output_columns(Wu, pi4, s4)
+    s = O.smooth_scales(X, [Wg_f, Wu_f])
+    pi = O.saliency_perm(s)
+    xh = O.flatten_permute(X, s, pi, False).astype(np.float64)
+    g = xh @ O.fold_weight(Wg_f, s, pi).astype(np.float64)
+    u = xh @ O.fold_weight(Wu_f, s, pi).astype(np.float64)
+    h = _silu64(g) * u                                # arrives already as X^_4
+    y = h @ O.fold_weight(Wd, s4, pi4).astype(np.float64)
+    Xd = X.astype(np.float64)
+    ref = (_silu64(Xd @ Wg) * (Xd @ Wu)) @ Wd.astype(np.float64)
+    assert np.max(np.abs(y - ref)) <= 1e-5 * np.max(np.abs(ref))
+    # and the intermediate is exactly down_proj's flattened, permuted input
+    h_direct = O.flatten_permute((_silu64(Xd @ Wg) * (Xd @ Wu)).astype(F32), s4, pi4, False)
+    np.testing.assert_allclose(h, h_direct, rtol=1e-5, atol=1e-6)
+
+
+def test_mlp_quantized_chain_tracks_full_precision():
+    """Statistical: the W4A4 chain stays near the fp64 block (4-bit RTN on
+    Gaussian data costs ~10-15% per layer) and a larger rank helps."""
+    blk = synth.mlp_block(M=32, K=256, F=512, rank=32, seed=14, n_calib=64)
+    Xd = blk.X.astype(np.float64)
+    ref = (_silu64(Xd @ blk.Wg) * (Xd @ blk.Wu)) @ blk.Wd.astype(np.float64)
+    rel = []
+    for r in (0, 128):
+        prep = O.prepare_mlp(blk.Wg, blk.Wu, blk.Wd, blk.X_calib, blk.H_calib, r)
+        y = O.mlp_forward(blk.X, prep)["y"]
+        rel.append(np.linalg.norm(y - ref) / np.linalg.norm(ref))
+    assert rel[1] < rel[0] < 0.4, rel
