@@ -1,0 +1,85 @@
+"""CPU checks of the C ABI: the library loads, exports every function that
+include/serq.h declares, and rejects bad arguments on the host before it
+touches a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "serq.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(serq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a4_rank_gemm_b200 import build
+    build.build()
+    from w4a4_rank_gemm_b200 import serq
+    return serq
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ("serq_prepare_group", "serq_prepare", "serq_quantize_act", "serq_linear",
+                 "serq_linear_accum", "serq_silu_mul_quantize", "serq_layer_destroy"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s+(serq_\w+)$", out, flags=re.M))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    # and the binding knows each of them
+    assert set(_declared()) <= set(lib.EXPORTS)
+
+
+def test_version_and_constants(lib):
+    assert "sm_100a" in lib.version()
+    assert lib.decode_max_m() == 32
+
+
+def test_host_side_argument_rejection(lib):
+    L = lib.lib
+    # null layer / null pointers are rejected before any device call
+    assert L.serq_linear(None, None, None, 16, None, 256, None) == lib.ERR_INVALID_ARG
+    assert b"null" in L.serq_last_error_string()
+    assert L.serq_quantize_act(None, lib.BF16, 4, 256, 256, lib.W4A4, None, None, None) == lib.ERR_INVALID_ARG
+    # K not a multiple of 32 is an unsupported shape (checked before device)
+    fake = ctypes.c_void_p(0x1000)
+    assert L.serq_quantize_act(fake, lib.BF16, 4, 100, 128, lib.W4A4, fake, fake, None) == lib.ERR_UNSUPPORTED_SHAPE
+    # misaligned row stride
+    assert L.serq_quantize_act(fake, lib.BF16, 4, 256, 260, lib.W4A4, fake, fake, None) == lib.ERR_INVALID_ARG
+    # K beyond the quantizer's register budget
+    assert L.serq_quantize_act(fake, lib.BF16, 4, 32768, 32768, lib.W4A4, fake, fake, None) == lib.ERR_UNSUPPORTED_SHAPE
+    # prepare: rank > K and bad N
+    W = (ctypes.c_void_p * 1)(0x1000)
+    N = (ctypes.c_int * 1)(256)
+    out = (ctypes.c_void_p * 1)()
+    assert L.serq_prepare_group(1, W, N, 256, fake, 8, 300, lib.W4A4, None, None, out) == lib.ERR_UNSUPPORTED_SHAPE
+    N[0] = 100
+    assert L.serq_prepare_group(1, W, N, 256, fake, 8, 16, lib.W4A4, None, None, out) == lib.ERR_UNSUPPORTED_SHAPE
+    assert out[0] is None
+    # silu: null inputs
+    assert L.serq_silu_mul_quantize(None, None, 4, 256, 256, lib.W4A4, None, None, None) == lib.ERR_INVALID_ARG
+
+
+def test_binding_refuses_to_load_without_library(tmp_path, monkeypatch):
+    """The product path fails loudly when the CUDA library is missing."""
+    import importlib.util
+    import shutil
+    pkg = tmp_path / "w4a4_rank_gemm_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "w4a4_rank_gemm_b200", "serq.py"), pkg / "serq.py")
+    spec = importlib.util.spec_from_file_location("serq_nolib", pkg / "serq.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="libserq.so not found"):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,296 @@
+// Prefill-regime SERQ linear on the 5th-generation tensor cores (sm_100a):
+//
+//   acc0 = Xq Wq^T            (all K columns)
+//   acc1 = Xq[:, :r] Rq^T     (the r salient columns; SERQ notes key design 2)
+//   Y    = sx * (sw * acc0 + sR * acc1)   -> bf16
+//
+// One CTA computes a 128 x BN output tile.  Warp roles:
+//   warp 0      TMA producer: packed INT4 tiles of X and W (or R) -> smem
+//   warp 1      TMEM owner + single-thread tcgen05.mma issuer
+//   warps 2..9  unpackers: packed nibbles -> int8 (x16) in the 128-byte
+//               swizzled K-major layout the MMA reads; afterwards the same
+//               warps run the epilogue out of TMEM.
+// The k loop runs K/128 main steps into acc0 followed by ceil(r/128)
+// residual steps into acc1; a residual step reloads the matching activation
+// block and takes R in place of W, so both accumulators use one pipeline.
+// Both accumulators stay in TMEM (int32, exact) until the epilogue applies
+// the per-token, per-channel and compensator scales separately.
+//
+// INT4 has no tensor-core input kind of its own, and no FP4 kind represents
+// the codes -7..7 exactly, so the codes are widened to int8 in shared memory
+// and multiplied by kind::i8.  The widening keeps each nibble in the high
+// half of its byte (value x16), so it costs two logic ops per four codes;
+// the factor 16 per widened operand leaves the accumulator exactly and is
+// removed by a shift.
+//
+// W4A8: X arrives as int8 and is loaded by TMA straight into the swizzled
+// layout; only W / R are widened.
+#pragma once
+#include "common.cuh"
+
+namespace serq {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 128;            // k per pipeline step (int8 bytes per row)
+constexpr int PS = 3;              // packed (TMA) stages
+constexpr int US = 2;              // unpacked stages
+constexpr int kUnpackWarps = 8;
+constexpr int kThreads = (2 + kUnpackWarps) * 32;
+
+struct Args {
+  int M, K, N, rpad;
+  int nkb, nrb;  // main and residual steps
+  const float* sx;
+  const float* sw;
+  const float* sr;
+  __nv_bfloat16* Y;
+  int ldy;
+  int32_t* acc0;
+  int32_t* acc1;
+};
+
+template <int BN, bool A8>
+struct Layout {
+  static constexpr int kUnA = BM * BK;                    // unpacked A tile (int8)
+  static constexpr int kUnB = BN * BK;                    // unpacked B tile (int8)
+  static constexpr int kPkA = A8 ? BM * BK : BM * BK / 2; // TMA A tile
+  static constexpr int kPkB = BN * BK / 2;                // TMA B/R tile (packed)
+  static constexpr int oUnA = 0;
+  static constexpr int oUnB = oUnA + (A8 ? 0 : US * kUnA);
+  static constexpr int oPkA = oUnB + US * kUnB;
+  static constexpr int oPkB = oPkA + PS * kPkA;
+  static constexpr int oSw = oPkB + PS * kPkB;
+  static constexpr int oSr = oSw + BN * 4;
+  static constexpr int oBar = oSr + BN * 4;
+  static constexpr int nBar = 2 * PS + 2 * US + 2;
+  static constexpr int oMisc = oBar + nBar * 8;
+  static constexpr int kBytes = oMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-B alignment
+  static constexpr uint32_t kTxBytes = kPkA + kPkB;
+  static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
+  static_assert(oPkA % 1024 == 0 && kPkA % 1024 == 0, "A TMA tiles must stay 1024-aligned");
+  static_assert(oUnB % 1024 == 0 && kUnB % 1024 == 0, "B tiles must stay 1024-aligned");
+};
+
+// One 8-byte packed chunk (16 codes) -> 16 int8 (x16) at the swizzled
+// position of chunk c in row `row` of a 128-byte-row tile.
+__device__ __forceinline__ void unpack_chunk(const uint8_t* src_row, uint8_t* dst_tile, int row, int c) {
+  const uint2 p = *reinterpret_cast<const uint2*>(src_row + 8 * c);
+  const uint2 a = unpack8_x16(p.x);
+  const uint2 b = unpack8_x16(p.y);
+  *reinterpret_cast<uint4*>(dst_tile + row * 128 + ((c ^ (row & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+}
+
+template <int BN, bool A8, bool ACC_OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const __grid_constant__ CUtensorMap tmR, const Args p) {
+  using L = Layout<BN, A8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::oBar);
+  uint64_t* full_pk = bar;              // TMA bytes landed            (tx)
+  uint64_t* empty_pk = bar + PS;        // packed stage consumed
+  uint64_t* full_un = bar + 2 * PS;     // unpacked stage written
+  uint64_t* empty_un = full_un + US;    // unpacked stage read by the MMAs
+  uint64_t* acc_full = empty_un + US;   // all MMAs complete
+  uint64_t* drain = acc_full + 1;       // abort path: MMAs complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::oMisc + 4);
+  float* sw_t = reinterpret_cast<float*>(smem + L::oSw);
+  float* sr_t = reinterpret_cast<float*>(smem + L::oSr);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int nsteps = p.nkb + p.nrb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PS; ++s) {
+      mbar_init(&full_pk[s], 1);
+      mbar_init(&empty_pk[s], kUnpackWarps + (A8 ? 1 : 0));
+    }
+    for (int s = 0; s < US; ++s) {
+      mbar_init(&full_un[s], kUnpackWarps);
+      mbar_init(&empty_un[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmR);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < BN; i += blockDim.x) {
+    const int n = n0 + i;
+    sw_t[i] = (n < p.N) ? p.sw[n] : 0.f;
+    sr_t[i] = (n < p.N) ? p.sr[n] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int step = 0; step < nsteps; ++step) {
+        const int s = step % PS;
+        const uint32_t ph = (step / PS) & 1;
+        if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) break;
+        mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
+        const bool res = step >= p.nkb;
+        const int j = res ? step - p.nkb : step;
+        tma_load_2d(smem + L::oPkA + s * L::kPkA, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
+        tma_load_2d(smem + L::oPkB + s * L::kPkB, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), n0);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_i8(BM, BN);
+      const uint32_t a_base = smem_u32(smem + (A8 ? L::oPkA : L::oUnA));
+      const uint32_t b_base = smem_u32(smem + L::oUnB);
+      bool ok = true;
+      for (int step = 0; step < nsteps && ok; ++step) {
+        const int u = step % US;
+        const uint32_t uph = (step / US) & 1;
+        const int s = step % PS;
+        const uint32_t ph = (step / PS) & 1;
+        if (!mbar_wait(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
+        if (A8 && !mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
+        tc_fence_after();
+        const bool res = step >= p.nkb;
+        const int j = res ? step - p.nkb : step;
+        const int nk = res ? min(BK / 32, (p.rpad - j * BK) / 32) : BK / 32;
+        const uint32_t d = tmem + (res ? (uint32_t)BN : 0u);
+        const uint32_t a_tile = a_base + (A8 ? s * L::kPkA : u * L::kUnA);
+        const uint32_t b_tile = b_base + u * L::kUnB;
+        for (int kk = 0; kk < nk; ++kk) {
+          umma_i8(d, umma_desc_k_sw128(a_tile + kk * 32), umma_desc_k_sw128(b_tile + kk * 32), idesc,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty_un[u]);
+        if (A8) umma_commit(&empty_pk[s]);
+      }
+      if (ok) {
+        umma_commit(acc_full);
+      } else {
+        umma_commit(drain);
+        mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ unpack
+    const int ut = threadIdx.x - 64;  // 0 .. 255
+    constexpr int kRows = (A8 ? 0 : BM) + BN;
+    constexpr int kChunks = kRows * 8;
+    bool ok = true;
+    for (int step = 0; step < nsteps; ++step) {
+      const int s = step % PS;
+      const uint32_t ph = (step / PS) & 1;
+      const int u = step % US;
+      const uint32_t uph = (step / US) & 1;
+      if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+      if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+      const uint8_t* pkA = smem + L::oPkA + s * L::kPkA;
+      const uint8_t* pkB = smem + L::oPkB + s * L::kPkB;
+      uint8_t* unA = smem + L::oUnA + u * L::kUnA;
+      uint8_t* unB = smem + L::oUnB + u * L::kUnB;
+#pragma unroll 4
+      for (int id = ut; id < kChunks; id += kUnpackWarps * 32) {
+        const int row = id >> 3, c = id & 7;
+        if (!A8 && row < BM) {
+          unpack_chunk(pkA + row * (BK / 2), unA, row, c);
+        } else {
+          const int rb = A8 ? row : row - BM;
+          unpack_chunk(pkB + rb * (BK / 2), unB, rb, c);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty_pk[s]);
+        mbar_arrive(&full_un[u]);
+      }
+    }
+
+    // ---------------------------------------------------------- epilogue
+    if (ok && mbar_wait(acc_full, 0, abort_flag, kDevTimeoutEpilogue)) {
+      tc_fence_after();
+      const int q = warp & 3;          // TMEM lane quadrant this warp may access
+      const int half = (warp - 2) >> 2;
+      const int row = m0 + q * 32 + lane;
+      const bool has_r = p.nrb > 0;
+      constexpr int kShift = A8 ? 4 : 8;
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+        uint32_t r0[32], r1[32];
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c;
+        __syncwarp();
+        tmem_ld_32x32b_x32(taddr, r0);
+        if (has_r) tmem_ld_32x32b_x32(taddr + BN, r1);
+        tmem_ld_wait();
+        if (!has_r) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r1[i] = 0;
+        }
+        if (row >= p.M || n0 + c >= p.N) {
+          // row past M (zero-filled A) or column tile past N: nothing to store
+        } else if (ACC_OUT) {
+          int32_t* o0 = p.acc0 + (size_t)row * p.N + n0 + c;
+          int32_t* o1 = p.acc1 + (size_t)row * p.N + n0 + c;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            *reinterpret_cast<int4*>(o0 + i) =
+                make_int4((int)r0[i] >> kShift, (int)r0[i + 1] >> kShift, (int)r0[i + 2] >> kShift,
+                          (int)r0[i + 3] >> kShift);
+            *reinterpret_cast<int4*>(o1 + i) =
+                make_int4((int)r1[i] >> kShift, (int)r1[i + 1] >> kShift, (int)r1[i + 2] >> kShift,
+                          (int)r1[i + 3] >> kShift);
+          }
+        } else {
+          const float sxm = p.sx[row];
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float y0 = sxm * fmaf(sw_t[c + i], (float)((int)r0[i] >> kShift),
+                                        sr_t[c + i] * (float)((int)r1[i] >> kShift));
+            const float y1 = sxm * fmaf(sw_t[c + i + 1], (float)((int)r0[i + 1] >> kShift),
+                                        sr_t[c + i + 1] * (float)((int)r1[i + 1] >> kShift));
+            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+            packed[i >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(p.Y + (size_t)row * p.ldy + n0 + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && warp == 0 && lane == 0) {
+    // Let TMA copies already issued land before the CTA's shared memory is
+    // released (they complete in microseconds; bounded).
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < 100000ull) {
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace tc
+}  // namespace serq

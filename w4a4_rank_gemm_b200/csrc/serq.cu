@@ -1,0 +1,528 @@
+// libserq C ABI: argument checking, the prepared-layer handle, tensor-map
+// construction and kernel dispatch.  Kernels live in the included headers;
+// everything is one translation unit so the device status word is shared.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+
+#include "../../include/serq.h"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv_decode.cuh"
+#include "prepare.cuh"
+#include "quant.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+serq_status fail(serq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+serq_status ok() {
+  g_last_error.clear();
+  return SERQ_OK;
+}
+
+serq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SERQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+serq_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  static int cached[64] = {0};  // 0 unknown, 1 ok, 2 bad
+  if (dev >= 0 && dev < 64 && cached[dev] == 1) return SERQ_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) {
+    return fail(SERQ_ERR_UNSUPPORTED_DEVICE, "device %d is sm_%d%d; libserq needs sm_100 (B200)", dev,
+                major, minor);
+  }
+  if (dev >= 0 && dev < 64) cached[dev] = 1;
+  return SERQ_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [rows][inner] with row stride `stride` bytes.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
+              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+struct serq_layer {
+  int K, N, rank, rpad, mode, device;
+  void* block;
+  uint8_t* wq;
+  uint8_t* rq;
+  float* sw;
+  float* sr;
+  int32_t* perm;
+  float* smooth;
+  CUtensorMap tmB[2];  // box rows 128, 256
+  CUtensorMap tmR[2];
+};
+
+namespace {
+
+serq_status alloc_layer(int K, int N, int rank, int mode, serq_layer** out) {
+  serq_layer* L = new (std::nothrow) serq_layer();
+  if (!L) return fail(SERQ_ERR_ALLOC, "host allocation failed");
+  std::memset(L, 0, sizeof(*L));
+  L->K = K;
+  L->N = N;
+  L->rank = rank;
+  L->rpad = (rank + 31) / 32 * 32;
+  L->mode = mode;
+  cudaGetDevice(&L->device);
+  const size_t s_wq = up256((size_t)N * K / 2);
+  const size_t s_rq = up256((size_t)N * L->rpad / 2);
+  const size_t s_n = up256((size_t)N * 4);
+  const size_t s_k = up256((size_t)K * 4);
+  const size_t total = s_wq + s_rq + 2 * s_n + 2 * s_k;
+  cudaError_t e = cudaMalloc(&L->block, total);
+  if (e != cudaSuccess) {
+    delete L;
+    cudaGetLastError();
+    return fail(SERQ_ERR_ALLOC, "cudaMalloc(%zu) failed: %s", total, cudaGetErrorString(e));
+  }
+  uint8_t* b = static_cast<uint8_t*>(L->block);
+  L->wq = b;
+  b += s_wq;
+  L->rq = L->rpad ? b : nullptr;
+  b += s_rq;
+  L->sw = reinterpret_cast<float*>(b);
+  b += s_n;
+  L->sr = reinterpret_cast<float*>(b);
+  b += s_n;
+  L->perm = reinterpret_cast<int32_t*>(b);
+  b += s_k;
+  L->smooth = reinterpret_cast<float*>(b);
+  *out = L;
+  return SERQ_OK;
+}
+
+void free_layer(serq_layer* L) {
+  if (!L) return;
+  if (L->block) cudaFree(L->block);
+  delete L;
+}
+
+bool build_weight_maps(serq_layer* L) {
+  const int boxes[2] = {128, 256};
+  for (int i = 0; i < 2; ++i) {
+    if (!make_map(&L->tmB[i], L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 64, boxes[i],
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+    if (L->rpad) {
+      if (!make_map(&L->tmR[i], L->rq, (uint64_t)L->rpad / 2, (uint64_t)L->N, (uint64_t)L->rpad / 2, 64,
+                    boxes[i], CU_TENSOR_MAP_SWIZZLE_NONE))
+        return false;
+    } else {
+      L->tmR[i] = L->tmB[i];  // never read when r = 0
+    }
+  }
+  return true;
+}
+
+serq_status check_layer(const serq_layer* L) {
+  if (!L) return fail(SERQ_ERR_INVALID_ARG, "null layer");
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != L->device)
+    return fail(SERQ_ERR_INVALID_ARG, "layer was prepared on device %d, current device is %d", L->device, dev);
+  return SERQ_OK;
+}
+
+template <class K>
+void set_smem(K kernel, int bytes) {
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// ------------------------------------------------------------ GEMM launch
+template <int BN, bool A8, bool ACC>
+cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, cudaStream_t st) {
+  using Lay = serq::tc::Layout<BN, A8>;
+  CUtensorMap tmA;
+  bool okm = A8 ? make_map(&tmA, Xq, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, 128, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B)
+                : make_map(&tmA, Xq, (uint64_t)a.K / 2, (uint64_t)a.M, (uint64_t)a.K / 2, 64, 128,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!okm) return cudaErrorInvalidValue;
+  const int bi = (BN == 256) ? 1 : 0;
+  auto kern = serq::tc::k_gemm<BN, A8, ACC>;
+  static int attr_set[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    set_smem(kern, Lay::kAlloc);
+    attr_set[dev] = 1;
+  }
+  dim3 grid((a.N + BN - 1) / BN, (a.M + serq::tc::BM - 1) / serq::tc::BM);
+  kern<<<grid, serq::tc::kThreads, Lay::kAlloc, st>>>(tmA, L->tmB[bi], L->tmR[bi], a);
+  return cudaGetLastError();
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (dev < 64) cached[dev] = sms;
+  return sms;
+}
+
+template <bool A8, bool ACC>
+cudaError_t dispatch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, serq_algo algo,
+                        cudaStream_t st) {
+  if (algo == SERQ_ALGO_PREFILL_N128) return launch_tc<128, A8, ACC>(L, Xq, a, st);
+  if (algo == SERQ_ALGO_PREFILL_N256) return launch_tc<256, A8, ACC>(L, Xq, a, st);
+  // 256-wide tiles unless that leaves most SMs idle.
+  const long tiles256 = (long)((a.N + 255) / 256) * ((a.M + 127) / 128);
+  if (tiles256 * 10 < (long)sm_count() * 9) return launch_tc<128, A8, ACC>(L, Xq, a, st);
+  return launch_tc<256, A8, ACC>(L, Xq, a, st);
+}
+
+serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, int M, void* Y, int ldy,
+                        int32_t* acc0, int32_t* acc1, serq_algo algo, void* stream) {
+  serq_status s;
+  if (!L) return fail(SERQ_ERR_INVALID_ARG, "null layer");
+  const bool accum = (acc0 != nullptr);
+  if (!Xq) return fail(SERQ_ERR_INVALID_ARG, "null Xq");
+  if (M < 1 || M > 65535 * 128) return fail(SERQ_ERR_INVALID_ARG, "M = %d out of range", M);
+  if (!aligned16(Xq)) return fail(SERQ_ERR_INVALID_ARG, "Xq must be 16-byte aligned");
+  if (accum) {
+    if (!acc1) return fail(SERQ_ERR_INVALID_ARG, "null acc1");
+    if (!aligned16(acc0) || !aligned16(acc1)) return fail(SERQ_ERR_INVALID_ARG, "acc0/acc1 must be 16-byte aligned");
+  } else {
+    if (!sx || !Y) return fail(SERQ_ERR_INVALID_ARG, "null sx or Y");
+    if (ldy < L->N) return fail(SERQ_ERR_INVALID_ARG, "ldy (%d) < N (%d)", ldy, L->N);
+    if (!aligned16(Y) || (ldy % 8) != 0)
+      return fail(SERQ_ERR_INVALID_ARG, "Y must be 16-byte aligned with ldy a multiple of 8");
+  }
+  if (algo == SERQ_ALGO_AUTO) algo = (M <= serq_decode_max_m()) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
+  if (algo == SERQ_ALGO_DECODE && M > serq::decode::kMaxTiles * 16)
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "decode kernel takes M <= %d (got %d)", serq::decode::kMaxTiles * 16, M);
+  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_PREFILL_N256) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
+  if ((s = check_device())) return s;
+  if ((s = check_layer(L))) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool a8 = (L->mode == SERQ_W4A8);
+  cudaError_t e;
+  if (algo == SERQ_ALGO_DECODE) {
+    serq::decode::Args a{static_cast<const uint8_t*>(Xq), sx, M, L->K, L->N, L->rpad, L->wq, L->rq, L->sw,
+                         L->sr, static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1};
+    if (a8)
+      e = accum ? serq::decode::launch<true, true>(a, st) : serq::decode::launch<true, false>(a, st);
+    else
+      e = accum ? serq::decode::launch<false, true>(a, st) : serq::decode::launch<false, false>(a, st);
+  } else {
+    serq::tc::Args a{M, L->K, L->N, L->rpad, (L->K + serq::tc::BK - 1) / serq::tc::BK,
+                     (L->rpad + serq::tc::BK - 1) / serq::tc::BK, sx, L->sw, L->sr,
+                     static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1};
+    if (a8)
+      e = accum ? dispatch_tc<true, true>(L, Xq, a, algo, st) : dispatch_tc<true, false>(L, Xq, a, algo, st);
+    else
+      e = accum ? dispatch_tc<false, true>(L, Xq, a, algo, st) : dispatch_tc<false, false>(L, Xq, a, algo, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "serq_linear launch");
+  return ok();
+}
+
+serq_status check_rows(const void* X, int M, int K, int ld, int elem, const char* name) {
+  if (!X) return fail(SERQ_ERR_INVALID_ARG, "null %s", name);
+  if (M < 1 || M > 2147483647 / 2) return fail(SERQ_ERR_INVALID_ARG, "M = %d out of range", M);
+  if (K < 32 || K % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "K = %d must be a positive multiple of 32", K);
+  if (ld < K) return fail(SERQ_ERR_INVALID_ARG, "leading dimension of %s (%d) < K (%d)", name, ld, K);
+  if (!aligned16(X) || ((size_t)ld * elem) % 16)
+    return fail(SERQ_ERR_INVALID_ARG, "%s rows must start 16-byte aligned", name);
+  return SERQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* serq_version(void) { return "libserq 0.1 (sm_100a)"; }
+
+const char* serq_last_error_string(void) { return g_last_error.c_str(); }
+
+int serq_decode_max_m(void) { return 32; }
+
+serq_status serq_check_device(void) {
+  serq_status s = check_device();
+  return s ? s : ok();
+}
+
+serq_status serq_device_error(int* code) {
+  if (!code) return fail(SERQ_ERR_INVALID_ARG, "null code");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, serq::g_device_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device status");
+  e = cudaMemcpyToSymbol(serq::g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device status");
+  *code = v;
+  return ok();
+}
+
+serq_status serq_prepare_group(int n_weights, const float* const* W, const int* N, int K,
+                               const float* X_calib, int n_calib, int rank, serq_mode mode,
+                               const int32_t* const* out_perm, const float* const* out_div,
+                               serq_layer** layers) {
+  if (!layers) return fail(SERQ_ERR_INVALID_ARG, "null layers");
+  if (n_weights < 1 || n_weights > 64) return fail(SERQ_ERR_INVALID_ARG, "n_weights = %d", n_weights);
+  for (int i = 0; i < n_weights; ++i) layers[i] = nullptr;
+  serq_status s;
+  if (!W || !N || !X_calib) return fail(SERQ_ERR_INVALID_ARG, "null W, N or X_calib");
+  if (K < 32 || K % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "K = %d must be a positive multiple of 32", K);
+  if (n_calib < 1) return fail(SERQ_ERR_INVALID_ARG, "n_calib = %d", n_calib);
+  if (rank < 0 || rank > K) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "rank %d not in [0, K=%d]", rank, K);
+  if (mode != SERQ_W4A4 && mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode %d", (int)mode);
+  for (int i = 0; i < n_weights; ++i) {
+    if (!W[i]) return fail(SERQ_ERR_INVALID_ARG, "null W[%d]", i);
+    if (N[i] < 32 || N[i] % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "N[%d] = %d must be a positive multiple of 32", i, N[i]);
+    if (out_div && out_div[i] && !(out_perm && out_perm[i]))
+      return fail(SERQ_ERR_INVALID_ARG, "out_div[%d] given without out_perm[%d]", i, i);
+  }
+  if ((s = check_device())) return s;
+
+  for (int i = 0; i < n_weights; ++i) {
+    s = alloc_layer(K, N[i], rank, mode, &layers[i]);
+    if (s) {
+      for (int j = 0; j < i; ++j) {
+        free_layer(layers[j]);
+        layers[j] = nullptr;
+      }
+      return s;
+    }
+  }
+  auto cleanup = [&](serq_status st) {
+    for (int i = 0; i < n_weights; ++i) {
+      free_layer(layers[i]);
+      layers[i] = nullptr;
+    }
+    return st;
+  };
+
+  cudaStream_t st;
+  cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaStreamCreate"));
+  using namespace serq::prep;
+  serq_layer* L0 = layers[0];
+  auto view = [&](int i) {
+    return WeightView{W[i], N[i], out_perm ? out_perm[i] : nullptr, out_div ? out_div[i] : nullptr};
+  };
+  // 1. flattening scales: amax_x into L0->smooth, amax_w into L0->perm's bytes
+  float* amax_w = reinterpret_cast<float*>(L0->perm);
+  k_colmax_abs<<<(K + 255) / 256, 256, 0, st>>>(X_calib, n_calib, K, L0->smooth);
+  cudaMemsetAsync(amax_w, 0, sizeof(float) * K, st);
+  for (int i = 0; i < n_weights; ++i) k_rowmax_abs<<<K, 256, 0, st>>>(view(i), K, amax_w);
+  k_smooth<<<(K + 255) / 256, 256, 0, st>>>(L0->smooth, amax_w, K);
+  // 2. saliency order
+  k_rank_perm<<<(K + 255) / 256, 256, 256 * sizeof(float), st>>>(L0->smooth, K, L0->perm);
+  for (int i = 1; i < n_weights; ++i) {
+    cudaMemcpyAsync(layers[i]->smooth, L0->smooth, sizeof(float) * K, cudaMemcpyDeviceToDevice, st);
+    cudaMemcpyAsync(layers[i]->perm, L0->perm, sizeof(int32_t) * K, cudaMemcpyDeviceToDevice, st);
+  }
+  // 3-4. per weight: quantize W^ per output channel, compensator R
+  for (int i = 0; i < n_weights; ++i) {
+    serq_layer* Li = layers[i];
+    const WeightView v = view(i);
+    const int Ni = N[i];
+    const int rows_per_block = 64;
+    cudaMemsetAsync(Li->sw, 0, sizeof(float) * Ni, st);
+    k_colmax_what<<<dim3((Ni + 255) / 256, (K + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(
+        v, L0->smooth, L0->perm, K, rows_per_block, Li->sw);
+    k_quant_pack_w<<<dim3((Ni + 127) / 128, K / 8), 128, 0, st>>>(v, L0->smooth, L0->perm, K, Li->sw, Li->wq);
+    if (rank > 0) {
+      k_colmax_resid<<<(Ni + 127) / 128, 128, 0, st>>>(v, L0->smooth, L0->perm, rank, Li->sw, Li->sr);
+      k_quant_pack_r<<<dim3((Ni + 127) / 128, Li->rpad / 8), 128, 0, st>>>(v, L0->smooth, L0->perm, rank,
+                                                                          Li->rpad, Li->sw, Li->sr, Li->rq);
+    }
+    k_finalize_scales<<<(Ni + 255) / 256, 256, 0, st>>>(Li->sw, Li->sr, Ni, rank > 0);
+  }
+  e = cudaGetLastError();
+  cudaError_t e2 = cudaStreamSynchronize(st);
+  cudaStreamDestroy(st);
+  if (e != cudaSuccess) return cleanup(cuda_fail(e, "serq_prepare launch"));
+  if (e2 != cudaSuccess) return cleanup(cuda_fail(e2, "serq_prepare"));
+  for (int i = 0; i < n_weights; ++i)
+    if (!build_weight_maps(layers[i])) return cleanup(fail(SERQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for weights"));
+  return ok();
+}
+
+serq_status serq_prepare(const float* W, int K, int N, const float* X_calib, int n_calib, int rank,
+                         serq_mode mode, const int32_t* out_perm, const float* out_div, serq_layer** layer) {
+  const float* Ws[1] = {W};
+  const int Ns[1] = {N};
+  const int32_t* ps[1] = {out_perm};
+  const float* ds[1] = {out_div};
+  return serq_prepare_group(1, Ws, Ns, K, X_calib, n_calib, rank, mode, ps, ds, layer);
+}
+
+void serq_layer_destroy(serq_layer* layer) { free_layer(layer); }
+
+serq_status serq_layer_info(const serq_layer* L, int* K, int* N, int* rank, int* mode) {
+  if (!L) return fail(SERQ_ERR_INVALID_ARG, "null layer");
+  if (K) *K = L->K;
+  if (N) *N = L->N;
+  if (rank) *rank = L->rank;
+  if (mode) *mode = L->mode;
+  return ok();
+}
+
+serq_status serq_layer_perm_smooth(const serq_layer* L, const int32_t** perm, const float** smooth) {
+  if (!L) return fail(SERQ_ERR_INVALID_ARG, "null layer");
+  if (perm) *perm = L->perm;
+  if (smooth) *smooth = L->smooth;
+  return ok();
+}
+
+serq_status serq_layer_get_packed(const serq_layer* L, uint8_t* wq, uint8_t* rq, float* sw, float* sr,
+                                  int32_t* perm, float* smooth) {
+  serq_status s = check_layer(L);
+  if (s) return s;
+  cudaError_t e = cudaSuccess;
+  auto cp = [&](void* dst, const void* src, size_t n) {
+    if (dst && src && n && e == cudaSuccess) e = cudaMemcpy(dst, src, n, cudaMemcpyDeviceToHost);
+  };
+  cp(wq, L->wq, (size_t)L->N * L->K / 2);
+  cp(rq, L->rq, (size_t)L->N * L->rpad / 2);
+  cp(sw, L->sw, sizeof(float) * L->N);
+  cp(sr, L->sr, sizeof(float) * L->N);
+  cp(perm, L->perm, sizeof(int32_t) * L->K);
+  cp(smooth, L->smooth, sizeof(float) * L->K);
+  if (e != cudaSuccess) return cuda_fail(e, "serq_layer_get_packed");
+  return ok();
+}
+
+serq_status serq_quantize_act(const void* X, serq_dtype dtype, int M, int K, int ldx, serq_mode mode, void* Xq,
+                              float* sx, void* stream) {
+  serq_status s;
+  if (dtype != SERQ_F32 && dtype != SERQ_BF16) return fail(SERQ_ERR_INVALID_ARG, "bad dtype");
+  if ((s = check_rows(X, M, K, ldx, dtype == SERQ_F32 ? 4 : 2, "X"))) return s;
+  if (K > 16384) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "quantize takes K <= 16384 (got %d)", K);
+  if (!Xq || !sx) return fail(SERQ_ERR_INVALID_ARG, "null Xq or sx");
+  if (!aligned16(Xq)) return fail(SERQ_ERR_INVALID_ARG, "Xq must be 16-byte aligned");
+  if (mode != SERQ_W4A4 && mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode");
+  if ((s = check_device())) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* q = static_cast<uint8_t*>(Xq);
+  cudaError_t e;
+  using namespace serq::quant;
+  if (dtype == SERQ_BF16) {
+    LoadBF16 ld{static_cast<const __nv_bfloat16*>(X), ldx};
+    e = (mode == SERQ_W4A4) ? launch_quant_rows<7>(ld, M, K, q, sx, st) : launch_quant_rows<127>(ld, M, K, q, sx, st);
+  } else {
+    LoadF32 ld{static_cast<const float*>(X), ldx};
+    e = (mode == SERQ_W4A4) ? launch_quant_rows<7>(ld, M, K, q, sx, st) : launch_quant_rows<127>(ld, M, K, q, sx, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "serq_quantize_act launch");
+  return ok();
+}
+
+serq_status serq_silu_mul_quantize(const void* G, const void* U, int M, int F, int ld, serq_mode mode, void* Xq,
+                                   float* sx, void* stream) {
+  serq_status s;
+  if ((s = check_rows(G, M, F, ld, 2, "G"))) return s;
+  if ((s = check_rows(U, M, F, ld, 2, "U"))) return s;
+  if (F > 16384) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "quantize takes K <= 16384 (got %d)", F);
+  if (!Xq || !sx) return fail(SERQ_ERR_INVALID_ARG, "null Xq or sx");
+  if (!aligned16(Xq)) return fail(SERQ_ERR_INVALID_ARG, "Xq must be 16-byte aligned");
+  if (mode != SERQ_W4A4 && mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode");
+  if ((s = check_device())) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  serq::quant::LoadSiluMul ldr{static_cast<const __nv_bfloat16*>(G), static_cast<const __nv_bfloat16*>(U), ld};
+  uint8_t* q = static_cast<uint8_t*>(Xq);
+  cudaError_t e = (mode == SERQ_W4A4) ? serq::quant::launch_quant_rows<7>(ldr, M, F, q, sx, st)
+                                      : serq::quant::launch_quant_rows<127>(ldr, M, F, q, sx, st);
+  if (e != cudaSuccess) return cuda_fail(e, "serq_silu_mul_quantize launch");
+  return ok();
+}
+
+serq_status serq_flatten_permute(const serq_layer* L, const void* X, serq_dtype in_dtype, int M, int ldx, void* Xh,
+                                 serq_dtype out_dtype, int ldxh, void* stream) {
+  serq_status s;
+  if (!L) return fail(SERQ_ERR_INVALID_ARG, "null layer");
+  if (!X || !Xh) return fail(SERQ_ERR_INVALID_ARG, "null X or Xh");
+  if (M < 1 || M > 65535) return fail(SERQ_ERR_INVALID_ARG, "M = %d out of range (1..65535)", M);
+  if (ldx < L->K || ldxh < L->K) return fail(SERQ_ERR_INVALID_ARG, "leading dimension < K");
+  const bool ib = (in_dtype == SERQ_BF16), ob = (out_dtype == SERQ_BF16);
+  if ((in_dtype != SERQ_F32 && !ib) || (out_dtype != SERQ_F32 && !ob)) return fail(SERQ_ERR_INVALID_ARG, "bad dtype");
+  if ((s = check_device())) return s;
+  if ((s = check_layer(L))) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid((L->K + 255) / 256, M);
+  using namespace serq::quant;
+  if (ib && ob) k_flatten_permute<true, true><<<grid, 256, 0, st>>>(X, ldx, L->perm, L->smooth, M, L->K, Xh, ldxh);
+  else if (ib) k_flatten_permute<true, false><<<grid, 256, 0, st>>>(X, ldx, L->perm, L->smooth, M, L->K, Xh, ldxh);
+  else if (ob) k_flatten_permute<false, true><<<grid, 256, 0, st>>>(X, ldx, L->perm, L->smooth, M, L->K, Xh, ldxh);
+  else k_flatten_permute<false, false><<<grid, 256, 0, st>>>(X, ldx, L->perm, L->smooth, M, L->K, Xh, ldxh);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "serq_flatten_permute launch");
+  return ok();
+}
+
+serq_status serq_linear(const serq_layer* layer, const void* Xq, const float* sx, int M, void* Y, int ldy,
+                        void* stream) {
+  return linear_impl(layer, Xq, sx, M, Y, ldy, nullptr, nullptr, SERQ_ALGO_AUTO, stream);
+}
+
+serq_status serq_linear_ex(const serq_layer* layer, const void* Xq, const float* sx, int M, void* Y, int ldy,
+                           serq_algo algo, void* stream) {
+  return linear_impl(layer, Xq, sx, M, Y, ldy, nullptr, nullptr, algo, stream);
+}
+
+serq_status serq_linear_accum(const serq_layer* layer, const void* Xq, int M, int32_t* acc0, int32_t* acc1,
+                              serq_algo algo, void* stream) {
+  if (!acc0 || !acc1) return fail(SERQ_ERR_INVALID_ARG, "null acc0 or acc1");
+  return linear_impl(layer, Xq, nullptr, M, nullptr, 0, acc0, acc1, algo, stream);
+}
+
+}  // extern "C"

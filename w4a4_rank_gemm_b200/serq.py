@@ -1,0 +1,252 @@
+"""Thin Python binding of libserq (ctypes).  Argument marshalling only: every
+step runs in the library's CUDA kernels.  torch is used for device memory and
+streams.  Importing this module fails loudly if libserq.so is missing."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libserq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libserq.so not found at {LIB_PATH}; build it with "
+        "`python -m w4a4_rank_gemm_b200.build` (there is no fallback path)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+# enums
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_UNSUPPORTED_DEVICE, ERR_ALLOC, ERR_CUDA, ERR_TIMEOUT = range(7)
+W4A4, W4A8 = 0, 1
+F32, BF16 = 0, 1
+ALGO_AUTO, ALGO_PREFILL, ALGO_DECODE, ALGO_PREFILL_N128, ALGO_PREFILL_N256 = 0, 1, 2, 3, 4
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+EXPORTS = {
+    "serq_prepare_group": (_i, [_i, ctypes.POINTER(_vp), ctypes.POINTER(_i), _i, _vp, _i, _i, _i,
+                                ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
+    "serq_prepare": (_i, [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp, ctypes.POINTER(_vp)]),
+    "serq_layer_destroy": (None, [_vp]),
+    "serq_layer_info": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "serq_layer_perm_smooth": (_i, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
+    "serq_layer_get_packed": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "serq_quantize_act": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "serq_linear": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp]),
+    "serq_linear_ex": (_i, [_vp, _vp, _vp, _i, _vp, _i, _i, _vp]),
+    "serq_linear_accum": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp]),
+    "serq_silu_mul_quantize": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "serq_flatten_permute": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _i, _vp]),
+    "serq_decode_max_m": (_i, []),
+    "serq_last_error_string": (ctypes.c_char_p, []),
+    "serq_check_device": (_i, []),
+    "serq_device_error": (_i, [ctypes.POINTER(_i)]),
+    "serq_version": (ctypes.c_char_p, []),
+}
+
+for _name, (_res, _args) in EXPORTS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class SerqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.serq_last_error_string().decode(errors="replace")
+        super().__init__(f"{where}: status {status}: {msg}")
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise SerqError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported activation dtype {t.dtype}")
+
+
+def _mode_code(mode) -> int:
+    if isinstance(mode, str):
+        return {"w4a4": W4A4, "w4a8": W4A8}[mode.lower()]
+    return int(mode)
+
+
+def _cuda2d(t: torch.Tensor, name: str):
+    if not t.is_cuda or t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D CUDA tensor with unit column stride")
+
+
+class Layer:
+    """Owner of one prepared SERQ layer (device-resident packed weights)."""
+
+    def __init__(self, handle: ctypes.c_void_p):
+        self._h = handle
+        K, N, r, m = _i(), _i(), _i(), _i()
+        _check(lib.serq_layer_info(handle, ctypes.byref(K), ctypes.byref(N), ctypes.byref(r), ctypes.byref(m)),
+               "serq_layer_info")
+        self.K, self.N, self.rank, self.mode = K.value, N.value, r.value, m.value
+        self.rpad = (self.rank + 31) // 32 * 32
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h:
+            lib.serq_layer_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def perm_smooth_ptrs(self) -> Tuple[int, int]:
+        p, s = _vp(), _vp()
+        _check(lib.serq_layer_perm_smooth(self._h, ctypes.byref(p), ctypes.byref(s)), "serq_layer_perm_smooth")
+        return p.value, s.value
+
+    def perm_smooth(self) -> Tuple[torch.Tensor, torch.Tensor]:
+        """Device copies of the saliency order (int32[K]) and scales (f32[K])."""
+        d = self.get_packed()
+        return d["perm"], d["smooth"]
+
+    def get_packed(self) -> dict:
+        """Host copies of everything prepare produced."""
+        import numpy as np
+        wq = np.empty(self.N * self.K // 2, np.uint8)
+        rq = np.empty(max(1, self.N * self.rpad // 2), np.uint8)
+        sw = np.empty(self.N, np.float32)
+        sr = np.empty(self.N, np.float32)
+        perm = np.empty(self.K, np.int32)
+        smooth = np.empty(self.K, np.float32)
+        c = lambda a: a.ctypes.data_as(_vp)
+        _check(lib.serq_layer_get_packed(self._h, c(wq), c(rq) if self.rpad else None, c(sw), c(sr), c(perm),
+                                         c(smooth)), "serq_layer_get_packed")
+        return dict(wq=wq.reshape(self.N, self.K // 2),
+                    rq=rq[: self.N * self.rpad // 2].reshape(self.N, self.rpad // 2),
+                    sw=sw, sr=sr, perm=perm, smooth=smooth)
+
+
+def prepare_group(weights: Sequence[torch.Tensor], X_calib: torch.Tensor, rank: int, mode="w4a4",
+                  out_perm: Optional[Sequence[Optional[torch.Tensor]]] = None,
+                  out_div: Optional[Sequence[Optional[torch.Tensor]]] = None) -> List[Layer]:
+    """serq_prepare_group: weights are CUDA fp32 K x N tensors sharing one input."""
+    n = len(weights)
+    K = weights[0].shape[0]
+    for w in weights:
+        _cuda2d(w, "W")
+        if w.dtype != torch.float32 or not w.is_contiguous() or w.shape[0] != K:
+            raise ValueError("weights must be contiguous fp32 K x N CUDA tensors with equal K")
+    _cuda2d(X_calib, "X_calib")
+    if X_calib.dtype != torch.float32 or not X_calib.is_contiguous():
+        raise ValueError("X_calib must be contiguous fp32")
+    Ws = (_vp * n)(*[w.data_ptr() for w in weights])
+    Ns = (_i * n)(*[w.shape[1] for w in weights])
+    ps = (_vp * n)(*[(p.data_ptr() if p is not None else None) for p in (out_perm or [None] * n)])
+    ds = (_vp * n)(*[(d.data_ptr() if d is not None else None) for d in (out_div or [None] * n)])
+    outs = (_vp * n)()
+    _check(lib.serq_prepare_group(n, Ws, Ns, K, _ptr(X_calib), X_calib.shape[0], rank, _mode_code(mode), ps, ds,
+                                  outs), "serq_prepare_group")
+    return [Layer(_vp(outs[i])) for i in range(n)]
+
+
+def prepare(W: torch.Tensor, X_calib: torch.Tensor, rank: int, mode="w4a4", out_perm=None,
+            out_div=None) -> Layer:
+    return prepare_group([W], X_calib, rank, mode, [out_perm], [out_div])[0]
+
+
+def act_bytes_per_row(K: int, mode) -> int:
+    return K // 2 if _mode_code(mode) == W4A4 else K
+
+
+def quantize_act(X: torch.Tensor, mode="w4a4", Xq: Optional[torch.Tensor] = None,
+                 sx: Optional[torch.Tensor] = None, stream=None):
+    _cuda2d(X, "X")
+    M, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((M, act_bytes_per_row(K, mode)), dtype=torch.uint8, device=X.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=X.device)
+    _check(lib.serq_quantize_act(_ptr(X), _dtype_code(X), M, K, X.stride(0), _mode_code(mode), _ptr(Xq), _ptr(sx),
+                                 _stream(stream)), "serq_quantize_act")
+    return Xq, sx
+
+
+def silu_mul_quantize(G: torch.Tensor, U: torch.Tensor, mode="w4a4", Xq=None, sx=None, stream=None):
+    _cuda2d(G, "G")
+    _cuda2d(U, "U")
+    if G.shape != U.shape or G.stride(0) != U.stride(0) or G.dtype != torch.bfloat16 or U.dtype != torch.bfloat16:
+        raise ValueError("G and U must be bf16 tensors of one shape and stride")
+    M, F = G.shape
+    if Xq is None:
+        Xq = torch.empty((M, act_bytes_per_row(F, mode)), dtype=torch.uint8, device=G.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=G.device)
+    _check(lib.serq_silu_mul_quantize(_ptr(G), _ptr(U), M, F, G.stride(0), _mode_code(mode), _ptr(Xq), _ptr(sx),
+                                      _stream(stream)), "serq_silu_mul_quantize")
+    return Xq, sx
+
+
+def flatten_permute(layer: Layer, X: torch.Tensor, out_dtype=torch.bfloat16, Xh=None, stream=None):
+    _cuda2d(X, "X")
+    M, K = X.shape
+    if Xh is None:
+        Xh = torch.empty((M, K), dtype=out_dtype, device=X.device)
+    _check(lib.serq_flatten_permute(layer.handle, _ptr(X), _dtype_code(X), M, X.stride(0), _ptr(Xh),
+                                    _dtype_code(Xh), Xh.stride(0), _stream(stream)), "serq_flatten_permute")
+    return Xh
+
+
+def linear(layer: Layer, Xq: torch.Tensor, sx: torch.Tensor, Y: Optional[torch.Tensor] = None,
+           algo: int = ALGO_AUTO, stream=None) -> torch.Tensor:
+    M = Xq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=Xq.device)
+    _check(lib.serq_linear_ex(layer.handle, _ptr(Xq), _ptr(sx), M, _ptr(Y), Y.stride(0), algo, _stream(stream)),
+           "serq_linear")
+    return Y
+
+
+def linear_accum(layer: Layer, Xq: torch.Tensor, algo: int = ALGO_AUTO, stream=None):
+    M = Xq.shape[0]
+    acc0 = torch.empty((M, layer.N), dtype=torch.int32, device=Xq.device)
+    acc1 = torch.empty((M, layer.N), dtype=torch.int32, device=Xq.device)
+    _check(lib.serq_linear_accum(layer.handle, _ptr(Xq), M, _ptr(acc0), _ptr(acc1), algo, _stream(stream)),
+           "serq_linear_accum")
+    return acc0, acc1
+
+
+def device_error() -> int:
+    c = _i()
+    _check(lib.serq_device_error(ctypes.byref(c)), "serq_device_error")
+    return c.value
+
+
+def decode_max_m() -> int:
+    return lib.serq_decode_max_m()
+
+
+def version() -> str:
+    return lib.serq_version().decode()
