@@ -320,8 +320,9 @@ def test_rejected_calls_launch_nothing(S):
         S.linear(L, Xq, sx, Y=Y, algo=S.ALGO_DECODE)     # M = 100 > 64
     with pytest.raises(S.SerqError, match="16-byte aligned"):
         S.linear(L, Xq[:, 1:], sx, Y=Y)                  # misaligned activation pointer
-    with pytest.raises(S.SerqError, match="ldy"):
-        S.lib.serq_linear(L.handle, S._ptr(Xq), S._ptr(sx), 100, S._ptr(Y), 64, None)  # ldy < N
+    # ldy < N, through the raw C entry point (returns a status, raises nothing)
+    assert S.lib.serq_linear(L.handle, S._ptr(Xq), S._ptr(sx), 100, S._ptr(Y), 64, None) == S.ERR_INVALID_ARG
+    assert b"ldy" in S.lib.serq_last_error_string()
     torch.cuda.synchronize()
     assert torch.all(Y == 3.0)
     assert S.device_error() == 0
