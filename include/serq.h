@@ -23,9 +23,11 @@
  *    it.  serq_prepare* and the serq_layer_get_* copies are synchronous.
  *  - Matrices are row-major.  K = d_in, N = d_out, M = tokens, r = rank.
  *    K and N must be multiples of 32; 0 <= r <= K.
- *  - Packed INT4: two's-complement nibbles, two per byte, the even column in
- *    the low nibble.  Activations: M rows of K/2 bytes (W4A4) or K bytes of
- *    int8 (W4A8).  Codes lie in [-7, 7] (INT4) or [-127, 127] (INT8).
+ *  - Packed INT4 (activations, weights, compensator): two's-complement
+ *    nibbles; every run of 32 consecutive codes of a row is 16 bytes, byte j
+ *    holding code j of the run in its low nibble and code j + 16 in its high
+ *    nibble.  Activations: M rows of K/2 bytes (W4A4) or K bytes of int8 in
+ *    natural order (W4A8).  Codes lie in [-7, 7] (INT4) or [-127, 127] (INT8).
  *  - Device pointers must be 16-byte aligned and leading dimensions must make
  *    every row start 16-byte aligned; otherwise SERQ_ERR_INVALID_ARG.
  */
@@ -147,7 +149,7 @@ serq_status serq_layer_get_packed(const serq_layer* layer, uint8_t* wq, uint8_t*
  *  X     DEVICE, M x K, dtype f32 or bf16, row stride ldx elements.
  *  Xq    DEVICE output: W4A4 -> M x K/2 bytes packed; W4A8 -> M x K int8.
  *  sx    DEVICE output float[M].
- * M >= 1, K <= 16384.  Asynchronous on `stream`.
+ * M >= 1.  Asynchronous on `stream`.
  */
 serq_status serq_quantize_act(const void* X, serq_dtype dtype, int M, int K, int ldx,
                               serq_mode mode, void* Xq, float* sx, void* stream);

@@ -149,27 +149,33 @@ def compensator(W_hat: np.ndarray, q_w: np.ndarray, s_w: np.ndarray, r: int) -> 
 
 
 # ---------------------------------------------------------------------------
-# Packing (storage format): two's-complement nibbles, even k in the low
-# nibble, rows of the N x K (output-channel major) weight / M x K activation.
+# Packing (storage format, not part of the method: the pages fix only that
+# codes are 4-bit).  Two's-complement nibbles; every run of 32 consecutive
+# codes of a row occupies 16 bytes, byte j holding code j of the run in its
+# low nibble and code j + 16 in its high nibble.  Rows are the N x K (output
+# channel major) weight / compensator and the M x K activations.
 # ---------------------------------------------------------------------------
 def pack_int4_rows(codes: np.ndarray) -> np.ndarray:
     c = np.asarray(codes, dtype=np.int16)
-    assert c.shape[-1] % 2 == 0
-    lo = (c[..., 0::2] & 0xF).astype(np.uint8)
-    hi = (c[..., 1::2] & 0xF).astype(np.uint8)
-    return (lo | (hi << 4)).astype(np.uint8)
+    L = c.shape[-1]
+    assert L % 32 == 0, "packed rows hold whole runs of 32 codes"
+    blk = c.reshape(c.shape[:-1] + (L // 32, 2, 16))
+    lo = (blk[..., 0, :] & 0xF).astype(np.uint8)
+    hi = (blk[..., 1, :] & 0xF).astype(np.uint8)
+    return (lo | (hi << 4)).reshape(c.shape[:-1] + (L // 2,)).astype(np.uint8)
 
 
 def unpack_int4_rows(packed: np.ndarray) -> np.ndarray:
     p = np.asarray(packed, dtype=np.uint8)
-    lo = (p & 0xF).astype(np.int16)
-    hi = (p >> 4).astype(np.int16)
+    B = p.shape[-1]
+    assert B % 16 == 0
+    blk = p.reshape(p.shape[:-1] + (B // 16, 16))
+    lo = (blk & 0xF).astype(np.int16)
+    hi = (blk >> 4).astype(np.int16)
     lo = np.where(lo >= 8, lo - 16, lo)
     hi = np.where(hi >= 8, hi - 16, hi)
-    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.int8)
-    out[..., 0::2] = lo
-    out[..., 1::2] = hi
-    return out
+    out = np.stack([lo, hi], axis=-2)            # (..., B/16, 2, 16)
+    return out.reshape(p.shape[:-1] + (B * 2,)).astype(np.int8)
 
 
 # ---------------------------------------------------------------------------

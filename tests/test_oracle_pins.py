@@ -27,15 +27,24 @@ def test_quantizer_golden(case):
     assert float(s[0]) == pytest.approx(case["scale"], rel=1e-7, abs=0)
 
 
-@pytest.mark.parametrize("case", GOLD["pack_int4"], ids=lambda c: c["why"])
-def test_pack_golden(case):
-    b = O.pack_int4_rows(np.array([case["codes"]], dtype=np.int8))
-    assert int(b[0, 0]) == case["byte"]
-    assert O.unpack_int4_rows(b)[0].tolist() == case["codes"]
+def test_pack_golden():
+    g = GOLD["pack_int4"]
+    codes = np.zeros((1, 32), np.int8)
+    for k, v in g["codes"].items():
+        codes[0, int(k)] = v
+    b = O.pack_int4_rows(codes)[0]
+    want = np.zeros(16, np.uint8)
+    for k, v in g["bytes"].items():
+        want[int(k)] = v
+    assert b.tolist() == want.tolist()
+    assert O.unpack_int4_rows(b[None])[0].tolist() == codes[0].tolist()
 
 
 def test_pack_roundtrip_all_codes():
-    codes = np.array([[a, b] for a in range(-8, 8) for b in range(-8, 8)], dtype=np.int8)
+    rng = np.random.default_rng(0)
+    codes = rng.integers(-8, 8, size=(7, 96)).astype(np.int8)
+    codes[0, :16] = np.arange(-8, 8)
+    codes[0, 16:32] = np.arange(7, -9, -1)
     assert np.array_equal(O.unpack_int4_rows(O.pack_int4_rows(codes)), codes)
 
 

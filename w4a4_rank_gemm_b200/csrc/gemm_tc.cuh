@@ -50,36 +50,43 @@ struct Args {
   int32_t* acc1;
 };
 
+// Shared memory: PS packed stages [A | B] written by TMA, US unpacked
+// stages [A | B] read by the MMAs (W4A8: A is consumed straight from the
+// packed stage, already in the MMA layout), per-column scales, barriers.
 template <int BN, bool A8>
 struct Layout {
-  static constexpr int kUnA = BM * BK;                    // unpacked A tile (int8)
-  static constexpr int kUnB = BN * BK;                    // unpacked B tile (int8)
-  static constexpr int kPkA = A8 ? BM * BK : BM * BK / 2; // TMA A tile
-  static constexpr int kPkB = BN * BK / 2;                // TMA B/R tile (packed)
-  static constexpr int oUnA = 0;
-  static constexpr int oUnB = oUnA + (A8 ? 0 : US * kUnA);
-  static constexpr int oPkA = oUnB + US * kUnB;
-  static constexpr int oPkB = oPkA + PS * kPkA;
-  static constexpr int oSw = oPkB + PS * kPkB;
+  static constexpr int kPkA = A8 ? BM * BK : BM * BK / 2;  // A part of a packed stage
+  static constexpr int kPkB = BN * BK / 2;                 // B/R part (packed INT4)
+  static constexpr int kPk = kPkA + kPkB;
+  static constexpr int kUnA = A8 ? 0 : BM * BK;            // A part of an unpacked stage
+  static constexpr int kUnB = BN * BK;
+  static constexpr int kUn = kUnA + kUnB;
+  static constexpr int oUn = 0;
+  static constexpr int oPk = oUn + US * kUn;
+  static constexpr int oSw = oPk + PS * kPk;
   static constexpr int oSr = oSw + BN * 4;
   static constexpr int oBar = oSr + BN * 4;
   static constexpr int nBar = 2 * PS + 2 * US + 2;
   static constexpr int oMisc = oBar + nBar * 8;
   static constexpr int kBytes = oMisc + 16;
-  static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-B alignment
-  static constexpr uint32_t kTxBytes = kPkA + kPkB;
+  static constexpr int kAlloc = kBytes + 1024;             // slack for 1024-B alignment
+  static constexpr uint32_t kTxBytes = kPk;
   static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
-  static_assert(oPkA % 1024 == 0 && kPkA % 1024 == 0, "A TMA tiles must stay 1024-aligned");
-  static_assert(oUnB % 1024 == 0 && kUnB % 1024 == 0, "B tiles must stay 1024-aligned");
+  // widening work: rows of 64 packed bytes per stage, four 16-byte pieces each
+  static constexpr int kRows = (A8 ? 0 : BM) + BN;
+  static constexpr int kPiecesPerThread = kRows * 4 / (kUnpackWarps * 32);
+  static_assert(kRows * 4 % (kUnpackWarps * 32) == 0, "pieces must divide evenly");
+  static_assert(kPk % 1024 == 0 && kUn % 1024 == 0 && oPk % 1024 == 0, "tiles must stay 1024-aligned");
 };
 
-// One 8-byte packed chunk (16 codes) -> 16 int8 (x16) at the swizzled
-// position of chunk c in row `row` of a 128-byte-row tile.
-__device__ __forceinline__ void unpack_chunk(const uint8_t* src_row, uint8_t* dst_tile, int row, int c) {
-  const uint2 p = *reinterpret_cast<const uint2*>(src_row + 8 * c);
-  const uint2 a = unpack8_x16(p.x);
-  const uint2 b = unpack8_x16(p.y);
-  *reinterpret_cast<uint4*>(dst_tile + row * 128 + ((c ^ (row & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+// Widens one 16-byte packed run (32 codes) into 32 int8 (x16) in natural k
+// order: byte j of the run holds code j low and code j + 16 high, so
+// (w << 4) & 0xF0F0F0F0 gives codes 4i..4i+3 of word i and w & 0xF0F0F0F0
+// gives codes 16+4i..16+4i+3.
+__device__ __forceinline__ void widen_run(const uint4 v, uint4& lo, uint4& hi) {
+  const uint32_t m = 0xF0F0F0F0u;
+  lo = make_uint4((v.x << 4) & m, (v.y << 4) & m, (v.z << 4) & m, (v.w << 4) & m);
+  hi = make_uint4(v.x & m, v.y & m, v.z & m, v.w & m);
 }
 
 template <int BN, bool A8, bool ACC_OUT>
@@ -148,16 +155,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
         const bool res = step >= p.nkb;
         const int j = res ? step - p.nkb : step;
-        tma_load_2d(smem + L::oPkA + s * L::kPkA, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
-        tma_load_2d(smem + L::oPkB + s * L::kPkB, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), n0);
+        uint8_t* stage = smem + L::oPk + s * L::kPk;
+        tma_load_2d(stage, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
+        tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), n0);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_i8(BM, BN);
-      const uint32_t a_base = smem_u32(smem + (A8 ? L::oPkA : L::oUnA));
-      const uint32_t b_base = smem_u32(smem + L::oUnB);
+      const uint32_t pk_base = smem_u32(smem + L::oPk);
+      const uint32_t un_base = smem_u32(smem + L::oUn);
       bool ok = true;
       for (int step = 0; step < nsteps && ok; ++step) {
         const int u = step % US;
@@ -171,8 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = res ? step - p.nkb : step;
         const int nk = res ? min(BK / 32, (p.rpad - j * BK) / 32) : BK / 32;
         const uint32_t d = tmem + (res ? (uint32_t)BN : 0u);
-        const uint32_t a_tile = a_base + (A8 ? s * L::kPkA : u * L::kUnA);
-        const uint32_t b_tile = b_base + u * L::kUnB;
+        const uint32_t a_tile = A8 ? pk_base + s * L::kPk : un_base + u * L::kUn;
+        const uint32_t b_tile = un_base + u * L::kUn + L::kUnA;
         for (int kk = 0; kk < nk; ++kk) {
           umma_i8(d, umma_desc_k_sw128(a_tile + kk * 32), umma_desc_k_sw128(b_tile + kk * 32), idesc,
                   (j > 0 || kk > 0) ? 1u : 0u);
@@ -189,9 +197,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ unpack
+    // Thread ut widens the same rows and pieces in every stage: piece
+    // p = ut + 256 i covers row p / 4 (A rows first, then B rows) and packed
+    // bytes [16 (p % 4), +16); its 32 int8 land in chunks 2 (p % 4) and
+    // 2 (p % 4) + 1 of the 128-byte row, swizzled by row % 8.  Four
+    // consecutive threads cover one row, so a warp reads 512 contiguous
+    // bytes and each quarter-warp store fills all 32 banks.
     const int ut = threadIdx.x - 64;  // 0 .. 255
-    constexpr int kRows = (A8 ? 0 : BM) + BN;
-    constexpr int kChunks = kRows * 8;
+    constexpr int NP = L::kPiecesPerThread;
+    uint32_t src_off[NP], dst_off[NP];
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const int pc = ut + i * kUnpackWarps * 32;
+      const int row = pc >> 2, q = pc & 3;
+      src_off[i] = (A8 ? L::kPkA : 0) + row * (BK / 2) + q * 16;
+      dst_off[i] = row * BK + (((2 * q) ^ (row & 7)) << 4);
+    }
     bool ok = true;
     for (int step = 0; step < nsteps; ++step) {
       const int s = step % PS;
@@ -200,19 +221,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t uph = (step / US) & 1;
       if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
       if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
-      const uint8_t* pkA = smem + L::oPkA + s * L::kPkA;
-      const uint8_t* pkB = smem + L::oPkB + s * L::kPkB;
-      uint8_t* unA = smem + L::oUnA + u * L::kUnA;
-      uint8_t* unB = smem + L::oUnB + u * L::kUnB;
-#pragma unroll 4
-      for (int id = ut; id < kChunks; id += kUnpackWarps * 32) {
-        const int row = id >> 3, c = id & 7;
-        if (!A8 && row < BM) {
-          unpack_chunk(pkA + row * (BK / 2), unA, row, c);
-        } else {
-          const int rb = A8 ? row : row - BM;
-          unpack_chunk(pkB + rb * (BK / 2), unB, rb, c);
-        }
+      const uint8_t* pk = smem + L::oPk + s * L::kPk;
+      uint8_t* un = smem + L::oUn + u * L::kUn;
+      uint4 v[NP];
+#pragma unroll
+      for (int i = 0; i < NP; ++i) v[i] = *reinterpret_cast<const uint4*>(pk + src_off[i]);
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        uint4 lo, hi;
+        widen_run(v[i], lo, hi);
+        *reinterpret_cast<uint4*>(un + dst_off[i]) = lo;
+        *reinterpret_cast<uint4*>(un + (dst_off[i] ^ 16u)) = hi;
       }
       fence_proxy_async_smem();
       __syncwarp();

@@ -12,11 +12,12 @@
 // channels).  The 8 warps' partial sums are reduced in shared memory and the
 // epilogue applies sx * (sw * acc0 + sR * acc1).
 //
-// k-order inside a segment: thread t of a quad covers k in
-// [128 seg + 32 t, +32); MMA step s takes its 4th word: the low nibbles
-// (k = base + 8s + {0,2,4,6}) as the first K-half fragment and the high
-// nibbles (+1) as the second.  Activations use the identical mapping, so
-// every product pairs equal k.
+// k-order inside a segment: thread t of a quad covers the 32-code run
+// k in [128 seg + 32 t, +32).  MMA step s takes word s of the run's 16
+// packed bytes: its low nibbles (k = base + 4s + {0..3}) form the first
+// K-half fragment and its high nibbles (k = base + 16 + 4s + {0..3}) the
+// second.  Activations use the identical mapping, so every product pairs
+// equal k.
 #pragma once
 #include "common.cuh"
 
@@ -105,15 +106,12 @@ __device__ __forceinline__ void mma_seg(const Seg<MT, A8>& s, bool with_r, int (
     for (int mt = 0; mt < MT; ++mt) {
       uint32_t a0, a1, a2, a3;
       if (A8) {
-        // int8 codes k = base + 8 st .. +7: even bytes -> first half, odd -> second
-        const uint4& p0 = s.a[mt][0][st >> 1];
-        const uint4& p1 = s.a[mt][1][st >> 1];
-        const uint32_t x0 = (st & 1) ? p0.z : p0.x, x1 = (st & 1) ? p0.w : p0.y;
-        const uint32_t y0 = (st & 1) ? p1.z : p1.x, y1 = (st & 1) ? p1.w : p1.y;
-        a0 = __byte_perm(x0, x1, 0x6420);
-        a2 = __byte_perm(x0, x1, 0x7531);
-        a1 = __byte_perm(y0, y1, 0x6420);
-        a3 = __byte_perm(y0, y1, 0x7531);
+        // int8 codes: word st of the first 16 bytes is k = base + 4 st + {0..3},
+        // word st of the second 16 bytes is k = base + 16 + 4 st + {0..3}
+        a0 = (&s.a[mt][0][0].x)[st];
+        a2 = (&s.a[mt][0][A8 ? 1 : 0].x)[st];
+        a1 = (&s.a[mt][1][0].x)[st];
+        a3 = (&s.a[mt][1][A8 ? 1 : 0].x)[st];
       } else {
         const uint32_t x = (&s.a[mt][0][0].x)[st];
         const uint32_t y = (&s.a[mt][1][0].x)[st];

@@ -125,21 +125,32 @@ __device__ __forceinline__ int code4(float v, float amax) {
   return max(-7, min(7, q));
 }
 
-// Quantize W^ per output channel and pack: wq[n, k/2] (N x K/2 bytes).  One
-// thread packs 8 consecutive k of one column into 4 bytes.
+// Packed storage: every run of 32 codes of a row is 16 bytes; byte j holds
+// code j (low nibble) and code j + 16 (high nibble), two's complement.  The
+// tensor-core kernels widen such a run to 32 int8 in natural order with three
+// logic ops per 4 bytes.
+__device__ __forceinline__ uint4 pack_run32(const int (&q)[32]) {
+  uint32_t w[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t b = (uint32_t)(q[j] & 0xF) | ((uint32_t)(q[j + 16] & 0xF) << 4);
+    w[j >> 2] |= b << (8 * (j & 3));
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Quantize W^ per output channel and pack into wq (N x K/2 bytes).  One
+// thread packs one 32-code run of one output channel.
 __global__ void k_quant_pack_w(WeightView w, const float* __restrict__ s, const int32_t* __restrict__ perm,
                                int K, const float* __restrict__ amax_col, uint8_t* __restrict__ wq) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  const int i0 = blockIdx.y * 8;
+  const int i0 = blockIdx.y * 32;
   if (n >= w.N || i0 >= K) return;
   const float amax = amax_col[n];
-  uint32_t word = 0;
+  int q[32];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const int q = code4(w_hat(w, s, perm, i0 + t, n), amax);
-    word |= (uint32_t)(q & 0xF) << (4 * t);
-  }
-  *reinterpret_cast<uint32_t*>(wq + (size_t)n * (K / 2) + i0 / 2) = word;
+  for (int t = 0; t < 32; ++t) q[t] = code4(w_hat(w, s, perm, i0 + t, n), amax);
+  *reinterpret_cast<uint4*>(wq + (size_t)n * (K / 2) + i0 / 2) = pack_run32(q);
 }
 
 // R[i, n] = W^[i, n] - code(W^[i, n]) * sw[n], sw = amax_col / 7 (the main
@@ -162,24 +173,23 @@ __global__ void k_colmax_resid(WeightView w, const float* __restrict__ s, const 
   amax_r[n] = m;
 }
 
-// Quantize R per output channel and pack into rq[n, k/2] (N x rpad/2 bytes,
-// zero past r).
+// Quantize R per output channel and pack into rq (N x rpad/2 bytes, codes
+// past r are zero).  One thread per 32-code run.
 __global__ void k_quant_pack_r(WeightView w, const float* __restrict__ s, const int32_t* __restrict__ perm,
                                int r, int rpad, const float* __restrict__ amax_col,
                                const float* __restrict__ amax_r, uint8_t* __restrict__ rq) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  const int i0 = blockIdx.y * 8;
+  const int i0 = blockIdx.y * 32;
   if (n >= w.N || i0 >= rpad) return;
   const float a = amax_col[n];
   const float ar = amax_r[n];
-  uint32_t word = 0;
+  int q[32];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
+  for (int t = 0; t < 32; ++t) {
     const int i = i0 + t;
-    const int q = (i < r) ? code4(resid(w, s, perm, i, n, a), ar) : 0;
-    word |= (uint32_t)(q & 0xF) << (4 * t);
+    q[t] = (i < r) ? code4(resid(w, s, perm, i, n, a), ar) : 0;
   }
-  *reinterpret_cast<uint32_t*>(rq + (size_t)n * (rpad / 2) + i0 / 2) = word;
+  *reinterpret_cast<uint4*>(rq + (size_t)n * (rpad / 2) + i0 / 2) = pack_run32(q);
 }
 
 // sw = amax_col / 7, sR = amax_r / 7 (in place)

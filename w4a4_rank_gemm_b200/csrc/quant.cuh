@@ -2,17 +2,14 @@
 // fused SiLU*mul + quantize of a folded MLP block, and the runtime
 // flatten-and-permute helper for layers whose producer was not folded.
 //
-// One CTA per token row.  The row is held in registers between the absmax
-// reduction and the quantization, so HBM sees one read of X and one write of
-// the codes.  Arithmetic is fp32 with one rounding per operation.
+// Arithmetic is fp32 with one rounding per operation, so the codes are
+// reproducible bit for bit.
 #pragma once
 #include "common.cuh"
 
 namespace serq {
 namespace quant {
 
-constexpr int kMaxThreads = 256;
-constexpr int kMaxChunks = 8;  // 8-element chunks held per thread (K <= 16384)
 
 // ------------------------------------------------------------- row loaders
 // Each loader returns 8 consecutive fp32 values of row m starting at k0.
@@ -83,82 +80,77 @@ struct LoadSiluMul {
 };
 
 // ------------------------------------------------------- quantize one row
-// Q = 7 (packed INT4 output, K/2 bytes per row) or 127 (int8, K bytes).
-template <int Q, int CH, class Loader>
-__global__ void __launch_bounds__(kMaxThreads) k_quant_rows(Loader load, int K, uint8_t* __restrict__ Xq,
-                                                           float* __restrict__ sx) {
-  const int m = blockIdx.x;
-  const int nchunks = K >> 3;
-  float v[CH][8];
+// One warp per token row, two passes: the first reads the row for its
+// absolute maximum, the second reads it again (from L2, the row was just
+// streamed) and writes the codes.  HBM sees X once; many rows are in flight
+// per SM, so the loads of different rows overlap.
+//
+// Output, Q = 7: the packed INT4 format, every run of 32 codes is 16 bytes
+// with byte j = code j (low nibble) | code j+16 (high nibble).  Q = 127: int8
+// codes in natural order.
+constexpr int kRowsPerCta = 8;
+
+template <int Q, class Loader>
+__global__ void __launch_bounds__(kRowsPerCta * 32) k_quant_rows(Loader load, int M, int K, uint8_t* __restrict__ Xq,
+                                                                float* __restrict__ sx) {
+  const int m = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  const int nrun = K >> 5;  // runs of 32
+
   float amax = 0.f;
+  for (int b = lane; b < nrun; b += 32) {
 #pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int ch = threadIdx.x + c * blockDim.x;
-    if (ch < nchunks) {
-      load(m, ch * 8, v[c]);
+    for (int c = 0; c < 4; ++c) {
+      float v[8];
+      load(m, b * 32 + c * 8, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[c][i]));
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
     }
   }
+#pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  __shared__ float red[kMaxThreads / 32];
-  const int nw = blockDim.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-  __syncthreads();
-  amax = red[0];
-  for (int i = 1; i < nw; ++i) amax = fmaxf(amax, red[i]);
 
   const float qf = (float)Q;
   const float inv = (amax > 0.f) ? __fdiv_rn(qf, amax) : 0.f;
-  if (threadIdx.x == 0) sx[m] = __fdiv_rn(amax, qf);
+  if (lane == 0) sx[m] = __fdiv_rn(amax, qf);
+
+  for (int b = lane; b < nrun; b += 32) {
+    int q[32];
 #pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int ch = threadIdx.x + c * blockDim.x;
-    if (ch < nchunks) {
-      int q[8];
+    for (int c = 0; c < 4; ++c) {
+      float v[8];
+      load(m, b * 32 + c * 8, v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int t = __float2int_rn(__fmul_rn(v[c][i], inv));
-        q[i] = max(-Q, min(Q, t));
+        const int t = __float2int_rn(__fmul_rn(v[i], inv));
+        q[c * 8 + i] = max(-Q, min(Q, t));
       }
-      if (Q == 7) {
-        uint32_t w = 0;
+    }
+    if (Q == 7) {
+      uint32_t w[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w |= (uint32_t)(q[i] & 0xF) << (4 * i);
-        *reinterpret_cast<uint32_t*>(Xq + (size_t)m * (K >> 1) + ch * 4) = w;
-      } else {
-        uint32_t lo = 0, hi = 0;
+      for (int j = 0; j < 16; ++j)
+        w[j >> 2] |= ((uint32_t)(q[j] & 0xF) | ((uint32_t)(q[j + 16] & 0xF) << 4)) << (8 * (j & 3));
+      *reinterpret_cast<uint4*>(Xq + (size_t)m * (K >> 1) + b * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      uint32_t w[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          lo |= (uint32_t)(q[i] & 0xFF) << (8 * i);
-          hi |= (uint32_t)(q[i + 4] & 0xFF) << (8 * i);
-        }
-        *reinterpret_cast<uint2*>(Xq + (size_t)m * K + ch * 8) = make_uint2(lo, hi);
-      }
+      for (int j = 0; j < 8; ++j)
+        w[j] = (uint32_t)(q[4 * j] & 0xFF) | ((uint32_t)(q[4 * j + 1] & 0xFF) << 8) |
+               ((uint32_t)(q[4 * j + 2] & 0xFF) << 16) | ((uint32_t)(q[4 * j + 3] & 0xFF) << 24);
+      uint4* dst = reinterpret_cast<uint4*>(Xq + (size_t)m * K + b * 32);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
   }
 }
 
-// Launch helper: block size = min(256, chunks rounded up to a warp), CH =
-// chunks per thread (1, 2, 4 or 8).
 template <int Q, class Loader>
 inline cudaError_t launch_quant_rows(const Loader& load, int M, int K, uint8_t* Xq, float* sx,
                                      cudaStream_t st) {
-  const int nchunks = K / 8;
-  int threads = ((nchunks + 31) / 32) * 32;
-  if (threads > kMaxThreads) threads = kMaxThreads;
-  const int ch = (nchunks + threads - 1) / threads;
-  dim3 grid(M), block(threads);
-  if (ch <= 1)
-    k_quant_rows<Q, 1, Loader><<<grid, block, 0, st>>>(load, K, Xq, sx);
-  else if (ch <= 2)
-    k_quant_rows<Q, 2, Loader><<<grid, block, 0, st>>>(load, K, Xq, sx);
-  else if (ch <= 4)
-    k_quant_rows<Q, 4, Loader><<<grid, block, 0, st>>>(load, K, Xq, sx);
-  else if (ch <= kMaxChunks)
-    k_quant_rows<Q, 8, Loader><<<grid, block, 0, st>>>(load, K, Xq, sx);
-  else
-    return cudaErrorInvalidValue;
+  const int ctas = (M + kRowsPerCta - 1) / kRowsPerCta;
+  k_quant_rows<Q, Loader><<<ctas, kRowsPerCta * 32, 0, st>>>(load, M, K, Xq, sx);
   return cudaGetLastError();
 }
 

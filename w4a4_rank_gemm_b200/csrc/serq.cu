@@ -379,10 +379,10 @@ serq_status serq_prepare_group(int n_weights, const float* const* W, const int* 
     cudaMemsetAsync(Li->sw, 0, sizeof(float) * Ni, st);
     k_colmax_what<<<dim3((Ni + 255) / 256, (K + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(
         v, L0->smooth, L0->perm, K, rows_per_block, Li->sw);
-    k_quant_pack_w<<<dim3((Ni + 127) / 128, K / 8), 128, 0, st>>>(v, L0->smooth, L0->perm, K, Li->sw, Li->wq);
+    k_quant_pack_w<<<dim3((Ni + 127) / 128, K / 32), 128, 0, st>>>(v, L0->smooth, L0->perm, K, Li->sw, Li->wq);
     if (rank > 0) {
       k_colmax_resid<<<(Ni + 127) / 128, 128, 0, st>>>(v, L0->smooth, L0->perm, rank, Li->sw, Li->sr);
-      k_quant_pack_r<<<dim3((Ni + 127) / 128, Li->rpad / 8), 128, 0, st>>>(v, L0->smooth, L0->perm, rank,
+      k_quant_pack_r<<<dim3((Ni + 127) / 128, Li->rpad / 32), 128, 0, st>>>(v, L0->smooth, L0->perm, rank,
                                                                           Li->rpad, Li->sw, Li->sr, Li->rq);
     }
     k_finalize_scales<<<(Ni + 255) / 256, 256, 0, st>>>(Li->sw, Li->sr, Ni, rank > 0);
@@ -447,7 +447,6 @@ serq_status serq_quantize_act(const void* X, serq_dtype dtype, int M, int K, int
   serq_status s;
   if (dtype != SERQ_F32 && dtype != SERQ_BF16) return fail(SERQ_ERR_INVALID_ARG, "bad dtype");
   if ((s = check_rows(X, M, K, ldx, dtype == SERQ_F32 ? 4 : 2, "X"))) return s;
-  if (K > 16384) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "quantize takes K <= 16384 (got %d)", K);
   if (!Xq || !sx) return fail(SERQ_ERR_INVALID_ARG, "null Xq or sx");
   if (!aligned16(Xq)) return fail(SERQ_ERR_INVALID_ARG, "Xq must be 16-byte aligned");
   if (mode != SERQ_W4A4 && mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode");
@@ -472,7 +471,6 @@ serq_status serq_silu_mul_quantize(const void* G, const void* U, int M, int F, i
   serq_status s;
   if ((s = check_rows(G, M, F, ld, 2, "G"))) return s;
   if ((s = check_rows(U, M, F, ld, 2, "U"))) return s;
-  if (F > 16384) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "quantize takes K <= 16384 (got %d)", F);
   if (!Xq || !sx) return fail(SERQ_ERR_INVALID_ARG, "null Xq or sx");
   if (!aligned16(Xq)) return fail(SERQ_ERR_INVALID_ARG, "Xq must be 16-byte aligned");
   if (mode != SERQ_W4A4 && mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode");
