@@ -149,7 +149,7 @@ serq_status serq_layer_get_packed(const serq_layer* layer, uint8_t* wq, uint8_t*
  *  X     DEVICE, M x K, dtype f32 or bf16, row stride ldx elements.
  *  Xq    DEVICE output: W4A4 -> M x K/2 bytes packed; W4A8 -> M x K int8.
  *  sx    DEVICE output float[M].
- * M >= 1.  Asynchronous on `stream`.
+ * M >= 1; K <= 32768 (bf16) or 16384 (fp32).  Asynchronous on `stream`.
  */
 serq_status serq_quantize_act(const void* X, serq_dtype dtype, int M, int K, int ldx,
                               serq_mode mode, void* Xq, float* sx, void* stream);
@@ -187,7 +187,7 @@ serq_status serq_linear_accum(const serq_layer* layer, const void* Xq, int M, in
  * as serq_quantize_act.  G and U arrive already in down_proj's saliency order
  * with U already divided by down_proj's smoothing scales (key design 3), so h
  * is down_proj's X^.
- *  G, U  DEVICE bf16, M x F, row stride ld elements.
+ *  G, U  DEVICE bf16, M x F (F <= 16384), row stride ld elements.
  *  Xq, sx as serq_quantize_act with K = F.
  */
 serq_status serq_silu_mul_quantize(const void* G, const void* U, int M, int F, int ld,

@@ -58,6 +58,8 @@ def test_host_side_argument_rejection(lib):
     assert L.serq_quantize_act(fake, lib.BF16, 4, 100, 128, lib.W4A4, fake, fake, None) == lib.ERR_UNSUPPORTED_SHAPE
     # misaligned row stride
     assert L.serq_quantize_act(fake, lib.BF16, 4, 256, 260, lib.W4A4, fake, fake, None) == lib.ERR_INVALID_ARG
+    # K beyond what the quantizer holds in registers
+    assert L.serq_quantize_act(fake, lib.BF16, 4, 65536, 65536, lib.W4A4, fake, fake, None) == lib.ERR_UNSUPPORTED_SHAPE
     # prepare: rank > K and bad N
     W = (ctypes.c_void_p * 1)(0x1000)
     N = (ctypes.c_int * 1)(256)

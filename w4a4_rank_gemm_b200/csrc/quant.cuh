@@ -12,12 +12,17 @@ namespace quant {
 
 
 // ------------------------------------------------------------- row loaders
-// Each loader returns 8 consecutive fp32 values of row m starting at k0.
+// A loader fetches the raw bytes of 8 consecutive elements of row m at k0
+// (`load`) and turns them into fp32 (`value`).  The raw form is what the
+// quantizer keeps in registers between its two uses of the row.
 struct LoadBF16 {
+  static constexpr int kWords = 1;  // uint4 per 8 elements
   const __nv_bfloat16* X;
   int ld;
-  __device__ __forceinline__ void operator()(int m, int k0, float (&v)[8]) const {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * ld + k0));
+  __device__ __forceinline__ void load(int m, int k0, uint4 (&r)[kWords]) const {
+    r[0] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * ld + k0));
+  }
+  __device__ __forceinline__ static void bf16x8(const uint4& u, float (&v)[8]) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -25,16 +30,23 @@ struct LoadBF16 {
       v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   }
+  __device__ __forceinline__ void value(const uint4 (&r)[kWords], float (&v)[8]) const { bf16x8(r[0], v); }
 };
 
 struct LoadF32 {
+  static constexpr int kWords = 2;
   const float* X;
   int ld;
-  __device__ __forceinline__ void operator()(int m, int k0, float (&v)[8]) const {
-    const float4* p = reinterpret_cast<const float4*>(X + (size_t)m * ld + k0);
-    const float4 a = __ldg(p), b = __ldg(p + 1);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  __device__ __forceinline__ void load(int m, int k0, uint4 (&r)[kWords]) const {
+    const uint4* p = reinterpret_cast<const uint4*>(X + (size_t)m * ld + k0);
+    r[0] = __ldg(p);
+    r[1] = __ldg(p + 1);
+  }
+  __device__ __forceinline__ void value(const uint4 (&r)[kWords], float (&v)[8]) const {
+    v[0] = __uint_as_float(r[0].x); v[1] = __uint_as_float(r[0].y);
+    v[2] = __uint_as_float(r[0].z); v[3] = __uint_as_float(r[0].w);
+    v[4] = __uint_as_float(r[1].x); v[5] = __uint_as_float(r[1].y);
+    v[6] = __uint_as_float(r[1].z); v[7] = __uint_as_float(r[1].w);
   }
 };
 
@@ -64,13 +76,18 @@ __device__ __forceinline__ float exp_cw(float x) {
 
 // h = silu(g) * u = g / (1 + e^-g) * u, fp32.
 struct LoadSiluMul {
+  static constexpr int kWords = 2;
   const __nv_bfloat16* G;
   const __nv_bfloat16* U;
   int ld;
-  __device__ __forceinline__ void operator()(int m, int k0, float (&v)[8]) const {
+  __device__ __forceinline__ void load(int m, int k0, uint4 (&r)[kWords]) const {
+    r[0] = __ldg(reinterpret_cast<const uint4*>(G + (size_t)m * ld + k0));
+    r[1] = __ldg(reinterpret_cast<const uint4*>(U + (size_t)m * ld + k0));
+  }
+  __device__ __forceinline__ void value(const uint4 (&r)[kWords], float (&v)[8]) const {
     float g[8], u[8];
-    LoadBF16{G, ld}(m, k0, g);
-    LoadBF16{U, ld}(m, k0, u);
+    LoadBF16::bf16x8(r[0], g);
+    LoadBF16::bf16x8(r[1], u);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float den = __fadd_rn(1.f, exp_cw(-g[i]));
@@ -80,51 +97,71 @@ struct LoadSiluMul {
 };
 
 // ------------------------------------------------------- quantize one row
-// One warp per token row, two passes: the first reads the row for its
-// absolute maximum, the second reads it again (from L2, the row was just
-// streamed) and writes the codes.  HBM sees X once; many rows are in flight
-// per SM, so the loads of different rows overlap.
+// One CTA per token row; lane l of warp w owns the 32-code runs
+// b = l + 32 (w + W i), i < RPL, and holds their raw input in registers, so
+// HBM sees the row once: load everything, reduce the absolute maximum
+// (shuffles, then shared memory across the W warps), quantize from registers.
 //
 // Output, Q = 7: the packed INT4 format, every run of 32 codes is 16 bytes
 // with byte j = code j (low nibble) | code j+16 (high nibble).  Q = 127: int8
 // codes in natural order.
-constexpr int kRowsPerCta = 8;
-
-template <int Q, class Loader>
-__global__ void __launch_bounds__(kRowsPerCta * 32) k_quant_rows(Loader load, int M, int K, uint8_t* __restrict__ Xq,
-                                                                float* __restrict__ sx) {
-  const int m = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (m >= M) return;
-  const int nrun = K >> 5;  // runs of 32
-
+template <int Q, int RPL, class Loader>
+__global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* __restrict__ Xq,
+                                                    float* __restrict__ sx) {
+  constexpr int W = Loader::kWords;
+  const int m = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int nrun = K >> 5;
+  uint4 raw[RPL][4][W];
   float amax = 0.f;
-  for (int b = lane; b < nrun; b += 32) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float v[8];
-      load(m, b * 32 + c * 8, v);
+  for (int i = 0; i < RPL; ++i) {
+    const int b = lane + 32 * (warp + nw * i);
+    if (b < nrun) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      for (int c = 0; c < 4; ++c) ld.load(m, b * 32 + c * 8, raw[i][c]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RPL; ++i) {
+    const int b = lane + 32 * (warp + nw * i);
+    if (b < nrun) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[8];
+        ld.value(raw[i][c], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+      }
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (nw > 1) {
+    __shared__ float red[8];
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = red[0];
+    for (int i = 1; i < nw; ++i) amax = fmaxf(amax, red[i]);
+  }
 
   const float qf = (float)Q;
   const float inv = (amax > 0.f) ? __fdiv_rn(qf, amax) : 0.f;
-  if (lane == 0) sx[m] = __fdiv_rn(amax, qf);
+  if (threadIdx.x == 0) sx[m] = __fdiv_rn(amax, qf);
 
-  for (int b = lane; b < nrun; b += 32) {
+#pragma unroll
+  for (int i = 0; i < RPL; ++i) {
+    const int b = lane + 32 * (warp + nw * i);
+    if (b >= nrun) continue;
     int q[32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float v[8];
-      load(m, b * 32 + c * 8, v);
+      ld.value(raw[i][c], v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = __float2int_rn(__fmul_rn(v[i], inv));
-        q[c * 8 + i] = max(-Q, min(Q, t));
+      for (int e = 0; e < 8; ++e) {
+        const int t = __float2int_rn(__fmul_rn(v[e], inv));
+        q[c * 8 + e] = max(-Q, min(Q, t));
       }
     }
     if (Q == 7) {
@@ -146,11 +183,16 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) k_quant_rows(Loader load, in
   }
 }
 
+// Runs per lane held in registers: 4 for bf16 input (64 registers of raw
+// data), 2 for fp32 or the two bf16 inputs of silu*mul.  Warps per row =
+// ceil(runs / (32 * RPL)) <= 8, so K <= 32768 (bf16) / 16384.
 template <int Q, class Loader>
-inline cudaError_t launch_quant_rows(const Loader& load, int M, int K, uint8_t* Xq, float* sx,
-                                     cudaStream_t st) {
-  const int ctas = (M + kRowsPerCta - 1) / kRowsPerCta;
-  k_quant_rows<Q, Loader><<<ctas, kRowsPerCta * 32, 0, st>>>(load, M, K, Xq, sx);
+inline cudaError_t launch_quant_rows(const Loader& ld, int M, int K, uint8_t* Xq, float* sx, cudaStream_t st) {
+  constexpr int RPL = (Loader::kWords == 1) ? 4 : 2;
+  const int nrun = K / 32;
+  const int warps = (nrun + 32 * RPL - 1) / (32 * RPL);
+  if (warps > 8) return cudaErrorInvalidValue;
+  k_quant_rows<Q, RPL, Loader><<<M, warps * 32, 0, st>>>(ld, K, Xq, sx);
   return cudaGetLastError();
 }
 

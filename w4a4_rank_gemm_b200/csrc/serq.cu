@@ -275,7 +275,7 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
 
 serq_status check_rows(const void* X, int M, int K, int ld, int elem, const char* name) {
   if (!X) return fail(SERQ_ERR_INVALID_ARG, "null %s", name);
-  if (M < 1 || M > 2147483647 / 2) return fail(SERQ_ERR_INVALID_ARG, "M = %d out of range", M);
+  if (M < 1 || M > 2147483647) return fail(SERQ_ERR_INVALID_ARG, "M = %d out of range", M);
   if (K < 32 || K % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "K = %d must be a positive multiple of 32", K);
   if (ld < K) return fail(SERQ_ERR_INVALID_ARG, "leading dimension of %s (%d) < K (%d)", name, ld, K);
   if (!aligned16(X) || ((size_t)ld * elem) % 16)
@@ -447,6 +447,9 @@ serq_status serq_quantize_act(const void* X, serq_dtype dtype, int M, int K, int
   serq_status s;
   if (dtype != SERQ_F32 && dtype != SERQ_BF16) return fail(SERQ_ERR_INVALID_ARG, "bad dtype");
   if ((s = check_rows(X, M, K, ldx, dtype == SERQ_F32 ? 4 : 2, "X"))) return s;
+  if (K > (dtype == SERQ_F32 ? 16384 : 32768))
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "quantize takes K <= %d for this dtype (got %d)",
+                dtype == SERQ_F32 ? 16384 : 32768, K);
   if (!Xq || !sx) return fail(SERQ_ERR_INVALID_ARG, "null Xq or sx");
   if (!aligned16(Xq)) return fail(SERQ_ERR_INVALID_ARG, "Xq must be 16-byte aligned");
   if (mode != SERQ_W4A4 && mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode");
@@ -471,6 +474,7 @@ serq_status serq_silu_mul_quantize(const void* G, const void* U, int M, int F, i
   serq_status s;
   if ((s = check_rows(G, M, F, ld, 2, "G"))) return s;
   if ((s = check_rows(U, M, F, ld, 2, "U"))) return s;
+  if (F > 16384) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "silu_mul_quantize takes F <= 16384 (got %d)", F);
   if (!Xq || !sx) return fail(SERQ_ERR_INVALID_ARG, "null Xq or sx");
   if (!aligned16(Xq)) return fail(SERQ_ERR_INVALID_ARG, "Xq must be 16-byte aligned");
   if (mode != SERQ_W4A4 && mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode");
