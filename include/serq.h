@@ -62,8 +62,10 @@ typedef enum {
   SERQ_ALGO_PREFILL = 1,       /* tcgen05 kind::i8 GEMM, TMEM accumulators; the
                                   output tile width is chosen from the shape  */
   SERQ_ALGO_DECODE = 2,        /* memory-bound split-K tensor-core GEMV, M <= 64 */
-  SERQ_ALGO_PREFILL_N128 = 3,  /* PREFILL with 128 x 128 output tiles          */
-  SERQ_ALGO_PREFILL_N256 = 4   /* PREFILL with 128 x 256 output tiles          */
+  SERQ_ALGO_PREFILL_N128 = 3,  /* PREFILL with 128 x 128 output tiles, one CTA  */
+  SERQ_ALGO_PREFILL_N256 = 4,  /* PREFILL with 128 x 256 output tiles, one CTA  */
+  SERQ_ALGO_PREFILL_PAIR_N256 = 5 /* PREFILL with 256 x 256 tiles on a CTA pair
+                                     (tcgen05 cta_group::2)                     */
 } serq_algo;
 
 typedef struct serq_layer serq_layer;

@@ -145,7 +145,8 @@ def _linear_case(S, M, K, N, r, mode, act_dtype="bf16", seed=0):
 def test_linear_accum_bit_exact(S, mode, M, K, N, r):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, r, mode)
     acc0, acc1 = O.linear_accum(xq, ol)
-    algos = [S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256] + ([S.ALGO_DECODE] if M <= 64 else [])
+    algos = [S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
+        ([S.ALGO_DECODE] if M <= 64 else [])
     for algo in algos:
         g0, g1 = S.linear_accum(L, Xq, algo)
         torch.cuda.synchronize()
@@ -160,7 +161,8 @@ def test_linear_output_within_tolerance(S, mode, M, K, N, r):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, r, mode, seed=1)
     acc0, acc1 = O.linear_accum(xq, ol)
     y_ref = O.linear_epilogue(acc0, acc1, osx, ol)
-    algos = [S.ALGO_AUTO, S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256] + ([S.ALGO_DECODE] if M <= 64 else [])
+    algos = [S.ALGO_AUTO, S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
+        ([S.ALGO_DECODE] if M <= 64 else [])
     for algo in algos:
         Y = S.linear(L, Xq, sx, algo=algo)
         torch.cuda.synchronize()

@@ -4,12 +4,20 @@
 //   acc1 = Xq[:, :r] Rq^T     (the r salient columns; SERQ notes key design 2)
 //   Y    = sx * (sw * acc0 + sR * acc1)   -> bf16
 //
-// One CTA computes a 128 x BN output tile.  Warp roles:
+// CG = 1: one CTA computes a 128 x BN output tile.
+// CG = 2: a cluster of two CTAs computes a 256 x BN tile with
+//   tcgen05.mma.cta_group::2 (M = 256): each CTA holds its 128 rows of X and
+//   half (BN/2 rows) of W, and its 128 x BN slice of both accumulators in its
+//   own TMEM.  Each SM then stages and widens half the weight tile, and the
+//   tensor cores of both SMs share every weight byte they read from shared
+//   memory (no TMA multicast is involved: each CTA loads its own halves).
+//
+// Warp roles (per CTA):
 //   warp 0      TMA producer: packed INT4 tiles of X and W (or R) -> smem
-//   warp 1      TMEM owner + single-thread tcgen05.mma issuer
+//   warp 1      TMEM owner; in CTA 0 of the pair, one thread issues the MMAs
 //   warps 2..9  unpackers: packed nibbles -> int8 (x16) in the 128-byte
 //               swizzled K-major layout the MMA reads; afterwards the same
-//               warps run the epilogue out of TMEM.
+//               warps run the epilogue out of this CTA's TMEM.
 // The k loop runs K/128 main steps into acc0 followed by ceil(r/128)
 // residual steps into acc1; a residual step reloads the matching activation
 // block and takes R in place of W, so both accumulators use one pipeline.
@@ -19,9 +27,9 @@
 // INT4 has no tensor-core input kind of its own, and no FP4 kind represents
 // the codes -7..7 exactly, so the codes are widened to int8 in shared memory
 // and multiplied by kind::i8.  The widening keeps each nibble in the high
-// half of its byte (value x16), so it costs two logic ops per four codes;
-// the factor 16 per widened operand leaves the accumulator exactly and is
-// removed by a shift.
+// half of its byte (value x16), three logic ops per four codes; the factor
+// 16 per widened operand leaves the accumulator exactly and is removed by a
+// shift.
 //
 // W4A8: X arrives as int8 and is loaded by TMA straight into the swizzled
 // layout; only W / R are widened.
@@ -31,10 +39,8 @@
 namespace serq {
 namespace tc {
 
-constexpr int BM = 128;
+constexpr int BM = 128;            // rows of X per CTA
 constexpr int BK = 128;            // k per pipeline step (int8 bytes per row)
-constexpr int PS = 3;              // packed (TMA) stages
-constexpr int US = 2;              // unpacked stages
 constexpr int kUnpackWarps = 8;
 constexpr int kThreads = (2 + kUnpackWarps) * 32;
 
@@ -53,13 +59,16 @@ struct Args {
 // Shared memory: PS packed stages [A | B] written by TMA, US unpacked
 // stages [A | B] read by the MMAs (W4A8: A is consumed straight from the
 // packed stage, already in the MMA layout), per-column scales, barriers.
-template <int BN, bool A8>
+template <int BN, bool A8, int CG>
 struct Layout {
+  static constexpr int PS = (CG == 2) ? 4 : 3;             // packed (TMA) stages
+  static constexpr int US = (CG == 2) ? 3 : 2;             // unpacked stages
+  static constexpr int BNL = BN / CG;                      // weight rows held by this CTA
   static constexpr int kPkA = A8 ? BM * BK : BM * BK / 2;  // A part of a packed stage
-  static constexpr int kPkB = BN * BK / 2;                 // B/R part (packed INT4)
+  static constexpr int kPkB = BNL * BK / 2;                // B/R part (packed INT4)
   static constexpr int kPk = kPkA + kPkB;
   static constexpr int kUnA = A8 ? 0 : BM * BK;            // A part of an unpacked stage
-  static constexpr int kUnB = BN * BK;
+  static constexpr int kUnB = BNL * BK;
   static constexpr int kUn = kUnA + kUnB;
   static constexpr int oUn = 0;
   static constexpr int oPk = oUn + US * kUn;
@@ -73,10 +82,11 @@ struct Layout {
   static constexpr uint32_t kTxBytes = kPk;
   static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
   // widening work: rows of 64 packed bytes per stage, four 16-byte pieces each
-  static constexpr int kRows = (A8 ? 0 : BM) + BN;
+  static constexpr int kRows = (A8 ? 0 : BM) + BNL;
   static constexpr int kPiecesPerThread = kRows * 4 / (kUnpackWarps * 32);
   static_assert(kRows * 4 % (kUnpackWarps * 32) == 0, "pieces must divide evenly");
   static_assert(kPk % 1024 == 0 && kUn % 1024 == 0 && oPk % 1024 == 0, "tiles must stay 1024-aligned");
+  static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
 // Widens one 16-byte packed run (32 codes) into 32 int8 (x16) in natural k
@@ -89,17 +99,26 @@ __device__ __forceinline__ void widen_run(const uint4 v, uint4& lo, uint4& hi) {
   hi = make_uint4(v.x & m, v.y & m, v.z & m, v.w & m);
 }
 
-template <int BN, bool A8, bool ACC_OUT>
+template <int CG>
+__device__ __forceinline__ void cta_sync() {
+  if (CG == 1)
+    __syncthreads();
+  else
+    cluster_sync_all();
+}
+
+template <int BN, bool A8, bool ACC_OUT, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmR, const Args p) {
-  using L = Layout<BN, A8>;
+  using L = Layout<BN, A8, CG>;
+  constexpr int PS = L::PS, US = L::US;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::oBar);
   uint64_t* full_pk = bar;              // TMA bytes landed            (tx)
   uint64_t* empty_pk = bar + PS;        // packed stage consumed
-  uint64_t* full_un = bar + 2 * PS;     // unpacked stage written
+  uint64_t* full_un = bar + 2 * PS;     // unpacked stage written (both CTAs, on CTA 0)
   uint64_t* empty_un = full_un + US;    // unpacked stage read by the MMAs
   uint64_t* acc_full = empty_un + US;   // all MMAs complete
   uint64_t* drain = acc_full + 1;       // abort path: MMAs complete
@@ -109,7 +128,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sr_t = reinterpret_cast<float*>(smem + L::oSr);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
+  const int n0 = blockIdx.y * BN;                       // output columns of this tile
+  const int nb0 = n0 + (int)rank * L::BNL;              // weight rows this CTA loads
+  const int m0 = blockIdx.x * BM;                       // X rows of this CTA
   const int nsteps = p.nkb + p.nrb;
 
   if (threadIdx.x == 0) {
@@ -118,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty_pk[s], kUnpackWarps + (A8 ? 1 : 0));
     }
     for (int s = 0; s < US; ++s) {
-      mbar_init(&full_un[s], kUnpackWarps);
+      mbar_init(&full_un[s], kUnpackWarps * CG);
       mbar_init(&empty_un[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -132,8 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmR);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, L::kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<CG>(tmem_slot, L::kTmemCols);
+    tmem_relinquish<CG>();
   }
   for (int i = threadIdx.x; i < BN; i += blockDim.x) {
     const int n = n0 + i;
@@ -141,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sr_t[i] = (n < p.N) ? p.sr[n] : 0.f;
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync<CG>();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -157,13 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = res ? step - p.nkb : step;
         uint8_t* stage = smem + L::oPk + s * L::kPk;
         tma_load_2d(stage, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
-        tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), n0);
+        tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_i8(BM, BN);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = umma_idesc_i8(BM * CG, BN);
       const uint32_t pk_base = smem_u32(smem + L::oPk);
       const uint32_t un_base = smem_u32(smem + L::oUn);
       bool ok = true;
@@ -172,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t uph = (step / US) & 1;
         const int s = step % PS;
         const uint32_t ph = (step / PS) & 1;
-        if (!mbar_wait(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait<CG == 2>(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
         if (A8 && !mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
         const bool res = step >= p.nkb;
@@ -182,16 +205,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_tile = A8 ? pk_base + s * L::kPk : un_base + u * L::kUn;
         const uint32_t b_tile = un_base + u * L::kUn + L::kUnA;
         for (int kk = 0; kk < nk; ++kk) {
-          umma_i8(d, umma_desc_k_sw128(a_tile + kk * 32), umma_desc_k_sw128(b_tile + kk * 32), idesc,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+          umma_i8<CG>(d, umma_desc_k_sw128(a_tile + kk * 32), umma_desc_k_sw128(b_tile + kk * 32), idesc,
+                      (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&empty_un[u]);
-        if (A8) umma_commit(&empty_pk[s]);
+        umma_commit<CG>(&empty_un[u]);
+        if (A8) umma_commit<CG>(&empty_pk[s]);
       }
       if (ok) {
-        umma_commit(acc_full);
+        umma_commit<CG>(acc_full);
       } else {
-        umma_commit(drain);
+        umma_commit<1>(drain);
         mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
       }
     }
@@ -237,7 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&empty_pk[s]);
-        mbar_arrive(&full_un[u]);
+        if (leader)
+          mbar_arrive(&full_un[u]);
+        else
+          mbar_arrive_remote(&full_un[u], 0);
       }
     }
 
@@ -304,10 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (global_ns() - t0 < 100000ull) {
     }
   }
-  __syncthreads();
+  // Neither CTA of a pair leaves (or frees TMEM) while its peer may still
+  // touch its barriers or shared memory.
+  cta_sync<CG>();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, L::kTmemCols);
+    tmem_dealloc<CG>(tmem, L::kTmemCols);
   }
 }
 

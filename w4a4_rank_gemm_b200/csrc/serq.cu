@@ -182,17 +182,19 @@ void set_smem(K kernel, int bytes) {
 }
 
 // ------------------------------------------------------------ GEMM launch
-template <int BN, bool A8, bool ACC>
+template <int BN, bool A8, bool ACC, int CG>
 cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, cudaStream_t st) {
-  using Lay = serq::tc::Layout<BN, A8>;
+  using Lay = serq::tc::Layout<BN, A8, CG>;
   CUtensorMap tmA;
   bool okm = A8 ? make_map(&tmA, Xq, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, 128, 128,
                            CU_TENSOR_MAP_SWIZZLE_128B)
                 : make_map(&tmA, Xq, (uint64_t)a.K / 2, (uint64_t)a.M, (uint64_t)a.K / 2, 64, 128,
                            CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!okm) return cudaErrorInvalidValue;
-  const int bi = (BN == 256) ? 1 : 0;
-  auto kern = serq::tc::k_gemm<BN, A8, ACC>;
+  // weight maps by box rows: [0] 128, [1] 256 (BN / CG rows per CTA)
+  const int bi = (BN / CG == 256) ? 1 : 0;
+  static_assert(BN / CG == 128 || BN / CG == 256, "weight box rows");
+  auto kern = serq::tc::k_gemm<BN, A8, ACC, CG>;
   static int attr_set[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -200,9 +202,21 @@ cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args&
     set_smem(kern, Lay::kAlloc);
     attr_set[dev] = 1;
   }
-  dim3 grid((a.N + BN - 1) / BN, (a.M + serq::tc::BM - 1) / serq::tc::BM);
-  kern<<<grid, serq::tc::kThreads, Lay::kAlloc, st>>>(tmA, L->tmB[bi], L->tmR[bi], a);
-  return cudaGetLastError();
+  const int mtiles = (a.M + serq::tc::BM * CG - 1) / (serq::tc::BM * CG);
+  dim3 grid(mtiles * CG, (a.N + BN - 1) / BN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(serq::tc::kThreads);
+  cfg.dynamicSmemBytes = Lay::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[bi], L->tmR[bi], a);
 }
 
 int sm_count() {
@@ -219,12 +233,17 @@ int sm_count() {
 template <bool A8, bool ACC>
 cudaError_t dispatch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, serq_algo algo,
                         cudaStream_t st) {
-  if (algo == SERQ_ALGO_PREFILL_N128) return launch_tc<128, A8, ACC>(L, Xq, a, st);
-  if (algo == SERQ_ALGO_PREFILL_N256) return launch_tc<256, A8, ACC>(L, Xq, a, st);
-  // 256-wide tiles unless that leaves most SMs idle.
-  const long tiles256 = (long)((a.N + 255) / 256) * ((a.M + 127) / 128);
-  if (tiles256 * 10 < (long)sm_count() * 9) return launch_tc<128, A8, ACC>(L, Xq, a, st);
-  return launch_tc<256, A8, ACC>(L, Xq, a, st);
+  switch (algo) {
+    case SERQ_ALGO_PREFILL_N128: return launch_tc<128, A8, ACC, 1>(L, Xq, a, st);
+    case SERQ_ALGO_PREFILL_N256: return launch_tc<256, A8, ACC, 1>(L, Xq, a, st);
+    case SERQ_ALGO_PREFILL_PAIR_N256: return launch_tc<256, A8, ACC, 2>(L, Xq, a, st);
+    default: break;
+  }
+  // CTA pairs with 256 x 256 tiles unless that leaves most SMs idle; then
+  // single-CTA 128 x 128 tiles.
+  const long ctas_pair = (long)((a.N + 255) / 256) * 2 * ((a.M + 255) / 256);
+  if (ctas_pair * 10 >= (long)sm_count() * 9) return launch_tc<256, A8, ACC, 2>(L, Xq, a, st);
+  return launch_tc<128, A8, ACC, 1>(L, Xq, a, st);
 }
 
 serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, int M, void* Y, int ldy,
@@ -247,7 +266,7 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
   if (algo == SERQ_ALGO_AUTO) algo = (M <= serq_decode_max_m()) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
   if (algo == SERQ_ALGO_DECODE && M > serq::decode::kMaxTiles * 16)
     return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "decode kernel takes M <= %d (got %d)", serq::decode::kMaxTiles * 16, M);
-  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_PREFILL_N256) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
+  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_PREFILL_PAIR_N256) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
   if ((s = check_device())) return s;
   if ((s = check_layer(L))) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
