@@ -149,33 +149,43 @@ __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* _
   const float inv = (amax > 0.f) ? __fdiv_rn(qf, amax) : 0.f;
   if (threadIdx.x == 0) sx[m] = __fdiv_rn(amax, qf);
 
+  // code = clamp(rint(x * inv), -Q, Q): clamping before rounding gives the
+  // same integer, and adding 1.5 * 2^23 rounds to the nearest integer (ties
+  // to even) exactly for |y| < 2^22; the sum's low mantissa bits are then
+  // the code in two's complement, so a nibble or byte is a mask away.
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23
 #pragma unroll
   for (int i = 0; i < RPL; ++i) {
     const int b = lane + 32 * (warp + nw * i);
     if (b >= nrun) continue;
-    int q[32];
+    uint32_t t[32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float v[8];
       ld.value(raw[i][c], v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int t = __float2int_rn(__fmul_rn(v[e], inv));
-        q[c * 8 + e] = max(-Q, min(Q, t));
+        const float y = fminf(fmaxf(__fmul_rn(v[e], inv), -qf), qf);
+        t[c * 8 + e] = __float_as_uint(__fadd_rn(y, kMagic));
       }
     }
     if (Q == 7) {
-      uint32_t w[4] = {0, 0, 0, 0};
+      uint32_t w[4];
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        w[j >> 2] |= ((uint32_t)(q[j] & 0xF) | ((uint32_t)(q[j + 16] & 0xF) << 4)) << (8 * (j & 3));
+      for (int k = 0; k < 4; ++k) {
+        uint32_t x = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          x |= ((t[4 * k + j] & 0xFu) | ((t[4 * k + j + 16] & 0xFu) << 4)) << (8 * j);
+        w[k] = x;
+      }
       *reinterpret_cast<uint4*>(Xq + (size_t)m * (K >> 1) + b * 16) = make_uint4(w[0], w[1], w[2], w[3]);
     } else {
       uint32_t w[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        w[j] = (uint32_t)(q[4 * j] & 0xFF) | ((uint32_t)(q[4 * j + 1] & 0xFF) << 8) |
-               ((uint32_t)(q[4 * j + 2] & 0xFF) << 16) | ((uint32_t)(q[4 * j + 3] & 0xFF) << 24);
+        w[j] = __byte_perm(__byte_perm(t[4 * j], t[4 * j + 1], 0x0040), __byte_perm(t[4 * j + 2], t[4 * j + 3], 0x0040),
+                           0x5410);
       uint4* dst = reinterpret_cast<uint4*>(Xq + (size_t)m * K + b * 32);
       dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
       dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
