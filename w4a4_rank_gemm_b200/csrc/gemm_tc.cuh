@@ -75,7 +75,7 @@ struct Layout {
   static constexpr int oSw = oPk + PS * kPk;
   static constexpr int oSr = oSw + BN * 4;
   static constexpr int oBar = oSr + BN * 4;
-  static constexpr int nBar = 2 * PS + 2 * US + 2;
+  static constexpr int nBar = 2 * PS + 3 * US + 2;
   static constexpr int oMisc = oBar + nBar * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;             // slack for 1024-B alignment
@@ -120,7 +120,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty_pk = bar + PS;        // packed stage consumed
   uint64_t* full_un = bar + 2 * PS;     // unpacked stage written (both CTAs, on CTA 0)
   uint64_t* empty_un = full_un + US;    // unpacked stage read by the MMAs
-  uint64_t* acc_full = empty_un + US;   // all MMAs complete
+  uint64_t* gather = empty_un + US;     // CTA 1 of a pair: its widening warps done
+  uint64_t* acc_full = gather + US;     // all MMAs complete
   uint64_t* drain = acc_full + 1;       // abort path: MMAs complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::oMisc + 4);
@@ -136,13 +137,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nsteps = p.nkb + p.nrb;
 
   if (threadIdx.x == 0) {
+    // full_un collects one arrival per widening warp of CTA 0 and, for a
+    // pair, a single arrival from CTA 1: there the warps arrive on a local
+    // gather barrier and one thread forwards it (a cluster-scope release
+    // carries a fence, so it is made once per stage, not once per warp).
     for (int s = 0; s < PS; ++s) {
       mbar_init(&full_pk[s], 1);
       mbar_init(&empty_pk[s], kUnpackWarps + (A8 ? 1 : 0));
     }
     for (int s = 0; s < US; ++s) {
-      mbar_init(&full_un[s], kUnpackWarps * CG);
+      mbar_init(&full_un[s], kUnpackWarps + (CG - 1));
       mbar_init(&empty_un[s], 1);
+      mbar_init(&gather[s], kUnpackWarps);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
@@ -260,10 +266,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&empty_pk[s]);
-        if (leader)
-          mbar_arrive(&full_un[u]);
-        else
-          mbar_arrive_remote(&full_un[u], 0);
+        mbar_arrive(leader ? &full_un[u] : &gather[u]);
+      }
+      if (CG == 2 && !leader && ut == 0) {
+        if (!mbar_wait(&gather[u], uph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        mbar_arrive_remote(&full_un[u], 0);
       }
     }
 

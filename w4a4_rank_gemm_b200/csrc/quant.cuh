@@ -149,10 +149,13 @@ __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* _
   const float inv = (amax > 0.f) ? __fdiv_rn(qf, amax) : 0.f;
   if (threadIdx.x == 0) sx[m] = __fdiv_rn(amax, qf);
 
-  // code = clamp(rint(x * inv), -Q, Q): clamping before rounding gives the
-  // same integer, and adding 1.5 * 2^23 rounds to the nearest integer (ties
-  // to even) exactly for |y| < 2^22; the sum's low mantissa bits are then
-  // the code in two's complement, so a nibble or byte is a mask away.
+  // code = clamp(rint(x * inv), -Q, Q).  |x| <= amax and inv = RN(Q/amax)
+  // give |RN(x * inv)| <= Q (1 + 2^-23), which rounds to at most Q, so the
+  // clamp never binds.  Adding 1.5 * 2^23 rounds to the nearest integer
+  // (ties to even) exactly for |y| < 2^22, and the sum's low mantissa bits
+  // are then the code in two's complement: a nibble or byte is a mask away.
+  // (The product and the sum stay two roundings; a fused multiply-add would
+  // round differently at ties.)
   const float kMagic = 12582912.0f;  // 1.5 * 2^23
 #pragma unroll
   for (int i = 0; i < RPL; ++i) {
@@ -165,8 +168,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* _
       ld.value(raw[i][c], v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float y = fminf(fmaxf(__fmul_rn(v[e], inv), -qf), qf);
-        t[c * 8 + e] = __float_as_uint(__fadd_rn(y, kMagic));
+        t[c * 8 + e] = __float_as_uint(__fadd_rn(__fmul_rn(v[e], inv), kMagic));
       }
     }
     if (Q == 7) {
