@@ -139,8 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     // full_un collects one arrival per widening warp of CTA 0 and, for a
     // pair, a single arrival from CTA 1: there the warps arrive on a local
-    // gather barrier and one thread forwards it (a cluster-scope release
-    // carries a fence, so it is made once per stage, not once per warp).
+    // gather barrier and warp 1 forwards it (a cluster-scope release carries
+    // a fence, so it is made once per stage, not once per warp).
     for (int s = 0; s < PS; ++s) {
       mbar_init(&full_pk[s], 1);
       mbar_init(&empty_pk[s], kUnpackWarps + (A8 ? 1 : 0));
@@ -223,6 +223,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit<1>(drain);
         mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
       }
+    } else if (CG == 2 && lane == 0 && !leader) {
+      // CTA 1 of a pair: forward "this CTA's widening warps are done with
+      // stage u" to CTA 0's full barrier, once per stage (a cluster-scope
+      // release), from a thread that has nothing else to do.
+      for (int step = 0; step < nsteps; ++step) {
+        const int u = step % US;
+        const uint32_t uph = (step / US) & 1;
+        if (!mbar_wait(&gather[u], uph, abort_flag, kDevTimeoutUnpack)) break;
+        mbar_arrive_remote(&full_un[u], 0);
+      }
     }
   } else {
     // ------------------------------------------------------------ unpack
@@ -267,10 +277,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         mbar_arrive(&empty_pk[s]);
         mbar_arrive(leader ? &full_un[u] : &gather[u]);
-      }
-      if (CG == 2 && !leader && ut == 0) {
-        if (!mbar_wait(&gather[u], uph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
-        mbar_arrive_remote(&full_un[u], 0);
       }
     }
 
