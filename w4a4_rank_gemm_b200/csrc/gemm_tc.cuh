@@ -75,7 +75,7 @@ struct Layout {
   static constexpr int oSw = oPk + PS * kPk;
   static constexpr int oSr = oSw + BN * 4;
   static constexpr int oBar = oSr + BN * 4;
-  static constexpr int nBar = 2 * PS + 3 * US + 2;
+  static constexpr int nBar = 2 * PS + 2 * US + 2;
   static constexpr int oMisc = oBar + nBar * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;             // slack for 1024-B alignment
@@ -120,8 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty_pk = bar + PS;        // packed stage consumed
   uint64_t* full_un = bar + 2 * PS;     // unpacked stage written (both CTAs, on CTA 0)
   uint64_t* empty_un = full_un + US;    // unpacked stage read by the MMAs
-  uint64_t* gather = empty_un + US;     // CTA 1 of a pair: its widening warps done
-  uint64_t* acc_full = gather + US;     // all MMAs complete
+  uint64_t* acc_full = empty_un + US;   // all MMAs complete
   uint64_t* drain = acc_full + 1;       // abort path: MMAs complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::oMisc + 4);
@@ -137,18 +136,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nsteps = p.nkb + p.nrb;
 
   if (threadIdx.x == 0) {
-    // full_un collects one arrival per widening warp of CTA 0 and, for a
-    // pair, a single arrival from CTA 1: there the warps arrive on a local
-    // gather barrier and warp 1 forwards it (a cluster-scope release carries
-    // a fence, so it is made once per stage, not once per warp).
+    // full_un (on CTA 0) collects one arrival per widening warp of every
+    // CTA of the pair.
     for (int s = 0; s < PS; ++s) {
       mbar_init(&full_pk[s], 1);
       mbar_init(&empty_pk[s], kUnpackWarps + (A8 ? 1 : 0));
     }
     for (int s = 0; s < US; ++s) {
-      mbar_init(&full_un[s], kUnpackWarps + (CG - 1));
+      mbar_init(&full_un[s], kUnpackWarps * CG);
       mbar_init(&empty_un[s], 1);
-      mbar_init(&gather[s], kUnpackWarps);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
@@ -201,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t uph = (step / US) & 1;
         const int s = step % PS;
         const uint32_t ph = (step / PS) & 1;
-        if (!mbar_wait<CG == 2>(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
         if (A8 && !mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
         const bool res = step >= p.nkb;
@@ -222,16 +218,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         umma_commit<1>(drain);
         mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
-      }
-    } else if (CG == 2 && lane == 0 && !leader) {
-      // CTA 1 of a pair: forward "this CTA's widening warps are done with
-      // stage u" to CTA 0's full barrier, once per stage (a cluster-scope
-      // release), from a thread that has nothing else to do.
-      for (int step = 0; step < nsteps; ++step) {
-        const int u = step % US;
-        const uint32_t uph = (step / US) & 1;
-        if (!mbar_wait(&gather[u], uph, abort_flag, kDevTimeoutUnpack)) break;
-        mbar_arrive_remote(&full_un[u], 0);
       }
     }
   } else {
@@ -276,7 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&empty_pk[s]);
-        mbar_arrive(leader ? &full_un[u] : &gather[u]);
+        if (leader)
+          mbar_arrive(&full_un[u]);
+        else
+          mbar_arrive_remote(&full_un[u], 0);
       }
     }
 
