@@ -1,11 +1,15 @@
 #!/usr/bin/env python
 """SERQ quantized-linear benchmark on B200.
 
-One step = one decoder layer's worth of the SERQ hot path on one batch of
-synthetic activations: per shared input, the per-token quantize-and-pack
-kernel, then every projection that reads it through the fused two-accumulator
-GEMM (Llama-2-7B shapes: q/k/v/o 4096x4096, gate/up 4096x11008, down
-11008x4096; W4A4; r = 128; M = 2048 tokens per GPU).
+Default workload (the headline): one step = one Llama-2-7B decoder layer's
+worth of the SERQ hot path on one batch of synthetic activations: per shared
+input the per-token quantize-and-pack kernel, then every projection that reads
+it through the fused two-accumulator GEMM (q/k/v/o 4096x4096, gate/up
+4096x11008, down 11008x4096; W4A4; r = 128; M = 2048 tokens per GPU).
+
+Other workloads (--workload): llama2_7b_decode (M tokens, default 16, CUDA
+graphs, HBM roofline), llama3_8b_w4a8 (M = 4096, INT8 activations),
+mlp_block (gate/up -> SiLU*mul + quantize -> down, M = 4096).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl serq|reference]
 
@@ -34,8 +38,9 @@ METRIC = "serq_linear TOPS and tokens/s at Llama-7B shapes; % of INT8-tensor / H
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 4.5 / 2.25          # nominal dense ratio (recipe)
-N_WEIGHT_COPIES = 8                  # 8 x 101 MB of packed weights > 126 MB L2
+N_WEIGHT_COPIES = 8                  # 8 x ~100 MB of packed weights > 126 MB L2
 N_ACT_COPIES = 2
+WORKLOADS = ("llama2_7b_prefill", "llama2_7b_decode", "llama3_8b_w4a8", "mlp_block")
 
 
 def parse():
@@ -44,13 +49,18 @@ def parse():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["serq", "reference"], default="serq")
-    ap.add_argument("--M", type=int, default=2048)
+    ap.add_argument("--workload", choices=WORKLOADS, default="llama2_7b_prefill")
+    ap.add_argument("--M", type=int, default=None, help="tokens per GPU (default per workload)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--profile", action="store_true",
-                    help="short run for a profiler: no e2e, no CPU baseline, no clocks")
-    return ap.parse_args()
+                    help="short run for a profiler: no e2e, no CPU baseline")
+    a = ap.parse_args()
+    if a.M is None:
+        a.M = {"llama2_7b_prefill": 2048, "llama2_7b_decode": 16, "llama3_8b_w4a8": 4096,
+               "mlp_block": 4096}[a.workload]
+    return a
 
 
 # --------------------------------------------------------------------------
@@ -68,6 +78,13 @@ def groups_of(wl):
 
 def ops_of(M, K, N, r):
     return 2.0 * M * N * (K + r)
+
+
+def linear_bytes(M, K, N, r, a_bits):
+    """Algorithmic DRAM bytes of one linear launch: packed W, packed R, the
+    two scale vectors, the activation codes and scales, the bf16 output."""
+    rpad = (r + 31) // 32 * 32
+    return N * K / 2 + N * rpad / 2 + 8 * N + M * K * a_bits / 8 + 4 * M + 2 * M * N
 
 
 def max_over_ranks(x: float, world: int, device=None) -> float:
@@ -92,15 +109,15 @@ def peaks():
                 "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_hash():
+def kernel_hash(files):
     h = hashlib.sha256()
-    for f in ("gemm_tc.cuh", "common.cuh"):
+    for f in files:
         h.update(open(os.path.join(ROOT, "w4a4_rank_gemm_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per launch of the prefill GEMM from the committed ncu
+def recorded_traffic(workload, files):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, if it was taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -108,7 +125,7 @@ def recorded_traffic(workload):
     except Exception:
         return None
     rec = d.get(workload)
-    if not rec or rec.get("kernel_hash") != kernel_hash():
+    if not rec or rec.get("kernel_hash") != kernel_hash(files):
         return None
     return rec.get("bytes_per_launch")
 
@@ -173,102 +190,251 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------
-# GPU arm
+# GPU workloads
 # --------------------------------------------------------------------------
+class LayerWorkload:
+    """Independent projections grouped by shared input (a decoder layer)."""
+
+    def __init__(self, args, S, torch, dev):
+        from w4a4_rank_gemm_b200 import synth
+        self.S, self.torch, self.dev = S, torch, dev
+        self.name = args.workload
+        M = self.M = args.M
+        if args.workload == "llama3_8b_w4a8":
+            wl = synth.llama3_8b(M=M)
+        else:
+            wl = synth.llama2_7b(M=M)
+        self.wl = wl
+        self.mode = wl.mode
+        self.a_bits = 4 if wl.mode == "w4a4" else 8
+        self.grp = groups_of(wl)
+        r = self.r = wl.rank
+        self.layers = [dict() for _ in range(N_WEIGHT_COPIES)]
+        self.flat = {}
+        for iname, projs in self.grp:
+            inp = wl.inputs[iname]
+            Ws = [torch.from_numpy(p.W).to(dev) for p in projs]
+            Xc = torch.from_numpy(inp.X_calib).to(dev)
+            for c in range(N_WEIGHT_COPIES):
+                for p, L in zip(projs, S.prepare_group(Ws, Xc, r, wl.mode)):
+                    self.layers[c][p.name] = L
+            L0 = self.layers[0][projs[0].name]
+            Xd = torch.from_numpy(inp.X).to(dev).to(torch.bfloat16)
+            self.flat[iname] = [S.flatten_permute(L0, Xd) for _ in range(N_ACT_COPIES)]
+            del Ws, Xc, Xd
+        torch.cuda.synchronize()
+        bpr = lambda K: K // 2 if self.a_bits == 4 else K
+        self.Xq = {i: torch.empty((M, bpr(wl.inputs[i].K)), dtype=torch.uint8, device=dev) for i, _ in self.grp}
+        self.sx = {i: torch.empty(M, dtype=torch.float32, device=dev) for i, _ in self.grp}
+        self.Y = {p.name: torch.empty((M, p.W.shape[1]), dtype=torch.bfloat16, device=dev)
+                  for p in wl.projections}
+        self.gemms = [(p.name, p.W.shape[0], p.W.shape[1]) for p in wl.projections]
+        self.ops_step = sum(ops_of(M, K, N, r) for _, K, N in self.gemms)
+        self.gemm_bytes_step = sum(linear_bytes(M, K, N, r, self.a_bits) for _, K, N in self.gemms)
+        self.launches_per_step = len(self.grp) + len(self.gemms)
+        self.weight_mb = sum(p.W.size for p in wl.projections) / 2 / 1e6
+        self.decode = M <= S.decode_max_m()
+
+    def describe(self):
+        shapes = ", ".join(f"{n} {K}x{N}" for n, K, N in self.gemms)
+        return (f"{self.name}_{self.mode}_r{self.r}: one decoder layer's {len(self.gemms)} projections "
+                f"({shapes}), {len(self.grp)} shared-input quantizes, M = {self.M} tokens per GPU")
+
+    def step(self, i, stream, events=None, gemm_only=False):
+        S, torch = self.S, self.torch
+        c, a = i % N_WEIGHT_COPIES, i % N_ACT_COPIES
+        for iname, projs in self.grp:
+            if not gemm_only:
+                S.quantize_act(self.flat[iname][a], self.mode, Xq=self.Xq[iname], sx=self.sx[iname], stream=stream)
+            for p in projs:
+                if events is not None:
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                S.linear(self.layers[c][p.name], self.Xq[iname], self.sx[iname], Y=self.Y[p.name], stream=stream)
+                if events is not None:
+                    e1.record(stream)
+                    events.append((p.name, e0, e1))
+
+    def e2e_step(self, i, stream, host_in, host_out):
+        S = self.S
+        c = i % N_WEIGHT_COPIES
+        for iname, projs in self.grp:
+            dev_in = self.flat[iname][1]
+            dev_in.copy_(host_in[iname], non_blocking=True)
+            S.quantize_act(dev_in, self.mode, Xq=self.Xq[iname], sx=self.sx[iname], stream=stream)
+            for p in projs:
+                S.linear(self.layers[c][p.name], self.Xq[iname], self.sx[iname], Y=self.Y[p.name], stream=stream)
+                host_out[p.name].copy_(self.Y[p.name], non_blocking=True)
+
+    def host_buffers(self):
+        torch = self.torch
+        host_in = {i: self.flat[i][0].cpu().pin_memory() for i, _ in self.grp}
+        host_out = {n: torch.empty(y.shape, dtype=y.dtype).pin_memory() for n, y in self.Y.items()}
+        return host_in, host_out
+
+
+class MLPWorkload:
+    """gate/up (down_proj's order folded into their columns) -> SiLU*mul +
+    quantize -> down, one Llama-2-7B MLP block."""
+
+    def __init__(self, args, S, torch, dev):
+        from w4a4_rank_gemm_b200 import synth
+        self.S, self.torch, self.dev = S, torch, dev
+        self.name = "mlp_block"
+        M = self.M = args.M
+        blk = synth.mlp_block(M=M)
+        self.r = r = blk.rank
+        self.mode, self.a_bits = "w4a4", 4
+        dv = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+        Wg, Wu, Wd, Xc, Hc = dv(blk.Wg), dv(blk.Wu), dv(blk.Wd), dv(blk.X_calib), dv(blk.H_calib)
+        self.copies = []
+        for c in range(N_WEIGHT_COPIES):
+            (Ld,) = S.prepare_group([Wd], Hc, r, "w4a4")
+            p4, s4 = Ld.perm_smooth()
+            Lg, Lu = S.prepare_group([Wg, Wu], Xc, r, "w4a4", out_perm=[dv(p4), dv(p4)], out_div=[None, dv(s4)])
+            self.copies.append((Lg, Lu, Ld))
+        Lg0 = self.copies[0][0]
+        Xd = dv(blk.X).to(torch.bfloat16)
+        self.flat = [S.flatten_permute(Lg0, Xd) for _ in range(N_ACT_COPIES)]
+        del Wg, Wu, Wd, Xc, Hc, Xd
+        K, F = blk.Wg.shape
+        self.K, self.F = K, F
+        self.Xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        self.sx = torch.empty(M, dtype=torch.float32, device=dev)
+        self.G = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+        self.U = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+        self.Hq = torch.empty((M, F // 2), dtype=torch.uint8, device=dev)
+        self.hsx = torch.empty(M, dtype=torch.float32, device=dev)
+        self.Yd = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        self.gemms = [("gate_proj", K, F), ("up_proj", K, F), ("down_proj", F, K)]
+        self.ops_step = sum(ops_of(M, k, n, r) for _, k, n in self.gemms)
+        self.gemm_bytes_step = sum(linear_bytes(M, k, n, r, 4) for _, k, n in self.gemms)
+        self.launches_per_step = 5
+        self.weight_mb = 3 * K * F / 2 / 1e6
+        self.decode = False
+        torch.cuda.synchronize()
+
+    def describe(self):
+        return (f"mlp_block_w4a4_r{self.r}: Llama-2-7B MLP, gate/up {self.K}x{self.F} with down_proj's saliency "
+                f"order folded into their columns -> SiLU*mul + quantize -> down {self.F}x{self.K}, "
+                f"M = {self.M} tokens per GPU")
+
+    def step(self, i, stream, events=None, gemm_only=False):
+        S, torch = self.S, self.torch
+        Lg, Lu, Ld = self.copies[i % N_WEIGHT_COPIES]
+        if not gemm_only:
+            S.quantize_act(self.flat[i % N_ACT_COPIES], "w4a4", Xq=self.Xq, sx=self.sx, stream=stream)
+        for name, L, xq, sx, y, pre in (("gate_proj", Lg, self.Xq, self.sx, self.G, None),
+                                        ("up_proj", Lu, self.Xq, self.sx, self.U, None),
+                                        ("down_proj", Ld, self.Hq, self.hsx, self.Yd, "silu")):
+            if pre == "silu" and not gemm_only:
+                S.silu_mul_quantize(self.G, self.U, "w4a4", Xq=self.Hq, sx=self.hsx, stream=stream)
+            if events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            S.linear(L, xq, sx, Y=y, stream=stream)
+            if events is not None:
+                e1.record(stream)
+                events.append((name, e0, e1))
+
+    def host_buffers(self):
+        torch = self.torch
+        return ({"x": self.flat[0].cpu().pin_memory()},
+                {"y": torch.empty(self.Yd.shape, dtype=self.Yd.dtype).pin_memory()})
+
+    def e2e_step(self, i, stream, host_in, host_out):
+        self.flat[1].copy_(host_in["x"], non_blocking=True)
+        self.step(1, stream)
+        host_out["y"].copy_(self.Yd, non_blocking=True)
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
     from w4a4_rank_gemm_b200 import build as _build
     _build.build()
     from w4a4_rank_gemm_b200 import serq as S
-    from w4a4_rank_gemm_b200 import synth
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    M = args.M
-    wl = synth.llama2_7b(M=M)
-    grp = groups_of(wl)
-    r = wl.rank
-
-    # offline: prepare N_WEIGHT_COPIES copies of the layer (untimed)
-    layers = [dict() for _ in range(N_WEIGHT_COPIES)]
-    flat = {}
-    for iname, projs in grp:
-        inp = wl.inputs[iname]
-        Ws = [torch.from_numpy(p.W).to(dev) for p in projs]
-        Xc = torch.from_numpy(inp.X_calib).to(dev)
-        for c in range(N_WEIGHT_COPIES):
-            for p, L in zip(projs, S.prepare_group(Ws, Xc, r, "w4a4")):
-                layers[c][p.name] = L
-        L0 = layers[0][projs[0].name]
-        Xd = torch.from_numpy(inp.X).to(dev).to(torch.bfloat16)
-        flat[iname] = [S.flatten_permute(L0, Xd) for _ in range(N_ACT_COPIES)]
-        del Ws, Xc, Xd
-    torch.cuda.synchronize()
-
-    Xq = {i: torch.empty((M, wl.inputs[i].K // 2), dtype=torch.uint8, device=dev) for i, _ in grp}
-    sx = {i: torch.empty(M, dtype=torch.float32, device=dev) for i, _ in grp}
-    Y = {p.name: torch.empty((M, p.W.shape[1]), dtype=torch.bfloat16, device=dev) for p in wl.projections}
-    ops_step = sum(ops_of(M, p.W.shape[0], p.W.shape[1], r) for p in wl.projections)
+    W = MLPWorkload(args, S, torch, dev) if args.workload == "mlp_block" else LayerWorkload(args, S, torch, dev)
     stream = torch.cuda.current_stream()
-
-    def step(i, gemm_events=None):
-        c, a = i % N_WEIGHT_COPIES, i % N_ACT_COPIES
-        for iname, projs in grp:
-            S.quantize_act(flat[iname][a], "w4a4", Xq=Xq[iname], sx=sx[iname], stream=stream)
-            for p in projs:
-                if gemm_events is not None:
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                S.linear(layers[c][p.name], Xq[iname], sx[iname], Y=Y[p.name], stream=stream)
-                if gemm_events is not None:
-                    e1.record(stream)
-                    gemm_events.append((p, e0, e1))
 
     def barrier():
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
 
+    graphs = None
+    if W.decode:
+        # decode kernels run for microseconds: replay one captured step per
+        # weight copy so host launch overhead does not enter the timing
+        for i in range(3):
+            W.step(i, stream)
+        torch.cuda.synchronize()
+        graphs, gemm_graphs = [], []
+        for c in range(N_WEIGHT_COPIES):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                W.step(c, torch.cuda.current_stream())
+            graphs.append(g)
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                W.step(c, torch.cuda.current_stream(), gemm_only=True)
+            gemm_graphs.append(g2)
+        run_step = lambda i: graphs[i % N_WEIGHT_COPIES].replay()
+    else:
+        run_step = lambda i: W.step(i, stream)
+
     for i in range(args.warmup):
-        step(i)
+        run_step(i)
     torch.cuda.synchronize()
     barrier()
 
-    gemm_events = []
+    events = []
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(args.steps):
-            step(i, gemm_events)
+            if graphs is None:
+                W.step(i, stream, events)
+            else:
+                run_step(i)
         t1.record(stream)
         torch.cuda.synchronize()
     elapsed_ms = t0.elapsed_time(t1)
     if S.device_error() != 0:
         raise RuntimeError("a kernel reported a timed-out wait")
-
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     barrier()
 
-    gemm_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in gemm_events)
-    gemm_ops = sum(ops_of(M, p.W.shape[0], p.W.shape[1], r) for p, _, _ in gemm_events)
     per_proj = {}
-    for p, e0, e1 in gemm_events:
-        per_proj.setdefault(p.name, []).append(e0.elapsed_time(e1))
+    if graphs is None:
+        gemm_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in events)
+        for n, e0, e1 in events:
+            per_proj.setdefault(n, []).append(e0.elapsed_time(e1))
+        gemm_note = "CUDA events around every GEMM launch inside the timed region"
+    else:
+        # GEMM-only replays (same kernels, no quantize), timed right after
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for i in range(args.steps):
+            gemm_graphs[i % N_WEIGHT_COPIES].replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        gemm_ms = g0.elapsed_time(g1)
+        gemm_note = "CUDA events around replays of a graph holding only the step's GEMM launches"
     secs = elapsed_ms / 1e3
-    value = ops_step * args.steps * world / secs / 1e12
 
     pk, pk_src = peaks()
     timed_alone = secs < 2.0
-    bf16 = pk.get("bf16_tflops") if timed_alone else pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-    peak_int8 = bf16 * INT8_PER_BF16
-    achieved = gemm_ops / (gemm_ms / 1e3) / 1e12
-    launches_per_step = len(grp) + len(wl.projections)
     res = {
         "metric": METRIC,
-        "value": round(value, 2),
+        "value": round(W.ops_step * args.steps * world / secs / 1e12, 3),
         "unit": "TOPS",
         "n_gpus": world,
         "steps": args.steps,
@@ -277,74 +443,71 @@ def run_gpu(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4 (W4A4 codes, int32 accumulate)",
-        "data": "synthetic (seeded; Llama-2-7B shapes, random-init weights, outlier-channel activations)",
-        "tokens_per_s": round(M * args.steps * world / secs, 1),
+        "dtype": "int4 (W4A4 codes, int32 accumulate)" if W.a_bits == 4 else "int4 weights x int8 activations, int32 accumulate",
+        "data": "synthetic (seeded; Llama shapes, random-init weights, outlier-channel activations)",
+        "tokens_per_s": round(W.M * args.steps * world / secs, 1),
         "config": {
-            "workload": "llama2_7b_prefill_w4a4_r128: one decoder layer's 7 projections "
-                        "(q/k/v/o 4096x4096, gate/up 4096x11008, down 11008x4096), 4 shared-input quantizes",
-            "tokens_per_gpu": M, "rank": r, "mode": "w4a4",
-            "global_batch": M * world, "parallelism": f"dp{world} (independent token batches)",
+            "workload": W.describe(),
+            "tokens_per_gpu": W.M, "rank": W.r, "mode": W.mode,
+            "global_batch": W.M * world, "parallelism": f"dp{world} (independent token batches)",
             "l2": f"inputs larger than L2: {N_WEIGHT_COPIES} prepared weight copies cycled "
-                  f"({N_WEIGHT_COPIES} x {sum(p.W.size for p in wl.projections) // 2 / 1e6:.0f} MB packed) "
-                  f"and {N_ACT_COPIES} activation copies alternated",
+                  f"({N_WEIGHT_COPIES} x {W.weight_mb:.0f} MB packed) and {N_ACT_COPIES} activation copies alternated",
+            "cuda_graphs": graphs is not None,
         },
-        "roofline": {
+        "gpu_launches": W.launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if W.decode:
+        peak = pk.get("hbm_gbs")
+        achieved = W.gemm_bytes_step * args.steps / (gemm_ms / 1e3) / 1e9
+        res["roofline"] = {
+            "kernel": "serq::decode::k_decode (split-K tensor-core GEMV, main + residual accumulators)",
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": recorded_traffic(f"{W.name}_M{W.M}", ["gemv_decode.cuh", "common.cuh"]),
+            "peak_source": f"{pk_src}: hbm_gbs" + (" -- of measured" if pk_src != "fallback" else " -- of fallback"),
+            "gemm_share_of_step": round(gemm_ms / max(elapsed_ms, 1e-9), 4),
+            "timing": gemm_note,
+        }
+    else:
+        bf16 = pk.get("bf16_tflops") if timed_alone else pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+        peak_int8 = bf16 * INT8_PER_BF16
+        achieved = W.ops_step * args.steps / (gemm_ms / 1e3) / 1e12
+        res["roofline"] = {
             "kernel": "serq::tc::k_gemm (tcgen05 kind::i8 prefill GEMM, main + residual accumulators)",
-            "bound": "tensor",
-            "achieved": round(achieved, 1),
-            "peak": round(peak_int8, 1),
-            "unit": "TFLOP/s",
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_int8, 1), "unit": "TFLOP/s",
             "frac": round(achieved / peak_int8, 4),
-            "traffic": recorded_traffic("llama2_7b_prefill"),
-            "peak_source": f"{pk_src}: {'bf16_tflops' if timed_alone else 'bf16_tflops_sustained'} "
-                           f"x {INT8_PER_BF16} (dense int8 : bf16) -- of measured" if pk_src != "fallback"
+            "traffic": recorded_traffic(W.name, ["gemm_tc.cuh", "common.cuh"]),
+            "peak_source": (f"{pk_src}: {'bf16_tflops' if timed_alone else 'bf16_tflops_sustained'} x "
+                            f"{INT8_PER_BF16} (dense int8 : bf16) -- of measured") if pk_src != "fallback"
                            else "fallback 1.59 PFLOP/s bf16 x 2 -- of fallback",
             "gemm_share_of_step": round(gemm_ms / max(elapsed_ms, 1e-9), 4),
             "per_projection_us": {k: round(1e3 * statistics.median(v), 2) for k, v in per_proj.items()},
-        },
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
-    }
-    return res, dict(S=S, torch=torch, wl=wl, grp=grp, layers=layers, flat=flat, Xq=Xq, sx=sx, Y=Y,
-                     ops_step=ops_step, dev=dev, stream=stream)
+            "timing": gemm_note,
+        }
+    return res, dict(S=S, torch=torch, W=W, dev=dev, stream=stream)
 
 
 def run_e2e(args, ctx, world):
     """Same step through the public API with the step's inputs copied from
     pinned host memory and every output copied back, inside the timed region."""
-    torch, S = ctx["torch"], ctx["S"]
-    grp, layers, flat, Xq, sx, Y = ctx["grp"], ctx["layers"], ctx["flat"], ctx["Xq"], ctx["sx"], ctx["Y"]
-    stream = ctx["stream"]
-    host_in = {i: flat[i][0].cpu().pin_memory() for i, _ in grp}
-    dev_in = {i: flat[i][1] for i, _ in grp}
-    host_out = {n: torch.empty(y.shape, dtype=y.dtype).pin_memory() for n, y in Y.items()}
+    torch, W, stream = ctx["torch"], ctx["W"], ctx["stream"]
+    host_in, host_out = W.host_buffers()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     steps = max(3, min(args.steps, 30))
-
-    def step(i):
-        c = i % N_WEIGHT_COPIES
-        for iname, projs in grp:
-            dev_in[iname].copy_(host_in[iname], non_blocking=True)
-            S.quantize_act(dev_in[iname], "w4a4", Xq=Xq[iname], sx=sx[iname], stream=stream)
-            for p in projs:
-                S.linear(layers[c][p.name], Xq[iname], sx[iname], Y=Y[p.name], stream=stream)
-                host_out[p.name].copy_(Y[p.name], non_blocking=True)
-
     for i in range(3):
-        step(i)
+        W.e2e_step(i, stream, host_in, host_out)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(steps):
-        step(i)
+        W.e2e_step(i, stream, host_in, host_out)
     t1.record(stream)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    ms = max_over_ranks(ms, world, ctx["dev"])
-    return {"value": round(ctx["ops_step"] * steps * world / (ms / 1e3) / 1e12, 3), "unit": "TOPS",
+    ms = max_over_ranks(t0.elapsed_time(t1), world, ctx["dev"])
+    return {"value": round(W.ops_step * steps * world / (ms / 1e3) / 1e12, 3), "unit": "TOPS",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 3)}
 
@@ -364,36 +527,54 @@ def cpu_threads():
 class OracleArm:
     """The oracle as it stands, on a bounded token sample of the workload."""
 
-    def __init__(self, M_sample, wl=None):
+    def __init__(self, workload, M_sample):
         from oracle import serq_oracle as O
         from w4a4_rank_gemm_b200 import synth
         self.O = O
-        self.wl = wl if wl is not None else synth.llama2_7b(M=2048)
-        self.grp = groups_of(self.wl)
+        self.workload = workload
         self.M_s = M_sample
-        self.prep = {}
-        self.xh = {}
+        if workload == "mlp_block":
+            blk = synth.mlp_block(M=max(M_sample, 16))
+            self.blk = blk
+            self.prep = O.prepare_mlp(blk.Wg, blk.Wu, blk.Wd, blk.X_calib, blk.H_calib, blk.rank)
+            self.X = blk.X[:M_sample]
+            K, F = blk.Wg.shape
+            self.ops = 2 * ops_of(M_sample, K, F, blk.rank) + ops_of(M_sample, F, K, blk.rank)
+            self.rank = blk.rank
+            return
+        wl = synth.llama3_8b(M=max(M_sample, 16)) if workload == "llama3_8b_w4a8" else \
+            synth.llama2_7b(M=max(M_sample, 16))
+        self.wl, self.grp = wl, groups_of(wl)
+        self.bits = 4 if wl.mode == "w4a4" else 8
+        self.rank = wl.rank
+        self.prep, self.xh = {}, {}
         for iname, projs in self.grp:
-            inp = self.wl.inputs[iname]
-            _, _, ls = O.prepare_group([p.W for p in projs], inp.X_calib, self.wl.rank)
+            inp = wl.inputs[iname]
+            _, _, ls = O.prepare_group([p.W for p in projs], inp.X_calib, wl.rank)
             for p, L in zip(projs, ls):
                 self.prep[p.name] = L
-            L0 = ls[0]
-            self.xh[iname] = O.flatten_permute(inp.X[:M_sample], L0.s, L0.pi, out_bf16=True)
-        self.ops = sum(ops_of(M_sample, p.W.shape[0], p.W.shape[1], self.wl.rank) for p in self.wl.projections)
+            self.xh[iname] = O.flatten_permute(inp.X[:M_sample], ls[0].s, ls[0].pi, out_bf16=True)
+        self.ops = sum(ops_of(M_sample, p.W.shape[0], p.W.shape[1], wl.rank) for p in wl.projections)
 
     def step(self):
         O = self.O
+        if self.workload == "mlp_block":
+            O.mlp_forward(self.X, self.prep)
+            return
         for iname, projs in self.grp:
-            xq, sx = O.quantize_act(self.xh[iname], 4)
+            xq, sx = O.quantize_act(self.xh[iname], self.bits)
             for p in projs:
                 L = self.prep[p.name]
                 acc0, acc1 = O.linear_accum(xq, L)
                 O.linear_epilogue(acc0, acc1, sx, L)
 
 
-def cpu_baseline(args, wl=None):
-    arm = OracleArm(64, wl)
+def oracle_sample(args):
+    return min(args.M, 64)
+
+
+def cpu_baseline(args):
+    arm = OracleArm(args.workload, oracle_sample(args))
     arm.step()  # warm (allocations)
     n, t = 0, 0.0
     while t < args.cpu_seconds or n < 2:
@@ -403,12 +584,12 @@ def cpu_baseline(args, wl=None):
         n += 1
     return {"value": round(arm.ops * n / t / 1e12, 5), "unit": "TOPS", "cores": cpu_threads(),
             "kind": "oracle",
-            "sample": f"{arm.M_s} tokens of each of the 4 layer inputs through all 7 projections "
-                      f"(quantize + two-accumulator integer GEMM + fp64 epilogue), {n} passes in {t:.1f} s"}
+            "sample": f"{arm.M_s} tokens through the workload's quantize + two-accumulator integer GEMM + "
+                      f"fp64 epilogue ({args.workload}), {n} passes in {t:.1f} s"}
 
 
 def run_reference(args):
-    arm = OracleArm(64)
+    arm = OracleArm(args.workload, oracle_sample(args))
     for _ in range(args.warmup):
         arm.step()
     t0 = time.perf_counter()
@@ -417,15 +598,15 @@ def run_reference(args):
     secs = time.perf_counter() - t0
     value = arm.ops * args.steps / secs / 1e12
     cores = cpu_threads()
-    sample = f"{arm.M_s} tokens per layer input through all 7 Llama-2-7B projections per step"
+    sample = f"{arm.M_s} tokens per step through the {args.workload} workload"
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "TOPS",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int4 codes, int64-exact integer GEMM + fp64 epilogue (CPU oracle)",
-        "data": "synthetic (seeded; Llama-2-7B shapes)",
-        "config": {"workload": "llama2_7b_prefill_w4a4_r128 (bounded token sample)", "tokens_per_step": arm.M_s,
-                   "rank": arm.wl.rank, "mode": "w4a4"},
+        "vs_baseline": None, "dtype": "integer codes, exact integer GEMM + fp64 epilogue (CPU oracle)",
+        "data": "synthetic (seeded; Llama shapes)",
+        "config": {"workload": f"{args.workload} (bounded token sample)", "tokens_per_step": arm.M_s,
+                   "rank": arm.rank},
         "cpu_baseline": {"value": round(value, 5), "unit": "TOPS", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 5), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -455,7 +636,7 @@ def main():
         if not args.profile and not args.no_e2e:
             res["e2e"] = run_e2e(args, ctx, world)
         if rank == 0 and world == 1 and not args.profile and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline(args, None)
+            res["cpu_baseline"] = cpu_baseline(args)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
