@@ -31,6 +31,7 @@ struct LoadBF16 {
     }
   }
   __device__ __forceinline__ void value(const uint4 (&r)[kWords], float (&v)[8]) const { bf16x8(r[0], v); }
+  __device__ __forceinline__ void finalize(uint4 (&)[kWords]) const {}
 };
 
 struct LoadF32 {
@@ -48,6 +49,7 @@ struct LoadF32 {
     v[4] = __uint_as_float(r[1].x); v[5] = __uint_as_float(r[1].y);
     v[6] = __uint_as_float(r[1].z); v[7] = __uint_as_float(r[1].w);
   }
+  __device__ __forceinline__ void finalize(uint4 (&)[kWords]) const {}
 };
 
 // e^x in fp32: Cody & Waite argument reduction x = k ln2 + r with ln 2 split
@@ -71,10 +73,16 @@ __device__ __forceinline__ float exp_cw(float x) {
   p = __fadd_rn(__fmul_rn(p, r), 0.5f);
   p = __fadd_rn(__fmul_rn(p, r), 1.0f);
   p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  return ldexpf(p, (int)k);
+  // p * 2^k, correctly rounded: a power-of-two factor is exact while the
+  // product stays normal; below that the last multiply rounds once.
+  const int ki = (int)k;  // -127 .. 127
+  if (ki >= -125) return __fmul_rn(p, __int_as_float((ki + 127) << 23));
+  return __fmul_rn(__fmul_rn(p, __int_as_float((ki + 129) << 23)), 0.25f);
 }
 
-// h = silu(g) * u = g / (1 + e^-g) * u, fp32.
+// h = silu(g) * u = g / (1 + e^-g) * u, fp32.  `finalize` replaces the raw
+// (g, u) bf16 pairs by the 8 fp32 values of h in the same two words, so h is
+// computed once per element.
 struct LoadSiluMul {
   static constexpr int kWords = 2;
   const __nv_bfloat16* G;
@@ -84,15 +92,23 @@ struct LoadSiluMul {
     r[0] = __ldg(reinterpret_cast<const uint4*>(G + (size_t)m * ld + k0));
     r[1] = __ldg(reinterpret_cast<const uint4*>(U + (size_t)m * ld + k0));
   }
-  __device__ __forceinline__ void value(const uint4 (&r)[kWords], float (&v)[8]) const {
-    float g[8], u[8];
+  __device__ __forceinline__ void finalize(uint4 (&r)[kWords]) const {
+    float g[8], u[8], h[8];
     LoadBF16::bf16x8(r[0], g);
     LoadBF16::bf16x8(r[1], u);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float den = __fadd_rn(1.f, exp_cw(-g[i]));
-      v[i] = __fmul_rn(__fdiv_rn(g[i], den), u[i]);
+      h[i] = __fmul_rn(__fdiv_rn(g[i], den), u[i]);
     }
+    r[0] = make_uint4(__float_as_uint(h[0]), __float_as_uint(h[1]), __float_as_uint(h[2]), __float_as_uint(h[3]));
+    r[1] = make_uint4(__float_as_uint(h[4]), __float_as_uint(h[5]), __float_as_uint(h[6]), __float_as_uint(h[7]));
+  }
+  __device__ __forceinline__ void value(const uint4 (&r)[kWords], float (&v)[8]) const {
+    v[0] = __uint_as_float(r[0].x); v[1] = __uint_as_float(r[0].y);
+    v[2] = __uint_as_float(r[0].z); v[3] = __uint_as_float(r[0].w);
+    v[4] = __uint_as_float(r[1].x); v[5] = __uint_as_float(r[1].y);
+    v[6] = __uint_as_float(r[1].z); v[7] = __uint_as_float(r[1].w);
   }
 };
 
@@ -129,6 +145,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* _
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float v[8];
+        ld.finalize(raw[i][c]);
         ld.value(raw[i][c], v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
