@@ -61,8 +61,10 @@ struct Args {
 // packed stage, already in the MMA layout), per-column scales, barriers.
 template <int BN, bool A8, int CG>
 struct Layout {
-  static constexpr int PS = (CG == 2) ? 4 : 3;             // packed (TMA) stages
-  static constexpr int US = (CG == 2) ? 3 : 2;             // unpacked stages
+  // ring depths: as deep as shared memory allows, so the MMA issue never
+  // waits on the two barrier hops (MMA done -> widening -> MMA)
+  static constexpr int PS = (CG == 2) ? 5 : 3;             // packed (TMA) stages
+  static constexpr int US = (CG == 2) ? 4 : (BN == 256 ? 3 : 4);  // unpacked stages
   static constexpr int BNL = BN / CG;                      // weight rows held by this CTA
   static constexpr int kPkA = A8 ? BM * BK : BM * BK / 2;  // A part of a packed stage
   static constexpr int kPkB = BNL * BK / 2;                // B/R part (packed INT4)
