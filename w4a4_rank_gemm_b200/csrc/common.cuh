@@ -148,6 +148,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// One lane of a converged warp (the warp keeps executing together, which
+// keeps the single-lane tcgen05 issue cheap).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred px;\n\t"
+      "elect.sync _|px, 0xffffffff;\n\t"
+      "@px mov.s32 %0, 1;\n\t}\n"
+      : "+r"(pred));
+  return pred != 0;
+}
+
 // ----------------------------------------------------------------- tcgen05
 // TMEM allocation by one warp; with CG = 2 both CTAs of the pair execute it
 // from the same warp and slot and receive the same address.

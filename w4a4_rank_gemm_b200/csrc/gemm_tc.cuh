@@ -189,12 +189,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0 && leader) {
+    // The whole warp runs the loop and waits together; one elected lane
+    // issues.  Descriptors are built once per stage and advanced by the
+    // 32-byte k step (2 in the 16-byte address field).
+    if (leader) {
       constexpr uint32_t idesc = umma_idesc_i8(BM * CG, BN);
       const uint32_t pk_base = smem_u32(smem + L::oPk);
       const uint32_t un_base = smem_u32(smem + L::oUn);
       bool ok = true;
-      for (int step = 0; step < nsteps && ok; ++step) {
+      for (int step = 0; step < nsteps; ++step) {
         const int u = step % US;
         const uint32_t uph = (step / US) & 1;
         const int s = step % PS;
@@ -204,23 +207,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const bool res = step >= p.nkb;
         const int j = res ? step - p.nkb : step;
-        const int nk = res ? min(BK / 32, (p.rpad - j * BK) / 32) : BK / 32;
         const uint32_t d = tmem + (res ? (uint32_t)BN : 0u);
-        const uint32_t a_tile = A8 ? pk_base + s * L::kPk : un_base + u * L::kUn;
-        const uint32_t b_tile = un_base + u * L::kUn + L::kUnA;
-        for (int kk = 0; kk < nk; ++kk) {
-          umma_i8<CG>(d, umma_desc_k_sw128(a_tile + kk * 32), umma_desc_k_sw128(b_tile + kk * 32), idesc,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t da = umma_desc_k_sw128(A8 ? pk_base + s * L::kPk : un_base + u * L::kUn);
+        const uint64_t db = umma_desc_k_sw128(un_base + u * L::kUn + L::kUnA);
+        if (!res) {
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk)
+              umma_i8<CG>(d, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_commit<CG>(&empty_un[u]);
+            if (A8) umma_commit<CG>(&empty_pk[s]);
+          }
+        } else {
+          const int nk = min(BK / 32, (p.rpad - j * BK) / 32);
+          if (elect_one()) {
+            for (int kk = 0; kk < nk; ++kk)
+              umma_i8<CG>(d, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_commit<CG>(&empty_un[u]);
+            if (A8) umma_commit<CG>(&empty_pk[s]);
+          }
         }
-        umma_commit<CG>(&empty_un[u]);
-        if (A8) umma_commit<CG>(&empty_pk[s]);
+        __syncwarp();
       }
-      if (ok) {
-        umma_commit<CG>(acc_full);
-      } else {
-        umma_commit<1>(drain);
-        mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
+      if (elect_one()) {
+        if (ok) {
+          umma_commit<CG>(acc_full);
+        } else {
+          umma_commit<1>(drain);
+          mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
+        }
       }
+      __syncwarp();
     }
   } else {
     // ------------------------------------------------------------ unpack
