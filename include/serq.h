@@ -64,8 +64,10 @@ typedef enum {
   SERQ_ALGO_DECODE = 2,        /* memory-bound split-K tensor-core GEMV, M <= 64 */
   SERQ_ALGO_PREFILL_N128 = 3,  /* PREFILL with 128 x 128 output tiles, one CTA  */
   SERQ_ALGO_PREFILL_N256 = 4,  /* PREFILL with 128 x 256 output tiles, one CTA  */
-  SERQ_ALGO_PREFILL_PAIR_N256 = 5 /* PREFILL with 256 x 256 tiles on a CTA pair
-                                     (tcgen05 cta_group::2)                     */
+  SERQ_ALGO_PREFILL_PAIR_N256 = 5, /* PREFILL with 256 x 256 tiles on a CTA pair
+                                      (tcgen05 cta_group::2)                    */
+  SERQ_ALGO_PREFILL_PAIR_TMEM_A = 6 /* W4A4 only: 256 x 192 tiles on a CTA pair with
+                                       the widened activations in tensor memory  */
 } serq_algo;
 
 typedef struct serq_layer serq_layer;

@@ -146,7 +146,7 @@ def test_linear_accum_bit_exact(S, mode, M, K, N, r):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, r, mode)
     acc0, acc1 = O.linear_accum(xq, ol)
     algos = [S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
-        ([S.ALGO_DECODE] if M <= 64 else [])
+        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE] if M <= 64 else [])
     for algo in algos:
         g0, g1 = S.linear_accum(L, Xq, algo)
         torch.cuda.synchronize()
@@ -162,7 +162,7 @@ def test_linear_output_within_tolerance(S, mode, M, K, N, r):
     acc0, acc1 = O.linear_accum(xq, ol)
     y_ref = O.linear_epilogue(acc0, acc1, osx, ol)
     algos = [S.ALGO_AUTO, S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
-        ([S.ALGO_DECODE] if M <= 64 else [])
+        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE] if M <= 64 else [])
     for algo in algos:
         Y = S.linear(L, Xq, sx, algo=algo)
         torch.cuda.synchronize()

@@ -362,3 +362,297 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace tc
 }  // namespace serq
+
+namespace serq {
+namespace tc {
+
+// ---------------------------------------------------------------------------
+// W4A4 prefill on CTA pairs with the activation operand in tensor memory.
+//
+// Each 128-k step of the pipeline above moves, per SM, the TMA writes, the
+// widening loads and stores and the tensor-core operand reads through shared
+// memory; with the widened activations written to TMEM instead (tcgen05.st
+// straight from the widening registers, read by the MMA as its A operand)
+// the activation half of the widened stores and of the operand reads leaves
+// shared memory.  TMEM then holds acc0 (BN columns), acc1 (BN) and TS widened
+// activation stages of 32 columns (128 int8 per lane, four per column), so
+// BN = 192: 2 * 192 + 4 * 32 = 512 columns.
+//
+// Warps: 0 TMA, 1 TMEM owner / MMA issue (CTA 0), 4..7 widen the 128
+// activation rows of this CTA into TMEM (warp w writes TMEM lanes
+// 32 (w % 4) .. +31, one row per thread), 2, 3, 8, 9 widen this CTA's BN/2
+// weight rows into shared memory; all eight run the epilogue.
+// The packed activation tile arrives with the 64-byte TMA swizzle, so the
+// per-thread row reads hit distinct banks.
+template <int BN>
+struct LayoutTA {
+  static constexpr int CG = 2;
+  static constexpr int BNL = BN / 2;                  // weight rows per CTA
+  static constexpr int PS = 6;                        // packed stages
+  static constexpr int US = 4;                        // widened stages (smem B + TMEM A)
+  static constexpr int kPkA = BM * BK / 2;            // 8 KB, 64-byte swizzled
+  static constexpr int kPkB = BNL * BK / 2;
+  static constexpr int kPk = kPkA + kPkB;
+  static constexpr int kUn = BNL * BK;                // widened weight rows
+  static constexpr int oUn = 0;
+  static constexpr int oPk = oUn + US * kUn;
+  static constexpr int oSw = oPk + PS * kPk;
+  static constexpr int oSr = oSw + BN * 4;
+  static constexpr int oBar = oSr + BN * 4;
+  static constexpr int nBar = 2 * PS + 2 * US + 2;
+  static constexpr int oMisc = oBar + nBar * 8;
+  static constexpr int kBytes = oMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr uint32_t kTxBytes = kPk;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemA = 2 * BN;          // first activation stage column
+  static constexpr int kPiecesB = BNL * 4 / 128;      // per weight-widening thread
+  static_assert(2 * BN + US * (BK / 4) <= 512, "TMEM budget");
+  static_assert(BNL * 4 % 128 == 0, "weight pieces must divide evenly");
+  static_assert(kPk % 1024 == 0 && kUn % 1024 == 0, "tiles must stay 1024-aligned");
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+template <int BN, bool ACC_OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_ta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmR, const Args p) {
+  using L = LayoutTA<BN>;
+  constexpr int PS = L::PS, US = L::US;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::oBar);
+  uint64_t* full_pk = bar;
+  uint64_t* empty_pk = bar + PS;
+  uint64_t* full_un = bar + 2 * PS;     // on CTA 0: both CTAs' widening warps
+  uint64_t* empty_un = full_un + US;
+  uint64_t* acc_full = empty_un + US;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::oMisc + 4);
+  float* sw_t = reinterpret_cast<float*>(smem + L::oSw);
+  float* sr_t = reinterpret_cast<float*>(smem + L::oSr);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int n0 = blockIdx.y * BN;
+  const int nb0 = n0 + (int)rank * L::BNL;
+  const int m0 = blockIdx.x * BM;
+  const int nsteps = p.nkb + p.nrb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PS; ++s) {
+      mbar_init(&full_pk[s], 1);
+      mbar_init(&empty_pk[s], kUnpackWarps);
+    }
+    for (int s = 0; s < US; ++s) {
+      mbar_init(&full_un[s], kUnpackWarps * 2);
+      mbar_init(&empty_un[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmR);
+  }
+  if (warp == 1) {
+    tmem_alloc<2>(tmem_slot, L::kTmemCols);
+    tmem_relinquish<2>();
+  }
+  for (int i = threadIdx.x; i < BN; i += blockDim.x) {
+    const int n = n0 + i;
+    sw_t[i] = (n < p.N) ? p.sw[n] : 0.f;
+    sr_t[i] = (n < p.N) ? p.sr[n] : 0.f;
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int step = 0; step < nsteps; ++step) {
+        const int s = step % PS;
+        const uint32_t ph = (step / PS) & 1;
+        if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) break;
+        mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
+        const bool res = step >= p.nkb;
+        const int j = res ? step - p.nkb : step;
+        uint8_t* stage = smem + L::oPk + s * L::kPk;
+        tma_load_2d(stage, &tmA, &full_pk[s], j * (BK / 2), m0);
+        tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issue
+    if (leader) {
+      constexpr uint32_t idesc = umma_idesc_i8(BM * 2, BN);
+      const uint32_t un_base = smem_u32(smem + L::oUn);
+      bool ok = true;
+      for (int step = 0; step < nsteps; ++step) {
+        const int u = step % US;
+        const uint32_t uph = (step / US) & 1;
+        if (!mbar_wait(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
+        tc_fence_after();
+        const bool res = step >= p.nkb;
+        const int j = res ? step - p.nkb : step;
+        const uint32_t d = tmem + (res ? (uint32_t)BN : 0u);
+        const uint32_t a = tmem + L::kTmemA + (uint32_t)(u * (BK / 4));
+        const uint64_t db = umma_desc_k_sw128(un_base + u * L::kUn);
+        const int nk = res ? min(BK / 32, (p.rpad - j * BK) / 32) : BK / 32;
+        if (elect_one()) {
+          for (int kk = 0; kk < nk; ++kk)
+            umma_i8_ts<2>(d, a + (uint32_t)(kk * 8), db + (uint64_t)(2 * kk), idesc, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit<2>(&empty_un[u]);
+        }
+        __syncwarp();
+      }
+      if (elect_one()) {
+        if (ok) {
+          umma_commit<2>(acc_full);
+        } else {
+          umma_commit<1>(drain);
+          mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
+        }
+      }
+      __syncwarp();
+    }
+  } else {
+    // ----------------------------------------------------------- widening
+    const bool act = (warp >= 4 && warp <= 7);
+    const int q = warp & 3;                            // TMEM lane quadrant
+    const int arow = q * 32 + lane;                    // activation row (act warps)
+    const int bt = act ? 0 : ((warp < 4 ? warp - 2 : warp - 6) * 32 + lane);  // 0..127
+    uint32_t a_off[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) a_off[c] = arow * (BK / 2) + ((c ^ ((arow >> 1) & 3)) << 4);
+    constexpr int NPB = L::kPiecesB;
+    uint32_t src_off[NPB], dst_off[NPB];
+#pragma unroll
+    for (int i = 0; i < NPB; ++i) {
+      const int pc = bt + i * 128;
+      const int row = pc >> 2, c = pc & 3;
+      src_off[i] = L::kPkA + row * (BK / 2) + c * 16;
+      dst_off[i] = row * BK + (((2 * c) ^ (row & 7)) << 4);
+    }
+    bool ok = true;
+    for (int step = 0; step < nsteps; ++step) {
+      const int s = step % PS;
+      const uint32_t ph = (step / PS) & 1;
+      const int u = step % US;
+      const uint32_t uph = (step / US) & 1;
+      if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+      if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+      const uint8_t* pk = smem + L::oPk + s * L::kPk;
+      if (act) {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(pk + a_off[c]);
+          uint4 lo, hi;
+          widen_run(v, lo, hi);
+          r[8 * c + 0] = lo.x; r[8 * c + 1] = lo.y; r[8 * c + 2] = lo.z; r[8 * c + 3] = lo.w;
+          r[8 * c + 4] = hi.x; r[8 * c + 5] = hi.y; r[8 * c + 6] = hi.z; r[8 * c + 7] = hi.w;
+        }
+        tmem_st_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + L::kTmemA + (uint32_t)(u * (BK / 4)), r);
+        tmem_st_wait();
+        tc_fence_before();
+      } else {
+        uint8_t* un = smem + L::oUn + u * L::kUn;
+        uint4 v[NPB];
+#pragma unroll
+        for (int i = 0; i < NPB; ++i) v[i] = *reinterpret_cast<const uint4*>(pk + src_off[i]);
+#pragma unroll
+        for (int i = 0; i < NPB; ++i) {
+          uint4 lo, hi;
+          widen_run(v[i], lo, hi);
+          *reinterpret_cast<uint4*>(un + dst_off[i]) = lo;
+          *reinterpret_cast<uint4*>(un + (dst_off[i] ^ 16u)) = hi;
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty_pk[s]);
+        if (leader)
+          mbar_arrive(&full_un[u]);
+        else
+          mbar_arrive_remote(&full_un[u], 0);
+      }
+    }
+
+    // ---------------------------------------------------------- epilogue
+    if (ok && mbar_wait(acc_full, 0, abort_flag, kDevTimeoutEpilogue)) {
+      tc_fence_after();
+      const int half = (warp - 2) >> 2;
+      const int row = m0 + q * 32 + lane;
+      const bool has_r = p.nrb > 0;
+      constexpr int kShift = 8;
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+        uint32_t r0[32], r1[32];
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c;
+        __syncwarp();
+        tmem_ld_32x32b_x32(taddr, r0);
+        if (has_r) tmem_ld_32x32b_x32(taddr + BN, r1);
+        tmem_ld_wait();
+        if (!has_r) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r1[i] = 0;
+        }
+        if (row >= p.M || n0 + c >= p.N) {
+          // row past M (zero-filled A) or column chunk past N: nothing to store
+        } else if (ACC_OUT) {
+          int32_t* o0 = p.acc0 + (size_t)row * p.N + n0 + c;
+          int32_t* o1 = p.acc1 + (size_t)row * p.N + n0 + c;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            *reinterpret_cast<int4*>(o0 + i) =
+                make_int4((int)r0[i] >> kShift, (int)r0[i + 1] >> kShift, (int)r0[i + 2] >> kShift,
+                          (int)r0[i + 3] >> kShift);
+            *reinterpret_cast<int4*>(o1 + i) =
+                make_int4((int)r1[i] >> kShift, (int)r1[i + 1] >> kShift, (int)r1[i + 2] >> kShift,
+                          (int)r1[i + 3] >> kShift);
+          }
+        } else {
+          const float sxm = p.sx[row];
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float y0 = sxm * fmaf(sw_t[c + i], (float)((int)r0[i] >> kShift),
+                                        sr_t[c + i] * (float)((int)r1[i] >> kShift));
+            const float y1 = sxm * fmaf(sw_t[c + i + 1], (float)((int)r0[i + 1] >> kShift),
+                                        sr_t[c + i + 1] * (float)((int)r1[i + 1] >> kShift));
+            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+            packed[i >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(p.Y + (size_t)row * p.ldy + n0 + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && warp == 0 && lane == 0) {
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < 100000ull) {
+    }
+  }
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<2>(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace tc
+}  // namespace serq

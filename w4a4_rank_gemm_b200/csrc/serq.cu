@@ -101,8 +101,8 @@ struct serq_layer {
   float* sr;
   int32_t* perm;
   float* smooth;
-  CUtensorMap tmB[2];  // box rows 128, 256
-  CUtensorMap tmR[2];
+  CUtensorMap tmB[3];  // box rows 128, 256, 96
+  CUtensorMap tmR[3];
 };
 
 namespace {
@@ -151,8 +151,8 @@ void free_layer(serq_layer* L) {
 }
 
 bool build_weight_maps(serq_layer* L) {
-  const int boxes[2] = {128, 256};
-  for (int i = 0; i < 2; ++i) {
+  const int boxes[3] = {128, 256, 96};
+  for (int i = 0; i < 3; ++i) {
     if (!make_map(&L->tmB[i], L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 64, boxes[i],
                   CU_TENSOR_MAP_SWIZZLE_NONE))
       return false;
@@ -219,6 +219,38 @@ cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args&
   return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[bi], L->tmR[bi], a);
 }
 
+// W4A4 on CTA pairs with the activations in tensor memory, 256 x 192 tiles.
+template <bool ACC>
+cudaError_t launch_tc_ta(const serq_layer* L, const void* Xq, const serq::tc::Args& a, cudaStream_t st) {
+  constexpr int BN = 192;
+  using Lay = serq::tc::LayoutTA<BN>;
+  CUtensorMap tmA;
+  if (!make_map(&tmA, Xq, (uint64_t)a.K / 2, (uint64_t)a.M, (uint64_t)a.K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  auto kern = serq::tc::k_gemm_ta<BN, ACC>;
+  static int attr_set[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    set_smem(kern, Lay::kAlloc);
+    attr_set[dev] = 1;
+  }
+  const int mtiles = (a.M + 255) / 256;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(mtiles * 2, (a.N + BN - 1) / BN);
+  cfg.blockDim = dim3(serq::tc::kThreads);
+  cfg.dynamicSmemBytes = Lay::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[2], L->tmR[2], a);
+}
+
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -237,6 +269,9 @@ cudaError_t dispatch_tc(const serq_layer* L, const void* Xq, const serq::tc::Arg
     case SERQ_ALGO_PREFILL_N128: return launch_tc<128, A8, ACC, 1>(L, Xq, a, st);
     case SERQ_ALGO_PREFILL_N256: return launch_tc<256, A8, ACC, 1>(L, Xq, a, st);
     case SERQ_ALGO_PREFILL_PAIR_N256: return launch_tc<256, A8, ACC, 2>(L, Xq, a, st);
+    case SERQ_ALGO_PREFILL_PAIR_TMEM_A:
+      if (A8) return cudaErrorInvalidValue;
+      return launch_tc_ta<ACC>(L, Xq, a, st);
     default: break;
   }
   // CTA pairs with 256 x 256 tiles unless that leaves most SMs idle; then
@@ -266,7 +301,9 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
   if (algo == SERQ_ALGO_AUTO) algo = (M <= serq_decode_max_m()) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
   if (algo == SERQ_ALGO_DECODE && M > serq::decode::kMaxTiles * 16)
     return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "decode kernel takes M <= %d (got %d)", serq::decode::kMaxTiles * 16, M);
-  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_PREFILL_PAIR_N256) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
+  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_PREFILL_PAIR_TMEM_A) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
+  if (algo == SERQ_ALGO_PREFILL_PAIR_TMEM_A && L->mode != SERQ_W4A4)
+    return fail(SERQ_ERR_INVALID_ARG, "SERQ_ALGO_PREFILL_PAIR_TMEM_A takes W4A4 layers");
   if ((s = check_device())) return s;
   if ((s = check_layer(L))) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
