@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--algo", type=int, default=0,
+                    help="serq_algo for every linear launch (0 = automatic choice)")
     ap.add_argument("--profile", action="store_true",
                     help="short run for a profiler: no e2e, no CPU baseline")
     a = ap.parse_args()
@@ -198,6 +200,7 @@ class LayerWorkload:
     def __init__(self, args, S, torch, dev):
         from w4a4_rank_gemm_b200 import synth
         self.S, self.torch, self.dev = S, torch, dev
+        self.algo = args.algo
         self.name = args.workload
         M = self.M = args.M
         if args.workload == "llama3_8b_w4a8":
@@ -251,7 +254,7 @@ class LayerWorkload:
                     e0 = torch.cuda.Event(enable_timing=True)
                     e1 = torch.cuda.Event(enable_timing=True)
                     e0.record(stream)
-                S.linear(self.layers[c][p.name], self.Xq[iname], self.sx[iname], Y=self.Y[p.name], stream=stream)
+                S.linear(self.layers[c][p.name], self.Xq[iname], self.sx[iname], Y=self.Y[p.name], algo=self.algo, stream=stream)
                 if events is not None:
                     e1.record(stream)
                     events.append((p.name, e0, e1))
@@ -264,7 +267,7 @@ class LayerWorkload:
             dev_in.copy_(host_in[iname], non_blocking=True)
             S.quantize_act(dev_in, self.mode, Xq=self.Xq[iname], sx=self.sx[iname], stream=stream)
             for p in projs:
-                S.linear(self.layers[c][p.name], self.Xq[iname], self.sx[iname], Y=self.Y[p.name], stream=stream)
+                S.linear(self.layers[c][p.name], self.Xq[iname], self.sx[iname], Y=self.Y[p.name], algo=self.algo, stream=stream)
                 host_out[p.name].copy_(self.Y[p.name], non_blocking=True)
 
     def host_buffers(self):
@@ -281,6 +284,7 @@ class MLPWorkload:
     def __init__(self, args, S, torch, dev):
         from w4a4_rank_gemm_b200 import synth
         self.S, self.torch, self.dev = S, torch, dev
+        self.algo = args.algo
         self.name = "mlp_block"
         M = self.M = args.M
         blk = synth.mlp_block(M=M)
@@ -334,7 +338,7 @@ class MLPWorkload:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            S.linear(L, xq, sx, Y=y, stream=stream)
+            S.linear(L, xq, sx, Y=y, algo=self.algo, stream=stream)
             if events is not None:
                 e1.record(stream)
                 events.append((name, e0, e1))
@@ -453,6 +457,7 @@ def run_gpu(args, rank, world, local_rank):
             "l2": f"inputs larger than L2: {N_WEIGHT_COPIES} prepared weight copies cycled "
                   f"({N_WEIGHT_COPIES} x {W.weight_mb:.0f} MB packed) and {N_ACT_COPIES} activation copies alternated",
             "cuda_graphs": graphs is not None,
+            "algo": args.algo,
         },
         "gpu_launches": W.launches_per_step * args.steps,
         "clocks": clk.summary(),
