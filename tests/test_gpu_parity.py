@@ -127,6 +127,8 @@ SHAPES = [
     (300, 1152, 320, 96),   # ragged M and N (N % 256 != 0), K % 128 != 0 ... K = 1152 = 9*128
     (257, 416, 256, 416),   # r = K (whole matrix compensated), K % 128 = 32
     (512, 2048, 1024, 128),
+    (2100, 384, 3200, 32),  # more tiles than CTA pairs / SMs: each CTA runs several tiles
+    (1100, 128, 5120, 0),   # one k step per tile, no residual, several tiles per CTA
 ]
 
 

@@ -16,8 +16,9 @@
 //   warp 0      TMA producer: packed INT4 tiles of X and W (or R) -> smem
 //   warp 1      TMEM owner; in CTA 0 of the pair, one thread issues the MMAs
 //   warps 2..9  unpackers: packed nibbles -> int8 (x16) in the 128-byte
-//               swizzled K-major layout the MMA reads; afterwards the same
-//               warps run the epilogue out of this CTA's TMEM.
+//               swizzled K-major layout the MMA reads; after a tile's last
+//               step the same warps run its epilogue out of this CTA's TMEM
+//               (bf16 tile staged in shared memory, written by TMA stores).
 // The k loop runs K/128 main steps into acc0 followed by ceil(r/128)
 // residual steps into acc1; a residual step reloads the matching activation
 // block and takes R in place of W, so both accumulators use one pipeline.
@@ -54,30 +55,35 @@ struct Args {
   int ldy;
   int32_t* acc0;
   int32_t* acc1;
+  int tiles_m, tiles_n;  // output tiles (BM * cluster rows x BN columns)
 };
 
-// Shared memory: PS packed stages [A | B] written by TMA, US unpacked
-// stages [A | B] read by the MMAs (W4A8: A is consumed straight from the
-// packed stage, already in the MMA layout), per-column scales, barriers.
+// Shared memory: PS packed stages [A | B] written by TMA, US widened stages
+// [A | B] read by the MMAs (W4A8: A is consumed straight from the packed
+// stage, already in the MMA layout), per-warp epilogue scales, barriers.
+// Between the last MMA of a tile and the first widening of the next, the
+// widened ring is idle; the epilogue stages the bf16 output tile there for
+// the TMA store.
 template <int BN, bool A8, int CG>
 struct Layout {
   // ring depths: as deep as shared memory allows, so the MMA issue never
   // waits on the two barrier hops (MMA done -> widening -> MMA)
   static constexpr int PS = (CG == 2) ? 5 : 3;             // packed (TMA) stages
-  static constexpr int US = (CG == 2) ? 4 : (BN == 256 ? 3 : 4);  // unpacked stages
+  static constexpr int US = (CG == 2) ? 4 : (BN == 256 ? 3 : 4);  // widened stages
   static constexpr int BNL = BN / CG;                      // weight rows held by this CTA
   static constexpr int kPkA = A8 ? BM * BK : BM * BK / 2;  // A part of a packed stage
   static constexpr int kPkB = BNL * BK / 2;                // B/R part (packed INT4)
   static constexpr int kPk = kPkA + kPkB;
-  static constexpr int kUnA = A8 ? 0 : BM * BK;            // A part of an unpacked stage
+  static constexpr int kUnA = A8 ? 0 : BM * BK;            // A part of a widened stage
   static constexpr int kUnB = BNL * BK;
   static constexpr int kUn = kUnA + kUnB;
   static constexpr int oUn = 0;
   static constexpr int oPk = oUn + US * kUn;
-  static constexpr int oSw = oPk + PS * kPk;
-  static constexpr int oSr = oSw + BN * 4;
-  static constexpr int oBar = oSr + BN * 4;
-  static constexpr int nBar = 2 * PS + 2 * US + 2;
+  // epilogue scales: each widening warp keeps sw and sr of its BN / 2 columns
+  static constexpr int oScl = oPk + PS * kPk;
+  static constexpr int kSclWarp = 2 * (BN / 2) * 4;
+  static constexpr int oBar = oScl + kUnpackWarps * kSclWarp;
+  static constexpr int nBar = 2 * PS + 2 * US + 3;
   static constexpr int oMisc = oBar + nBar * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;             // slack for 1024-B alignment
@@ -86,8 +92,15 @@ struct Layout {
   // widening work: rows of 64 packed bytes per stage, four 16-byte pieces each
   static constexpr int kRows = (A8 ? 0 : BM) + BNL;
   static constexpr int kPiecesPerThread = kRows * 4 / (kUnpackWarps * 32);
+  // output staging: boxes of 32 rows x 64 bf16 (4 KB, 128-byte swizzle),
+  // (BN / 64) per TMEM lane quadrant, packed into whole widened stages
+  static constexpr int kBoxBytes = 32 * 128;
+  static constexpr int kBoxes = 4 * (BN / 64);
+  static constexpr int kBoxesPerStage = kUn / kBoxBytes;
+  static constexpr int kStgStages = (kBoxes + kBoxesPerStage - 1) / kBoxesPerStage;
   static_assert(kRows * 4 % (kUnpackWarps * 32) == 0, "pieces must divide evenly");
   static_assert(kPk % 1024 == 0 && kUn % 1024 == 0 && oPk % 1024 == 0, "tiles must stay 1024-aligned");
+  static_assert(kUn % kBoxBytes == 0 && kStgStages <= US, "output staging must fit the widened ring");
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
@@ -109,10 +122,21 @@ __device__ __forceinline__ void cta_sync() {
     cluster_sync_all();
 }
 
+// Persistent: the grid holds at most one CTA (pair) per SM (pair of SMs),
+// and CTA (pair) c takes output tiles c, c + G, c + 2G, ... (G = number of
+// CTAs or pairs), M-tile fastest so that concurrent tiles share weight tiles
+// in L2.  The packed and widened rings run on across tile boundaries, so the
+// next tile's operands stream in while the epilogue drains the accumulators.
+//
+// TMEM holds one tile's acc0 and acc1 (2 BN columns); the first MMA of the
+// next tile waits, through the widened-stage barrier, until every widening
+// warp has finished the previous epilogue's TMEM reads (tcgen05.wait::ld ->
+// tcgen05.fence::before_thread_sync -> mbarrier arrive -> MMA warp wait ->
+// tcgen05.fence::after_thread_sync).
 template <int BN, bool A8, bool ACC_OUT, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           const __grid_constant__ CUtensorMap tmR, const Args p) {
+           const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmY, const Args p) {
   using L = Layout<BN, A8, CG>;
   constexpr int PS = L::PS, US = L::US;
   extern __shared__ uint8_t smem_raw[];
@@ -120,21 +144,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::oBar);
   uint64_t* full_pk = bar;              // TMA bytes landed            (tx)
   uint64_t* empty_pk = bar + PS;        // packed stage consumed
-  uint64_t* full_un = bar + 2 * PS;     // unpacked stage written (both CTAs, on CTA 0)
-  uint64_t* empty_un = full_un + US;    // unpacked stage read by the MMAs
-  uint64_t* acc_full = empty_un + US;   // all MMAs complete
+  uint64_t* full_un = bar + 2 * PS;     // widened stage written (both CTAs, on CTA 0)
+  uint64_t* empty_un = full_un + US;    // widened stage read by the MMAs
+  uint64_t* acc_full = empty_un + US;   // all MMAs of a tile complete
   uint64_t* drain = acc_full + 1;       // abort path: MMAs complete
+  uint64_t* stg_done = drain + 1;       // output staging read by the TMA stores
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::oMisc + 4);
-  float* sw_t = reinterpret_cast<float*>(smem + L::oSw);
-  float* sr_t = reinterpret_cast<float*>(smem + L::oSr);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
   const bool leader = (rank == 0);
-  const int n0 = blockIdx.y * BN;                       // output columns of this tile
-  const int nb0 = n0 + (int)rank * L::BNL;              // weight rows this CTA loads
-  const int m0 = blockIdx.x * BM;                       // X rows of this CTA
+  const int cta_tile = (int)blockIdx.x / CG;            // this CTA (pair)'s first tile
+  const int tile_stride = (int)gridDim.x / CG;
+  const int ntiles = p.tiles_m * p.tiles_n;
   const int nsteps = p.nkb + p.nrb;
 
   if (threadIdx.x == 0) {
@@ -150,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    mbar_init(stg_done, kUnpackWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -157,15 +181,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmR);
+    if (!ACC_OUT) tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc<CG>(tmem_slot, L::kTmemCols);
     tmem_relinquish<CG>();
-  }
-  for (int i = threadIdx.x; i < BN; i += blockDim.x) {
-    const int n = n0 + i;
-    sw_t[i] = (n < p.N) ? p.sw[n] : 0.f;
-    sr_t[i] = (n < p.N) ? p.sr[n] : 0.f;
   }
   tc_fence_before();
   cta_sync<CG>();
@@ -175,16 +195,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      for (int step = 0; step < nsteps; ++step) {
-        const int s = step % PS;
-        const uint32_t ph = (step / PS) & 1;
-        if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) break;
-        mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
-        const bool res = step >= p.nkb;
-        const int j = res ? step - p.nkb : step;
-        uint8_t* stage = smem + L::oPk + s * L::kPk;
-        tma_load_2d(stage, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
-        tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
+      int g = 0;  // pipeline step across tiles
+      bool ok = true;
+      for (int t = cta_tile; ok && t < ntiles; t += tile_stride) {
+        const int m0 = ((t % p.tiles_m) * CG + (int)rank) * BM;
+        const int nb0 = (t / p.tiles_m) * BN + (int)rank * L::BNL;
+        for (int step = 0; step < nsteps; ++step, ++g) {
+          const int s = g % PS;
+          const uint32_t ph = (g / PS) & 1;
+          if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
+          const bool res = step >= p.nkb;
+          const int j = res ? step - p.nkb : step;
+          uint8_t* stage = smem + L::oPk + s * L::kPk;
+          tma_load_2d(stage, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
+          tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
+        }
       }
     }
   } else if (warp == 1) {
@@ -197,50 +223,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t pk_base = smem_u32(smem + L::oPk);
       const uint32_t un_base = smem_u32(smem + L::oUn);
       bool ok = true;
-      for (int step = 0; step < nsteps; ++step) {
-        const int u = step % US;
-        const uint32_t uph = (step / US) & 1;
-        const int s = step % PS;
-        const uint32_t ph = (step / PS) & 1;
-        if (!mbar_wait(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
-        if (A8 && !mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
-        tc_fence_after();
-        const bool res = step >= p.nkb;
-        const int j = res ? step - p.nkb : step;
-        const uint32_t d = tmem + (res ? (uint32_t)BN : 0u);
-        const uint64_t da = umma_desc_k_sw128(A8 ? pk_base + s * L::kPk : un_base + u * L::kUn);
-        const uint64_t db = umma_desc_k_sw128(un_base + u * L::kUn + L::kUnA);
-        if (!res) {
+      int g = 0;
+      for (int t = cta_tile; ok && t < ntiles; t += tile_stride) {
+        for (int step = 0; step < nsteps; ++step, ++g) {
+          const int u = g % US;
+          const uint32_t uph = (g / US) & 1;
+          const int s = g % PS;
+          const uint32_t ph = (g / PS) & 1;
+          if (!mbar_wait(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
+          if (A8 && !mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          const bool res = step >= p.nkb;
+          const int j = res ? step - p.nkb : step;
+          const uint32_t d = tmem + (res ? (uint32_t)BN : 0u);
+          const uint64_t da = umma_desc_k_sw128(A8 ? pk_base + s * L::kPk : un_base + u * L::kUn);
+          const uint64_t db = umma_desc_k_sw128(un_base + u * L::kUn + L::kUnA);
+          const int nk = res ? min(BK / 32, (p.rpad - j * BK) / 32) : BK / 32;
           if (elect_one()) {
+            if (nk == BK / 32) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk)
-              umma_i8<CG>(d, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc, (j > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < BK / 32; ++kk)
+                umma_i8<CG>(d, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+            } else {
+              for (int kk = 0; kk < nk; ++kk)
+                umma_i8<CG>(d, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+            }
             umma_commit<CG>(&empty_un[u]);
             if (A8) umma_commit<CG>(&empty_pk[s]);
+            if (step == nsteps - 1) umma_commit<CG>(acc_full);
           }
-        } else {
-          const int nk = min(BK / 32, (p.rpad - j * BK) / 32);
-          if (elect_one()) {
-            for (int kk = 0; kk < nk; ++kk)
-              umma_i8<CG>(d, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc, (j > 0 || kk > 0) ? 1u : 0u);
-            umma_commit<CG>(&empty_un[u]);
-            if (A8) umma_commit<CG>(&empty_pk[s]);
-          }
+          __syncwarp();
         }
-        __syncwarp();
       }
-      if (elect_one()) {
-        if (ok) {
-          umma_commit<CG>(acc_full);
-        } else {
+      if (!ok) {
+        if (elect_one()) {
           umma_commit<1>(drain);
           mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
         }
+        __syncwarp();
       }
-      __syncwarp();
     }
   } else {
-    // ------------------------------------------------------------ unpack
+    // ------------------------------------------------- widening + epilogue
     // Thread ut widens the same rows and pieces in every stage: piece
     // p = ut + 256 i covers row p / 4 (A rows first, then B rows) and packed
     // bytes [16 (p % 4), +16); its 32 int8 land in chunks 2 (p % 4) and
@@ -257,89 +283,184 @@ __global__ void __launch_bounds__(kThreads, 1)
       src_off[i] = (A8 ? L::kPkA : 0) + row * (BK / 2) + q * 16;
       dst_off[i] = row * BK + (((2 * q) ^ (row & 7)) << 4);
     }
-    bool ok = true;
-    for (int step = 0; step < nsteps; ++step) {
-      const int s = step % PS;
-      const uint32_t ph = (step / PS) & 1;
-      const int u = step % US;
-      const uint32_t uph = (step / US) & 1;
-      if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
-      if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
-      const uint8_t* pk = smem + L::oPk + s * L::kPk;
-      uint8_t* un = smem + L::oUn + u * L::kUn;
-      uint4 v[NP];
-#pragma unroll
-      for (int i = 0; i < NP; ++i) v[i] = *reinterpret_cast<const uint4*>(pk + src_off[i]);
-#pragma unroll
-      for (int i = 0; i < NP; ++i) {
-        uint4 lo, hi;
-        widen_run(v[i], lo, hi);
-        *reinterpret_cast<uint4*>(un + dst_off[i]) = lo;
-        *reinterpret_cast<uint4*>(un + (dst_off[i] ^ 16u)) = hi;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&empty_pk[s]);
-        if (leader)
-          mbar_arrive(&full_un[u]);
-        else
-          mbar_arrive_remote(&full_un[u], 0);
-      }
-    }
+    // Epilogue geometry: this warp may read TMEM lanes 32 (warp % 4) .. +31
+    // (rows of its quadrant) and takes half of the BN columns.
+    const int eq = warp & 3;
+    const int eh = (warp - 2) >> 2;
+    constexpr int kHalf = BN / 2;
+    constexpr int kCpl = kHalf / 32;  // scale columns prefetched per lane
+    constexpr int kShift = A8 ? 4 : 8;
+    float* scl = reinterpret_cast<float*>(smem + L::oScl + (warp - 2) * L::kSclWarp);  // [sw | sr]
+    const bool has_r = p.nrb > 0;
 
-    // ---------------------------------------------------------- epilogue
-    if (ok && mbar_wait(acc_full, 0, abort_flag, kDevTimeoutEpilogue)) {
-      tc_fence_after();
-      const int q = warp & 3;          // TMEM lane quadrant this warp may access
-      const int half = (warp - 2) >> 2;
-      const int row = m0 + q * 32 + lane;
-      const bool has_r = p.nrb > 0;
-      constexpr int kShift = A8 ? 4 : 8;
-      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
-        uint32_t r0[32], r1[32];
-        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c;
-        __syncwarp();
-        tmem_ld_32x32b_x32(taddr, r0);
-        if (has_r) tmem_ld_32x32b_x32(taddr + BN, r1);
-        tmem_ld_wait();
-        if (!has_r) {
+    uint32_t stg_mask = 0;   // widened stages holding output boxes not yet released
+    uint32_t stg_parity = 0;
+    bool stg_arrive = false;  // this warp's TMA stores of those boxes were issued
+    auto release_staging = [&]() -> bool {
+      if (stg_mask == 0) return true;
+      if (lane == 0 && stg_arrive) {
+        bulk_wait_read_all();
+        mbar_arrive(stg_done);
+      }
+      stg_arrive = false;
+      const bool r = mbar_wait(stg_done, stg_parity, abort_flag, kDevTimeoutEpilogue);
+      stg_parity ^= 1u;
+      stg_mask = 0;
+      return r;
+    };
+
+    bool ok = true;
+    int g = 0;
+    int it = 0;
+    for (int t = cta_tile; ok && t < ntiles; t += tile_stride, ++it) {
+      const int tm = t % p.tiles_m;
+      const int m0 = (tm * CG + (int)rank) * BM;
+      const int n0 = (t / p.tiles_m) * BN;
+      // prefetch this tile's epilogue scales (consumed after the k loop)
+      float swv[kCpl], srv[kCpl], sxv = 0.f;
+      if (!ACC_OUT) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r1[i] = 0;
+        for (int i = 0; i < kCpl; ++i) {
+          const int n = n0 + eh * kHalf + kCpl * lane + i;
+          swv[i] = (n < p.N) ? __ldg(p.sw + n) : 0.f;
+          srv[i] = (n < p.N) ? __ldg(p.sr + n) : 0.f;
         }
-        if (row >= p.M || n0 + c >= p.N) {
-          // row past M (zero-filled A) or column tile past N: nothing to store
-        } else if (ACC_OUT) {
-          int32_t* o0 = p.acc0 + (size_t)row * p.N + n0 + c;
-          int32_t* o1 = p.acc1 + (size_t)row * p.N + n0 + c;
+        const int row = m0 + eq * 32 + lane;
+        sxv = (row < p.M) ? __ldg(p.sx + row) : 0.f;
+      }
+
+      for (int step = 0; step < nsteps; ++step, ++g) {
+        const int s = g % PS;
+        const uint32_t ph = (g / PS) & 1;
+        const int u = g % US;
+        const uint32_t uph = (g / US) & 1;
+        if ((stg_mask >> u) & 1u) {
+          if (!release_staging()) { ok = false; break; }
+        }
+        if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        const uint8_t* pk = smem + L::oPk + s * L::kPk;
+        uint8_t* un = smem + L::oUn + u * L::kUn;
+        uint4 v[NP];
+#pragma unroll
+        for (int i = 0; i < NP; ++i) v[i] = *reinterpret_cast<const uint4*>(pk + src_off[i]);
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+          uint4 lo, hi;
+          widen_run(v[i], lo, hi);
+          *reinterpret_cast<uint4*>(un + dst_off[i]) = lo;
+          *reinterpret_cast<uint4*>(un + (dst_off[i] ^ 16u)) = hi;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&empty_pk[s]);
+          if (leader)
+            mbar_arrive(&full_un[u]);
+          else
+            mbar_arrive_remote(&full_un[u], 0);
+        }
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      if (!release_staging()) { ok = false; break; }
+      if (!mbar_wait(acc_full, (uint32_t)it & 1u, abort_flag, kDevTimeoutEpilogue)) { ok = false; break; }
+      tc_fence_after();
+      const int row = m0 + eq * 32 + lane;
+      const uint32_t tq = tmem + ((uint32_t)(eq * 32) << 16);
+      if (ACC_OUT) {
+        for (int c = eh * kHalf; c < (eh + 1) * kHalf; c += 32) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tq + (uint32_t)c, r0);
+          if (has_r) tmem_ld_32x32b_x32(tq + (uint32_t)(BN + c), r1);
+          tmem_ld_wait();
+          if (!has_r) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r1[i] = 0;
+          }
+          if (row < p.M && n0 + c < p.N) {
+            int32_t* o0 = p.acc0 + (size_t)row * p.N + n0 + c;
+            int32_t* o1 = p.acc1 + (size_t)row * p.N + n0 + c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              *reinterpret_cast<int4*>(o0 + i) =
+                  make_int4((int)r0[i] >> kShift, (int)r0[i + 1] >> kShift, (int)r0[i + 2] >> kShift,
+                            (int)r0[i + 3] >> kShift);
+              *reinterpret_cast<int4*>(o1 + i) =
+                  make_int4((int)r1[i] >> kShift, (int)r1[i + 1] >> kShift, (int)r1[i + 2] >> kShift,
+                            (int)r1[i + 3] >> kShift);
+            }
+          }
+        }
+        tc_fence_before();
+      } else {
+        // scales of this warp's columns -> its private smem copy
+#pragma unroll
+        for (int i = 0; i < kCpl; ++i) {
+          scl[kCpl * lane + i] = swv[i];
+          scl[kHalf + kCpl * lane + i] = srv[i];
+        }
+        __syncwarp();
+        // output staging: box b = 32 rows x 64 columns of the tile, stored
+        // in widened stage (first stage of the next tile's ring order that
+        // is left for last) + b / kBoxesPerStage
+        const int g_next = g;  // first pipeline step of the next tile
+        auto box_ptr = [&](int b) -> uint8_t* {
+          const int su = (g_next + US - L::kStgStages + b / L::kBoxesPerStage) % US;
+          return smem + L::oUn + su * L::kUn + (b % L::kBoxesPerStage) * L::kBoxBytes;
+        };
+        const float4* sw4 = reinterpret_cast<const float4*>(scl);
+        const float4* sr4 = reinterpret_cast<const float4*>(scl + kHalf);
+        for (int cc = 0; cc < kHalf; cc += 32) {
+          const int c = eh * kHalf + cc;  // tile column of this chunk
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tq + (uint32_t)c, r0);
+          if (has_r) tmem_ld_32x32b_x32(tq + (uint32_t)(BN + c), r1);
+          tmem_ld_wait();
+          if (!has_r) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r1[i] = 0;
+          }
+          uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
-            *reinterpret_cast<int4*>(o0 + i) =
-                make_int4((int)r0[i] >> kShift, (int)r0[i + 1] >> kShift, (int)r0[i + 2] >> kShift,
-                          (int)r0[i + 3] >> kShift);
-            *reinterpret_cast<int4*>(o1 + i) =
-                make_int4((int)r1[i] >> kShift, (int)r1[i + 1] >> kShift, (int)r1[i + 2] >> kShift,
-                          (int)r1[i + 3] >> kShift);
+            const float4 w = sw4[(cc + i) >> 2];
+            const float4 rr = sr4[(cc + i) >> 2];
+            const float y0 = sxv * fmaf(w.x, (float)((int)r0[i] >> kShift), rr.x * (float)((int)r1[i] >> kShift));
+            const float y1 = sxv * fmaf(w.y, (float)((int)r0[i + 1] >> kShift), rr.y * (float)((int)r1[i + 1] >> kShift));
+            const float y2 = sxv * fmaf(w.z, (float)((int)r0[i + 2] >> kShift), rr.z * (float)((int)r1[i + 2] >> kShift));
+            const float y3 = sxv * fmaf(w.w, (float)((int)r0[i + 3] >> kShift), rr.w * (float)((int)r1[i + 3] >> kShift));
+            const __nv_bfloat162 h0 = __floats2bfloat162_rn(y0, y1);
+            const __nv_bfloat162 h1 = __floats2bfloat162_rn(y2, y3);
+            pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h0);
+            pk[(i >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h1);
           }
-        } else {
-          const float sxm = p.sx[row];
-          uint32_t packed[16];
+          // 128-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)
+          uint8_t* bp = box_ptr(eq * (BN / 64) + (c >> 6)) + lane * 128;
+          const int k0 = (c & 32) >> 3;  // first 16-byte chunk of these 32 columns
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float y0 = sxm * fmaf(sw_t[c + i], (float)((int)r0[i] >> kShift),
-                                        sr_t[c + i] * (float)((int)r1[i] >> kShift));
-            const float y1 = sxm * fmaf(sw_t[c + i + 1], (float)((int)r0[i + 1] >> kShift),
-                                        sr_t[c + i + 1] * (float)((int)r1[i + 1] >> kShift));
-            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-            packed[i >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(p.Y + (size_t)row * p.ldy + n0 + c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(bp + (((k0 + k) ^ (lane & 7)) << 4)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int y = m0 + eq * 32;
+#pragma unroll
+          for (int b = 0; b < kHalf / 64; ++b) {
+            const int x = n0 + eh * kHalf + b * 64;
+            if (x < p.N && y < p.M) tma_store_2d(&tmY, box_ptr(eq * (BN / 64) + eh * (kHalf / 64) + b), x, y);
+          }
+          bulk_commit_group();
+        }
+        stg_arrive = true;
+        for (int k = 0; k < L::kStgStages; ++k) stg_mask |= 1u << ((g_next + US - L::kStgStages + k) % US);
       }
     }
+    if (!ACC_OUT && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();

@@ -73,18 +73,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D byte tensor [rows][inner] with row stride `stride` bytes.
+// 2-D tensor [rows][inner] of `dtype` elements with row stride `stride`
+// bytes (inner and box_inner in elements).
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
-              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+              uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {stride};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -181,6 +182,17 @@ void set_smem(K kernel, int bytes) {
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (dev < 64) cached[dev] = sms;
+  return sms;
+}
+
 // ------------------------------------------------------------ GEMM launch
 template <int BN, bool A8, bool ACC, int CG>
 cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, cudaStream_t st) {
@@ -191,6 +203,11 @@ cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args&
                 : make_map(&tmA, Xq, (uint64_t)a.K / 2, (uint64_t)a.M, (uint64_t)a.K / 2, 64, 128,
                            CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!okm) return cudaErrorInvalidValue;
+  // output: bf16 [M][N] with row stride ldy, boxes of 32 rows x 64 columns
+  CUtensorMap tmY = tmA;
+  if (!ACC && !make_map(&tmY, a.Y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.ldy * 2, 64, 32,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+    return cudaErrorInvalidValue;
   // weight maps by box rows: [0] 128, [1] 256 (BN / CG rows per CTA)
   const int bi = (BN / CG == 256) ? 1 : 0;
   static_assert(BN / CG == 128 || BN / CG == 256, "weight box rows");
@@ -202,8 +219,13 @@ cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args&
     set_smem(kern, Lay::kAlloc);
     attr_set[dev] = 1;
   }
-  const int mtiles = (a.M + serq::tc::BM * CG - 1) / (serq::tc::BM * CG);
-  dim3 grid(mtiles * CG, (a.N + BN - 1) / BN);
+  // persistent: one CTA (pair) per SM (pair of SMs), tiles strided over them
+  serq::tc::Args ap = a;
+  ap.tiles_m = (a.M + serq::tc::BM * CG - 1) / (serq::tc::BM * CG);
+  ap.tiles_n = (a.N + BN - 1) / BN;
+  const long ntiles = (long)ap.tiles_m * ap.tiles_n;
+  const long slots = sm_count() / CG;
+  dim3 grid((unsigned)((ntiles < slots ? ntiles : slots) * CG), 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(serq::tc::kThreads);
@@ -216,7 +238,7 @@ cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args&
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[bi], L->tmR[bi], a);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[bi], L->tmR[bi], tmY, ap);
 }
 
 // W4A4 on CTA pairs with the activations in tensor memory, 256 x 192 tiles.
@@ -251,16 +273,6 @@ cudaError_t launch_tc_ta(const serq_layer* L, const void* Xq, const serq::tc::Ar
   return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[2], L->tmR[2], a);
 }
 
-int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && cached[dev]) return cached[dev];
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (dev < 64) cached[dev] = sms;
-  return sms;
-}
 
 template <bool A8, bool ACC>
 cudaError_t dispatch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, serq_algo algo,
