@@ -66,10 +66,23 @@ struct Args {
 // the TMA store.
 template <int BN, bool A8, int CG>
 struct Layout {
-  // ring depths: as deep as shared memory allows, so the MMA issue never
-  // waits on the two barrier hops (MMA done -> widening -> MMA)
-  static constexpr int PS = (CG == 2) ? 5 : 3;             // packed (TMA) stages
-  static constexpr int US = (CG == 2) ? 4 : (BN == 256 ? 3 : 4);  // widened stages
+  // Ring depths, as deep as shared memory allows.  The widening warps form
+  // G groups that take turns on the pipeline steps (group g % G widens step
+  // g), so G steps are widened at once and each step's shared-memory round
+  // trip and proxy fence overlap the others'.
+  //
+  // Parity waits need the waiter to be at most one phase ahead of the
+  // barrier.  A group owns fixed widened slots (G divides US), so it waits on
+  // their phases in order.  Packed slots are shared between groups; a group
+  // waits for its packed slot only after its widened slot is free, which
+  // means the MMAs of step g - US, and so the widening of every step up to
+  // g - US >= g - PS, are complete: the slot's previous phase is behind it.
+  static constexpr bool kBig1 = (CG == 1 && BN == 256);
+  static constexpr int PS = kBig1 ? 3 : ((CG == 2 && A8) ? 6 : 5);  // packed (TMA) stages
+  static constexpr int US = kBig1 ? 3 : 4;                             // widened stages
+  static constexpr int G = kBig1 ? 1 : 4;
+  static constexpr int kGroupWarps = kUnpackWarps / G;
+  static_assert(US % G == 0 && PS >= US && kUnpackWarps % G == 0, "group ring ownership");
   static constexpr int BNL = BN / CG;                      // weight rows held by this CTA
   static constexpr int kPkA = A8 ? BM * BK : BM * BK / 2;  // A part of a packed stage
   static constexpr int kPkB = BNL * BK / 2;                // B/R part (packed INT4)
@@ -83,7 +96,7 @@ struct Layout {
   static constexpr int oScl = oPk + PS * kPk;
   static constexpr int kSclWarp = 2 * (BN / 2) * 4;
   static constexpr int oBar = oScl + kUnpackWarps * kSclWarp;
-  static constexpr int nBar = 2 * PS + 2 * US + 3;
+  static constexpr int nBar = 2 * PS + 2 * US + 4;
   static constexpr int oMisc = oBar + nBar * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;             // slack for 1024-B alignment
@@ -91,14 +104,14 @@ struct Layout {
   static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
   // widening work: rows of 64 packed bytes per stage, four 16-byte pieces each
   static constexpr int kRows = (A8 ? 0 : BM) + BNL;
-  static constexpr int kPiecesPerThread = kRows * 4 / (kUnpackWarps * 32);
+  static constexpr int kPiecesPerThread = kRows * 4 / (kGroupWarps * 32);
   // output staging: boxes of 32 rows x 64 bf16 (4 KB, 128-byte swizzle),
   // (BN / 64) per TMEM lane quadrant, packed into whole widened stages
   static constexpr int kBoxBytes = 32 * 128;
   static constexpr int kBoxes = 4 * (BN / 64);
   static constexpr int kBoxesPerStage = kUn / kBoxBytes;
   static constexpr int kStgStages = (kBoxes + kBoxesPerStage - 1) / kBoxesPerStage;
-  static_assert(kRows * 4 % (kUnpackWarps * 32) == 0, "pieces must divide evenly");
+  static_assert(kRows * 4 % (kGroupWarps * 32) == 0, "pieces must divide evenly");
   static_assert(kPk % 1024 == 0 && kUn % 1024 == 0 && oPk % 1024 == 0, "tiles must stay 1024-aligned");
   static_assert(kUn % kBoxBytes == 0 && kStgStages <= US, "output staging must fit the widened ring");
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -129,10 +142,9 @@ __device__ __forceinline__ void cta_sync() {
 // next tile's operands stream in while the epilogue drains the accumulators.
 //
 // TMEM holds one tile's acc0 and acc1 (2 BN columns); the first MMA of the
-// next tile waits, through the widened-stage barrier, until every widening
-// warp has finished the previous epilogue's TMEM reads (tcgen05.wait::ld ->
-// tcgen05.fence::before_thread_sync -> mbarrier arrive -> MMA warp wait ->
-// tcgen05.fence::after_thread_sync).
+// next tile waits on tmem_empty until every epilogue warp of the pair has
+// finished its TMEM reads (tcgen05.wait::ld -> tcgen05.fence::before_thread_sync
+// -> mbarrier arrive -> MMA warp wait -> tcgen05.fence::after_thread_sync).
 template <int BN, bool A8, bool ACC_OUT, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -149,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = empty_un + US;   // all MMAs of a tile complete
   uint64_t* drain = acc_full + 1;       // abort path: MMAs complete
   uint64_t* stg_done = drain + 1;       // output staging read by the TMA stores
+  uint64_t* tmem_empty = stg_done + 1;  // (CTA 0) every epilogue warp of the pair read its TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::oMisc + 4);
 
@@ -161,19 +174,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nsteps = p.nkb + p.nrb;
 
   if (threadIdx.x == 0) {
-    // full_un (on CTA 0) collects one arrival per widening warp of every
-    // CTA of the pair.
+    // full_un (on CTA 0) collects one arrival per widening warp of the
+    // step's group in every CTA of the pair.
     for (int s = 0; s < PS; ++s) {
       mbar_init(&full_pk[s], 1);
-      mbar_init(&empty_pk[s], kUnpackWarps + (A8 ? 1 : 0));
+      mbar_init(&empty_pk[s], L::kGroupWarps + (A8 ? 1 : 0));
     }
     for (int s = 0; s < US; ++s) {
-      mbar_init(&full_un[s], kUnpackWarps * CG);
+      mbar_init(&full_un[s], L::kGroupWarps * CG);
       mbar_init(&empty_un[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     mbar_init(stg_done, kUnpackWarps);
+    mbar_init(tmem_empty, kUnpackWarps * CG);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -224,7 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t un_base = smem_u32(smem + L::oUn);
       bool ok = true;
       int g = 0;
-      for (int t = cta_tile; ok && t < ntiles; t += tile_stride) {
+      int it = 0;
+      for (int t = cta_tile; ok && t < ntiles; t += tile_stride, ++it) {
+        // the accumulators are rewritten only after the previous tile's
+        // epilogue has read them in both CTAs
+        if (it > 0 && !mbar_wait<CG == 2>(tmem_empty, (uint32_t)(it - 1) & 1u, abort_flag, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
         for (int step = 0; step < nsteps; ++step, ++g) {
           const int u = g % US;
           const uint32_t uph = (g / US) & 1;
@@ -267,22 +288,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------- widening + epilogue
-    // Thread ut widens the same rows and pieces in every stage: piece
-    // p = ut + 256 i covers row p / 4 (A rows first, then B rows) and packed
+    // Group wg widens the steps g with g % G == wg.  Thread ut of
+    // the group widens the same rows and pieces in each of its steps: piece
+    // p = ut + 32 kGroupWarps i covers row p / 4 (A rows first, then B rows) and packed
     // bytes [16 (p % 4), +16); its 32 int8 land in chunks 2 (p % 4) and
     // 2 (p % 4) + 1 of the 128-byte row, swizzled by row % 8.  Four
     // consecutive threads cover one row, so a warp reads 512 contiguous
     // bytes and each quarter-warp store fills all 32 banks.
-    const int ut = threadIdx.x - 64;  // 0 .. 255
+    constexpr int kGroupWarps = L::kGroupWarps;
+    const int wg = (warp - 2) / kGroupWarps;
+    const int ut = threadIdx.x - 64 - wg * kGroupWarps * 32;
+    // Piece i of thread ut sits kRowStep rows below piece i - 1: same
+    // 16-byte column q and the same swizzle phase (kRowStep % 8 == 0).
     constexpr int NP = L::kPiecesPerThread;
-    uint32_t src_off[NP], dst_off[NP];
-#pragma unroll
-    for (int i = 0; i < NP; ++i) {
-      const int pc = ut + i * kUnpackWarps * 32;
-      const int row = pc >> 2, q = pc & 3;
-      src_off[i] = (A8 ? L::kPkA : 0) + row * (BK / 2) + q * 16;
-      dst_off[i] = row * BK + (((2 * q) ^ (row & 7)) << 4);
-    }
+    constexpr int kRowStep = kGroupWarps * 32 / 4;
+    static_assert(kRowStep % 8 == 0, "pieces of a thread share the swizzle phase");
+    const int urow = ut >> 2, uq = ut & 3;
+    const uint32_t src0 = (A8 ? L::kPkA : 0) + urow * (BK / 2) + uq * 16;
+    const uint32_t dst0 = urow * BK + (((2 * uq) ^ (urow & 7)) << 4);
     // Epilogue geometry: this warp may read TMEM lanes 32 (warp % 4) .. +31
     // (rows of its quadrant) and takes half of the BN columns.
     const int eq = warp & 3;
@@ -293,16 +316,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* scl = reinterpret_cast<float*>(smem + L::oScl + (warp - 2) * L::kSclWarp);  // [sw | sr]
     const bool has_r = p.nrb > 0;
 
-    uint32_t stg_mask = 0;   // widened stages holding output boxes not yet released
+    // Widened stages holding output boxes whose TMA stores may still read
+    // them; every widening warp arrives on stg_done once its own stores have
+    // read their sources.
+    uint32_t stg_mask = 0;
     uint32_t stg_parity = 0;
-    bool stg_arrive = false;  // this warp's TMA stores of those boxes were issued
     auto release_staging = [&]() -> bool {
       if (stg_mask == 0) return true;
-      if (lane == 0 && stg_arrive) {
-        bulk_wait_read_all();
-        mbar_arrive(stg_done);
-      }
-      stg_arrive = false;
       const bool r = mbar_wait(stg_done, stg_parity, abort_flag, kDevTimeoutEpilogue);
       stg_parity ^= 1u;
       stg_mask = 0;
@@ -330,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       for (int step = 0; step < nsteps; ++step, ++g) {
+        if (g % L::G != wg) continue;
         const int s = g % PS;
         const uint32_t ph = (g / PS) & 1;
         const int u = g % US;
@@ -337,19 +358,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((stg_mask >> u) & 1u) {
           if (!release_staging()) { ok = false; break; }
         }
-        if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        // widened slot first: see the ring notes in Layout
         if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
         const uint8_t* pk = smem + L::oPk + s * L::kPk;
         uint8_t* un = smem + L::oUn + u * L::kUn;
-        uint4 v[NP];
+        constexpr int NB = NP < 8 ? NP : 8;  // pieces in registers at a time
+        static_assert(NP % NB == 0, "pieces come in whole batches");
 #pragma unroll
-        for (int i = 0; i < NP; ++i) v[i] = *reinterpret_cast<const uint4*>(pk + src_off[i]);
+        for (int b = 0; b < NP; b += NB) {
+          uint4 v[NB];
 #pragma unroll
-        for (int i = 0; i < NP; ++i) {
-          uint4 lo, hi;
-          widen_run(v[i], lo, hi);
-          *reinterpret_cast<uint4*>(un + dst_off[i]) = lo;
-          *reinterpret_cast<uint4*>(un + (dst_off[i] ^ 16u)) = hi;
+          for (int i = 0; i < NB; ++i)
+            v[i] = *reinterpret_cast<const uint4*>(pk + src0 + (b + i) * kRowStep * (BK / 2));
+#pragma unroll
+          for (int i = 0; i < NB; ++i) {
+            uint4 lo, hi;
+            widen_run(v[i], lo, hi);
+            const uint32_t d = dst0 + (b + i) * kRowStep * BK;
+            *reinterpret_cast<uint4*>(un + d) = lo;
+            *reinterpret_cast<uint4*>(un + (d ^ 16u)) = hi;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -394,6 +423,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(tmem_empty);
+          else
+            mbar_arrive_remote(tmem_empty, 0);
+        }
       } else {
         // scales of this warp's columns -> its private smem copy
 #pragma unroll
@@ -412,42 +448,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         const float4* sw4 = reinterpret_cast<const float4*>(scl);
         const float4* sr4 = reinterpret_cast<const float4*>(scl + kHalf);
-        for (int cc = 0; cc < kHalf; cc += 32) {
-          const int c = eh * kHalf + cc;  // tile column of this chunk
-          uint32_t r0[32], r1[32];
-          tmem_ld_32x32b_x32(tq + (uint32_t)c, r0);
-          if (has_r) tmem_ld_32x32b_x32(tq + (uint32_t)(BN + c), r1);
+        for (int cc = 0; cc < kHalf; cc += 16) {
+          const int c = eh * kHalf + cc;  // tile column of this 16-column chunk
+          uint32_t r0[16], r1[16];
+          tmem_ld_32x32b_x16(tq + (uint32_t)c, r0);
+          if (has_r) tmem_ld_32x32b_x16(tq + (uint32_t)(BN + c), r1);
           tmem_ld_wait();
           if (!has_r) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r1[i] = 0;
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 w = sw4[(cc + i) >> 2];
-            const float4 rr = sr4[(cc + i) >> 2];
-            const float y0 = sxv * fmaf(w.x, (float)((int)r0[i] >> kShift), rr.x * (float)((int)r1[i] >> kShift));
-            const float y1 = sxv * fmaf(w.y, (float)((int)r0[i + 1] >> kShift), rr.y * (float)((int)r1[i + 1] >> kShift));
-            const float y2 = sxv * fmaf(w.z, (float)((int)r0[i + 2] >> kShift), rr.z * (float)((int)r1[i + 2] >> kShift));
-            const float y3 = sxv * fmaf(w.w, (float)((int)r0[i + 3] >> kShift), rr.w * (float)((int)r1[i + 3] >> kShift));
-            const __nv_bfloat162 h0 = __floats2bfloat162_rn(y0, y1);
-            const __nv_bfloat162 h1 = __floats2bfloat162_rn(y2, y3);
-            pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h0);
-            pk[(i >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h1);
+            for (int i = 0; i < 16; ++i) r1[i] = 0;
           }
           // 128-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)
           uint8_t* bp = box_ptr(eq * (BN / 64) + (c >> 6)) + lane * 128;
-          const int k0 = (c & 32) >> 3;  // first 16-byte chunk of these 32 columns
+          const int k0 = (c & 63) >> 3;  // first 16-byte chunk of these 16 columns
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(bp + (((k0 + k) ^ (lane & 7)) << 4)) =
-                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          for (int k = 0; k < 2; ++k) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 8; i += 4) {
+              const int e = 8 * k + i;
+              const float4 w = sw4[(cc + e) >> 2];
+              const float4 rr = sr4[(cc + e) >> 2];
+              const float y0 = sxv * fmaf(w.x, (float)((int)r0[e] >> kShift), rr.x * (float)((int)r1[e] >> kShift));
+              const float y1 = sxv * fmaf(w.y, (float)((int)r0[e + 1] >> kShift), rr.y * (float)((int)r1[e + 1] >> kShift));
+              const float y2 = sxv * fmaf(w.z, (float)((int)r0[e + 2] >> kShift), rr.z * (float)((int)r1[e + 2] >> kShift));
+              const float y3 = sxv * fmaf(w.w, (float)((int)r0[e + 3] >> kShift), rr.w * (float)((int)r1[e + 3] >> kShift));
+              const __nv_bfloat162 h0 = __floats2bfloat162_rn(y0, y1);
+              const __nv_bfloat162 h1 = __floats2bfloat162_rn(y2, y3);
+              pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h0);
+              pk[(i >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h1);
+            }
+            *reinterpret_cast<uint4*>(bp + (((k0 + k) ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
         }
         tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
+          if (leader)
+            mbar_arrive(tmem_empty);
+          else
+            mbar_arrive_remote(tmem_empty, 0);
           const int y = m0 + eq * 32;
 #pragma unroll
           for (int b = 0; b < kHalf / 64; ++b) {
@@ -455,8 +496,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (x < p.N && y < p.M) tma_store_2d(&tmY, box_ptr(eq * (BN / 64) + eh * (kHalf / 64) + b), x, y);
           }
           bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(stg_done);
         }
-        stg_arrive = true;
         for (int k = 0; k < L::kStgStages; ++k) stg_mask |= 1u << ((g_next + US - L::kStgStages + k) % US);
       }
     }
@@ -502,24 +544,31 @@ namespace tc {
 // Warps: 0 TMA, 1 TMEM owner / MMA issue (CTA 0), 4..7 widen the 128
 // activation rows of this CTA into TMEM (warp w writes TMEM lanes
 // 32 (w % 4) .. +31, one row per thread), 2, 3, 8, 9 widen this CTA's BN/2
-// weight rows into shared memory; all eight run the epilogue.
+// weight rows into shared memory; all eight run the epilogue, which stages
+// the bf16 tile in a shared-memory area of its own (freed by the activation
+// stages' absence) and writes it with TMA stores.
 // The packed activation tile arrives with the 64-byte TMA swizzle, so the
 // per-thread row reads hit distinct banks.
 template <int BN>
 struct LayoutTA {
   static constexpr int CG = 2;
   static constexpr int BNL = BN / 2;                  // weight rows per CTA
-  static constexpr int PS = 6;                        // packed stages
+  static constexpr int PS = 8;                        // packed stages
   static constexpr int US = 4;                        // widened stages (smem B + TMEM A)
   static constexpr int kPkA = BM * BK / 2;            // 8 KB, 64-byte swizzled
   static constexpr int kPkB = BNL * BK / 2;
   static constexpr int kPk = kPkA + kPkB;
   static constexpr int kUn = BNL * BK;                // widened weight rows
+  // output staging: boxes of 32 rows x 32 bf16 (2 KB, 64-byte swizzle), BN / 32
+  // per TMEM lane quadrant; each epilogue warp owns the boxes it writes
+  static constexpr int kBoxBytes = 32 * 64;
+  static constexpr int kBoxes = 4 * (BN / 32);
   static constexpr int oUn = 0;
   static constexpr int oPk = oUn + US * kUn;
-  static constexpr int oSw = oPk + PS * kPk;
-  static constexpr int oSr = oSw + BN * 4;
-  static constexpr int oBar = oSr + BN * 4;
+  static constexpr int oStg = oPk + PS * kPk;
+  static constexpr int oScl = oStg + kBoxes * kBoxBytes;
+  static constexpr int kSclWarp = 2 * (BN / 2) * 4;  // sw and sr of a warp's BN / 2 columns
+  static constexpr int oBar = oScl + kUnpackWarps * kSclWarp;
   static constexpr int nBar = 2 * PS + 2 * US + 2;
   static constexpr int oMisc = oBar + nBar * 8;
   static constexpr int kBytes = oMisc + 16;
@@ -529,15 +578,18 @@ struct LayoutTA {
   static constexpr uint32_t kTmemA = 2 * BN;          // first activation stage column
   static constexpr int kPiecesB = BNL * 4 / 128;      // per weight-widening thread
   static_assert(2 * BN + US * (BK / 4) <= 512, "TMEM budget");
-  static_assert(BNL * 4 % 128 == 0, "weight pieces must divide evenly");
-  static_assert(kPk % 1024 == 0 && kUn % 1024 == 0, "tiles must stay 1024-aligned");
+  static_assert(BNL * 4 % 128 == 0 && BN % 64 == 0, "weight pieces must divide evenly");
+  static_assert(kPk % 1024 == 0 && kUn % 1024 == 0 && oStg % 1024 == 0, "tiles must stay 1024-aligned");
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
+// Persistent like k_gemm: CTA pair c takes tiles c, c + G, ... (M-tile
+// fastest), the rings run on across tiles, and the first MMA of a tile waits
+// through the widened-stage barrier for the previous epilogue's TMEM reads.
 template <int BN, bool ACC_OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_ta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmR, const Args p) {
+              const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmY, const Args p) {
   using L = LayoutTA<BN>;
   constexpr int PS = L::PS, US = L::US;
   extern __shared__ uint8_t smem_raw[];
@@ -551,15 +603,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::oMisc + 4);
-  float* sw_t = reinterpret_cast<float*>(smem + L::oSw);
-  float* sr_t = reinterpret_cast<float*>(smem + L::oSr);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = (rank == 0);
-  const int n0 = blockIdx.y * BN;
-  const int nb0 = n0 + (int)rank * L::BNL;
-  const int m0 = blockIdx.x * BM;
+  const int cta_tile = (int)blockIdx.x / 2;
+  const int tile_stride = (int)gridDim.x / 2;
+  const int ntiles = p.tiles_m * p.tiles_n;
   const int nsteps = p.nkb + p.nrb;
 
   if (threadIdx.x == 0) {
@@ -580,15 +630,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmR);
+    if (!ACC_OUT) tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc<2>(tmem_slot, L::kTmemCols);
     tmem_relinquish<2>();
-  }
-  for (int i = threadIdx.x; i < BN; i += blockDim.x) {
-    const int n = n0 + i;
-    sw_t[i] = (n < p.N) ? p.sw[n] : 0.f;
-    sr_t[i] = (n < p.N) ? p.sr[n] : 0.f;
   }
   tc_fence_before();
   cluster_sync_all();
@@ -598,16 +644,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      for (int step = 0; step < nsteps; ++step) {
-        const int s = step % PS;
-        const uint32_t ph = (step / PS) & 1;
-        if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) break;
-        mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
-        const bool res = step >= p.nkb;
-        const int j = res ? step - p.nkb : step;
-        uint8_t* stage = smem + L::oPk + s * L::kPk;
-        tma_load_2d(stage, &tmA, &full_pk[s], j * (BK / 2), m0);
-        tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
+      int g = 0;
+      bool ok = true;
+      for (int t = cta_tile; ok && t < ntiles; t += tile_stride) {
+        const int m0 = ((t % p.tiles_m) * 2 + (int)rank) * BM;
+        const int nb0 = (t / p.tiles_m) * BN + (int)rank * L::BNL;
+        for (int step = 0; step < nsteps; ++step, ++g) {
+          const int s = g % PS;
+          const uint32_t ph = (g / PS) & 1;
+          if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
+          const bool res = step >= p.nkb;
+          const int j = res ? step - p.nkb : step;
+          uint8_t* stage = smem + L::oPk + s * L::kPk;
+          tma_load_2d(stage, &tmA, &full_pk[s], j * (BK / 2), m0);
+          tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
+        }
       }
     }
   } else if (warp == 1) {
@@ -616,36 +668,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = umma_idesc_i8(BM * 2, BN);
       const uint32_t un_base = smem_u32(smem + L::oUn);
       bool ok = true;
-      for (int step = 0; step < nsteps; ++step) {
-        const int u = step % US;
-        const uint32_t uph = (step / US) & 1;
-        if (!mbar_wait(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
-        tc_fence_after();
-        const bool res = step >= p.nkb;
-        const int j = res ? step - p.nkb : step;
-        const uint32_t d = tmem + (res ? (uint32_t)BN : 0u);
-        const uint32_t a = tmem + L::kTmemA + (uint32_t)(u * (BK / 4));
-        const uint64_t db = umma_desc_k_sw128(un_base + u * L::kUn);
-        const int nk = res ? min(BK / 32, (p.rpad - j * BK) / 32) : BK / 32;
-        if (elect_one()) {
-          for (int kk = 0; kk < nk; ++kk)
-            umma_i8_ts<2>(d, a + (uint32_t)(kk * 8), db + (uint64_t)(2 * kk), idesc, (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit<2>(&empty_un[u]);
+      int g = 0;
+      for (int t = cta_tile; ok && t < ntiles; t += tile_stride) {
+        for (int step = 0; step < nsteps; ++step, ++g) {
+          const int u = g % US;
+          const uint32_t uph = (g / US) & 1;
+          if (!mbar_wait(&full_un[u], uph, abort_flag, kDevTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          const bool res = step >= p.nkb;
+          const int j = res ? step - p.nkb : step;
+          const uint32_t d = tmem + (res ? (uint32_t)BN : 0u);
+          const uint32_t a = tmem + L::kTmemA + (uint32_t)(u * (BK / 4));
+          const uint64_t db = umma_desc_k_sw128(un_base + u * L::kUn);
+          const int nk = res ? min(BK / 32, (p.rpad - j * BK) / 32) : BK / 32;
+          if (elect_one()) {
+            if (nk == BK / 32) {
+#pragma unroll
+              for (int kk = 0; kk < BK / 32; ++kk)
+                umma_i8_ts<2>(d, a + (uint32_t)(kk * 8), db + (uint64_t)(2 * kk), idesc,
+                              (j > 0 || kk > 0) ? 1u : 0u);
+            } else {
+              for (int kk = 0; kk < nk; ++kk)
+                umma_i8_ts<2>(d, a + (uint32_t)(kk * 8), db + (uint64_t)(2 * kk), idesc,
+                              (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit<2>(&empty_un[u]);
+            if (step == nsteps - 1) umma_commit<2>(acc_full);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
-      if (elect_one()) {
-        if (ok) {
-          umma_commit<2>(acc_full);
-        } else {
+      if (!ok) {
+        if (elect_one()) {
           umma_commit<1>(drain);
           mbar_wait(drain, 0, nullptr, kDevTimeoutMma);
         }
+        __syncwarp();
       }
-      __syncwarp();
     }
   } else {
-    // ----------------------------------------------------------- widening
+    // ------------------------------------------------- widening + epilogue
     const bool act = (warp >= 4 && warp <= 7);
     const int q = warp & 3;                            // TMEM lane quadrant
     const int arow = q * 32 + lane;                    // activation row (act warps)
@@ -662,103 +724,170 @@ __global__ void __launch_bounds__(kThreads, 1)
       src_off[i] = L::kPkA + row * (BK / 2) + c * 16;
       dst_off[i] = row * BK + (((2 * c) ^ (row & 7)) << 4);
     }
+    // epilogue geometry: TMEM lanes of quadrant q, columns [eh BN/2, +BN/2)
+    const int eh = (warp - 2) >> 2;
+    constexpr int kHalf = BN / 2;
+    constexpr int kCpl = kHalf / 32;
+    constexpr int kShift = 8;
+    float* scl = reinterpret_cast<float*>(smem + L::oScl + (warp - 2) * L::kSclWarp);  // [sw | sr]
+    const bool has_r = p.nrb > 0;
+    bool stores_pending = false;
+
     bool ok = true;
-    for (int step = 0; step < nsteps; ++step) {
-      const int s = step % PS;
-      const uint32_t ph = (step / PS) & 1;
-      const int u = step % US;
-      const uint32_t uph = (step / US) & 1;
-      if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
-      if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
-      const uint8_t* pk = smem + L::oPk + s * L::kPk;
-      if (act) {
-        uint32_t r[32];
+    int g = 0;
+    int it = 0;
+    for (int t = cta_tile; ok && t < ntiles; t += tile_stride, ++it) {
+      const int m0 = ((t % p.tiles_m) * 2 + (int)rank) * BM;
+      const int n0 = (t / p.tiles_m) * BN;
+      float swv[kCpl], srv[kCpl], sxv = 0.f;
+      if (!ACC_OUT) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(pk + a_off[c]);
-          uint4 lo, hi;
-          widen_run(v, lo, hi);
-          r[8 * c + 0] = lo.x; r[8 * c + 1] = lo.y; r[8 * c + 2] = lo.z; r[8 * c + 3] = lo.w;
-          r[8 * c + 4] = hi.x; r[8 * c + 5] = hi.y; r[8 * c + 6] = hi.z; r[8 * c + 7] = hi.w;
+        for (int i = 0; i < kCpl; ++i) {
+          const int n = n0 + eh * kHalf + 32 * i + lane;
+          swv[i] = (n < p.N) ? __ldg(p.sw + n) : 0.f;
+          srv[i] = (n < p.N) ? __ldg(p.sr + n) : 0.f;
         }
-        tmem_st_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + L::kTmemA + (uint32_t)(u * (BK / 4)), r);
-        tmem_st_wait();
+        const int row = m0 + q * 32 + lane;
+        sxv = (row < p.M) ? __ldg(p.sx + row) : 0.f;
+      }
+      for (int step = 0; step < nsteps; ++step, ++g) {
+        const int s = g % PS;
+        const uint32_t ph = (g / PS) & 1;
+        const int u = g % US;
+        const uint32_t uph = (g / US) & 1;
+        if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        const uint8_t* pk = smem + L::oPk + s * L::kPk;
+        if (act) {
+          uint32_t r[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(pk + a_off[c]);
+            uint4 lo, hi;
+            widen_run(v, lo, hi);
+            r[8 * c + 0] = lo.x; r[8 * c + 1] = lo.y; r[8 * c + 2] = lo.z; r[8 * c + 3] = lo.w;
+            r[8 * c + 4] = hi.x; r[8 * c + 5] = hi.y; r[8 * c + 6] = hi.z; r[8 * c + 7] = hi.w;
+          }
+          tmem_st_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + L::kTmemA + (uint32_t)(u * (BK / 4)), r);
+          tmem_st_wait();
+          tc_fence_before();
+        } else {
+          uint8_t* un = smem + L::oUn + u * L::kUn;
+          uint4 v[NPB];
+#pragma unroll
+          for (int i = 0; i < NPB; ++i) v[i] = *reinterpret_cast<const uint4*>(pk + src_off[i]);
+#pragma unroll
+          for (int i = 0; i < NPB; ++i) {
+            uint4 lo, hi;
+            widen_run(v[i], lo, hi);
+            *reinterpret_cast<uint4*>(un + dst_off[i]) = lo;
+            *reinterpret_cast<uint4*>(un + (dst_off[i] ^ 16u)) = hi;
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&empty_pk[s]);
+          if (leader)
+            mbar_arrive(&full_un[u]);
+          else
+            mbar_arrive_remote(&full_un[u], 0);
+        }
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      if (!mbar_wait(acc_full, (uint32_t)it & 1u, abort_flag, kDevTimeoutEpilogue)) { ok = false; break; }
+      tc_fence_after();
+      const int row = m0 + q * 32 + lane;
+      const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+      if (ACC_OUT) {
+        for (int c = eh * kHalf; c < (eh + 1) * kHalf; c += 32) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tq + (uint32_t)c, r0);
+          if (has_r) tmem_ld_32x32b_x32(tq + (uint32_t)(BN + c), r1);
+          tmem_ld_wait();
+          if (!has_r) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r1[i] = 0;
+          }
+          if (row < p.M && n0 + c < p.N) {
+            int32_t* o0 = p.acc0 + (size_t)row * p.N + n0 + c;
+            int32_t* o1 = p.acc1 + (size_t)row * p.N + n0 + c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              *reinterpret_cast<int4*>(o0 + i) =
+                  make_int4((int)r0[i] >> kShift, (int)r0[i + 1] >> kShift, (int)r0[i + 2] >> kShift,
+                            (int)r0[i + 3] >> kShift);
+              *reinterpret_cast<int4*>(o1 + i) =
+                  make_int4((int)r1[i] >> kShift, (int)r1[i + 1] >> kShift, (int)r1[i + 2] >> kShift,
+                            (int)r1[i + 3] >> kShift);
+            }
+          }
+        }
         tc_fence_before();
       } else {
-        uint8_t* un = smem + L::oUn + u * L::kUn;
-        uint4 v[NPB];
-#pragma unroll
-        for (int i = 0; i < NPB; ++i) v[i] = *reinterpret_cast<const uint4*>(pk + src_off[i]);
-#pragma unroll
-        for (int i = 0; i < NPB; ++i) {
-          uint4 lo, hi;
-          widen_run(v[i], lo, hi);
-          *reinterpret_cast<uint4*>(un + dst_off[i]) = lo;
-          *reinterpret_cast<uint4*>(un + (dst_off[i] ^ 16u)) = hi;
+        // this warp's staging boxes were read by its previous TMA stores
+        if (stores_pending) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
         }
-        fence_proxy_async_smem();
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&empty_pk[s]);
-        if (leader)
-          mbar_arrive(&full_un[u]);
-        else
-          mbar_arrive_remote(&full_un[u], 0);
-      }
-    }
-
-    // ---------------------------------------------------------- epilogue
-    if (ok && mbar_wait(acc_full, 0, abort_flag, kDevTimeoutEpilogue)) {
-      tc_fence_after();
-      const int half = (warp - 2) >> 2;
-      const int row = m0 + q * 32 + lane;
-      const bool has_r = p.nrb > 0;
-      constexpr int kShift = 8;
-      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
-        uint32_t r0[32], r1[32];
-        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c;
+#pragma unroll
+        for (int i = 0; i < kCpl; ++i) {
+          scl[32 * i + lane] = swv[i];
+          scl[kHalf + 32 * i + lane] = srv[i];
+        }
         __syncwarp();
-        tmem_ld_32x32b_x32(taddr, r0);
-        if (has_r) tmem_ld_32x32b_x32(taddr + BN, r1);
-        tmem_ld_wait();
-        if (!has_r) {
+        const float4* sw4 = reinterpret_cast<const float4*>(scl);
+        const float4* sr4 = reinterpret_cast<const float4*>(scl + kHalf);
+        for (int cc = 0; cc < kHalf; cc += 32) {
+          const int c = eh * kHalf + cc;  // tile column of this chunk = one box
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tq + (uint32_t)c, r0);
+          if (has_r) tmem_ld_32x32b_x32(tq + (uint32_t)(BN + c), r1);
+          tmem_ld_wait();
+          if (!has_r) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r1[i] = 0;
-        }
-        if (row >= p.M || n0 + c >= p.N) {
-          // row past M (zero-filled A) or column chunk past N: nothing to store
-        } else if (ACC_OUT) {
-          int32_t* o0 = p.acc0 + (size_t)row * p.N + n0 + c;
-          int32_t* o1 = p.acc1 + (size_t)row * p.N + n0 + c;
+            for (int i = 0; i < 32; ++i) r1[i] = 0;
+          }
+          uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
-            *reinterpret_cast<int4*>(o0 + i) =
-                make_int4((int)r0[i] >> kShift, (int)r0[i + 1] >> kShift, (int)r0[i + 2] >> kShift,
-                          (int)r0[i + 3] >> kShift);
-            *reinterpret_cast<int4*>(o1 + i) =
-                make_int4((int)r1[i] >> kShift, (int)r1[i + 1] >> kShift, (int)r1[i + 2] >> kShift,
-                          (int)r1[i + 3] >> kShift);
+            const float4 w = sw4[(cc + i) >> 2];
+            const float4 rr = sr4[(cc + i) >> 2];
+            const float y0 = sxv * fmaf(w.x, (float)((int)r0[i] >> kShift), rr.x * (float)((int)r1[i] >> kShift));
+            const float y1 = sxv * fmaf(w.y, (float)((int)r0[i + 1] >> kShift), rr.y * (float)((int)r1[i + 1] >> kShift));
+            const float y2 = sxv * fmaf(w.z, (float)((int)r0[i + 2] >> kShift), rr.z * (float)((int)r1[i + 2] >> kShift));
+            const float y3 = sxv * fmaf(w.w, (float)((int)r0[i + 3] >> kShift), rr.w * (float)((int)r1[i + 3] >> kShift));
+            const __nv_bfloat162 h0 = __floats2bfloat162_rn(y0, y1);
+            const __nv_bfloat162 h1 = __floats2bfloat162_rn(y2, y3);
+            pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h0);
+            pk[(i >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h1);
           }
-        } else {
-          const float sxm = p.sx[row];
-          uint32_t packed[16];
+          // 64-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ ((r / 2) % 4)
+          uint8_t* bp = smem + L::oStg + (q * (BN / 32) + (c >> 5)) * L::kBoxBytes + lane * 64;
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float y0 = sxm * fmaf(sw_t[c + i], (float)((int)r0[i] >> kShift),
-                                        sr_t[c + i] * (float)((int)r1[i] >> kShift));
-            const float y1 = sxm * fmaf(sw_t[c + i + 1], (float)((int)r0[i + 1] >> kShift),
-                                        sr_t[c + i + 1] * (float)((int)r1[i + 1] >> kShift));
-            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-            packed[i >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(p.Y + (size_t)row * p.ldy + n0 + c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(bp + ((k ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int y = m0 + q * 32;
+#pragma unroll
+          for (int b = 0; b < kCpl; ++b) {
+            const int x = n0 + eh * kHalf + 32 * b;
+            if (x < p.N && y < p.M)
+              tma_store_2d(&tmY, smem + L::oStg + (q * (BN / 32) + eh * kCpl + b) * L::kBoxBytes, x, y);
+          }
+          bulk_commit_group();
+        }
+        stores_pending = true;
       }
     }
+    if (!ACC_OUT && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();

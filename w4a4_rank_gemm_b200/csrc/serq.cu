@@ -249,6 +249,10 @@ cudaError_t launch_tc_ta(const serq_layer* L, const void* Xq, const serq::tc::Ar
   CUtensorMap tmA;
   if (!make_map(&tmA, Xq, (uint64_t)a.K / 2, (uint64_t)a.M, (uint64_t)a.K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
+  CUtensorMap tmY = tmA;
+  if (!ACC && !make_map(&tmY, a.Y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.ldy * 2, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+    return cudaErrorInvalidValue;
   auto kern = serq::tc::k_gemm_ta<BN, ACC>;
   static int attr_set[64] = {0};
   int dev = 0;
@@ -257,9 +261,13 @@ cudaError_t launch_tc_ta(const serq_layer* L, const void* Xq, const serq::tc::Ar
     set_smem(kern, Lay::kAlloc);
     attr_set[dev] = 1;
   }
-  const int mtiles = (a.M + 255) / 256;
+  serq::tc::Args ap = a;
+  ap.tiles_m = (a.M + 255) / 256;
+  ap.tiles_n = (a.N + BN - 1) / BN;
+  const long ntiles = (long)ap.tiles_m * ap.tiles_n;
+  const long slots = sm_count() / 2;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(mtiles * 2, (a.N + BN - 1) / BN);
+  cfg.gridDim = dim3((unsigned)((ntiles < slots ? ntiles : slots) * 2), 1);
   cfg.blockDim = dim3(serq::tc::kThreads);
   cfg.dynamicSmemBytes = Lay::kAlloc;
   cfg.stream = st;
@@ -270,9 +278,8 @@ cudaError_t launch_tc_ta(const serq_layer* L, const void* Xq, const serq::tc::Ar
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[2], L->tmR[2], a);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[2], L->tmR[2], tmY, ap);
 }
-
 
 template <bool A8, bool ACC>
 cudaError_t dispatch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, serq_algo algo,
