@@ -541,10 +541,11 @@ namespace tc {
 // activation stages of 32 columns (128 int8 per lane, four per column), so
 // BN = 192: 2 * 192 + 4 * 32 = 512 columns.
 //
-// Warps: 0 TMA, 1 TMEM owner / MMA issue (CTA 0), 4..7 widen the 128
+// Warps: 0 TMA, 1 TMEM owner / MMA issue (CTA 0), 2..9 widen in two groups
+// of four that take alternate steps; in its steps a group widens the 128
 // activation rows of this CTA into TMEM (warp w writes TMEM lanes
-// 32 (w % 4) .. +31, one row per thread), 2, 3, 8, 9 widen this CTA's BN/2
-// weight rows into shared memory; all eight run the epilogue, which stages
+// 32 (w % 4) .. +31, one row per thread) and this CTA's BN/2 weight rows
+// into shared memory.  All eight run the epilogue, which stages
 // the bf16 tile in a shared-memory area of its own (freed by the activation
 // stages' absence) and writes it with TMA stores.
 // The packed activation tile arrives with the 64-byte TMA swizzle, so the
@@ -555,6 +556,9 @@ struct LayoutTA {
   static constexpr int BNL = BN / 2;                  // weight rows per CTA
   static constexpr int PS = 8;                        // packed stages
   static constexpr int US = 4;                        // widened stages (smem B + TMEM A)
+  // two widening groups of four warps take alternate steps (see Layout)
+  static constexpr int G = 2;
+  static constexpr int kGroupWarps = kUnpackWarps / G;
   static constexpr int kPkA = BM * BK / 2;            // 8 KB, 64-byte swizzled
   static constexpr int kPkB = BNL * BK / 2;
   static constexpr int kPk = kPkA + kPkB;
@@ -569,7 +573,7 @@ struct LayoutTA {
   static constexpr int oScl = oStg + kBoxes * kBoxBytes;
   static constexpr int kSclWarp = 2 * (BN / 2) * 4;  // sw and sr of a warp's BN / 2 columns
   static constexpr int oBar = oScl + kUnpackWarps * kSclWarp;
-  static constexpr int nBar = 2 * PS + 2 * US + 2;
+  static constexpr int nBar = 2 * PS + 2 * US + 3;
   static constexpr int oMisc = oBar + nBar * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -578,6 +582,7 @@ struct LayoutTA {
   static constexpr uint32_t kTmemA = 2 * BN;          // first activation stage column
   static constexpr int kPiecesB = BNL * 4 / 128;      // per weight-widening thread
   static_assert(2 * BN + US * (BK / 4) <= 512, "TMEM budget");
+  static_assert(US % G == 0 && PS >= US && kGroupWarps == 4, "group ring ownership, one warp per lane quadrant");
   static_assert(BNL * 4 % 128 == 0 && BN % 64 == 0, "weight pieces must divide evenly");
   static_assert(kPk % 1024 == 0 && kUn % 1024 == 0 && oStg % 1024 == 0, "tiles must stay 1024-aligned");
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -601,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty_un = full_un + US;
   uint64_t* acc_full = empty_un + US;
   uint64_t* drain = acc_full + 1;
+  uint64_t* tmem_empty = drain + 1;     // (CTA 0) every epilogue warp of the pair read its TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::oMisc + 4);
 
@@ -615,14 +621,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < PS; ++s) {
       mbar_init(&full_pk[s], 1);
-      mbar_init(&empty_pk[s], kUnpackWarps);
+      mbar_init(&empty_pk[s], L::kGroupWarps);
     }
     for (int s = 0; s < US; ++s) {
-      mbar_init(&full_un[s], kUnpackWarps * 2);
+      mbar_init(&full_un[s], L::kGroupWarps * 2);
       mbar_init(&empty_un[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    mbar_init(tmem_empty, kUnpackWarps * 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -669,7 +676,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t un_base = smem_u32(smem + L::oUn);
       bool ok = true;
       int g = 0;
-      for (int t = cta_tile; ok && t < ntiles; t += tile_stride) {
+      int it = 0;
+      for (int t = cta_tile; ok && t < ntiles; t += tile_stride, ++it) {
+        if (it > 0 && !mbar_wait<true>(tmem_empty, (uint32_t)(it - 1) & 1u, abort_flag, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
         for (int step = 0; step < nsteps; ++step, ++g) {
           const int u = g % US;
           const uint32_t uph = (g / US) & 1;
@@ -708,10 +720,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------- widening + epilogue
-    const bool act = (warp >= 4 && warp <= 7);
+    // Group wg = warps 2 + 4 wg .. 5 + 4 wg widens steps g with g % 2 == wg:
+    // each thread widens one activation row of its warp's TMEM lane quadrant
+    // and three 16-byte weight pieces.
+    const int wg = (warp - 2) >> 2;
     const int q = warp & 3;                            // TMEM lane quadrant
-    const int arow = q * 32 + lane;                    // activation row (act warps)
-    const int bt = act ? 0 : ((warp < 4 ? warp - 2 : warp - 6) * 32 + lane);  // 0..127
+    const int arow = q * 32 + lane;                    // activation row
+    const int bt = ((warp - 2) & 3) * 32 + lane;       // 0..127 within the group
     uint32_t a_off[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) a_off[c] = arow * (BK / 2) + ((c ^ ((arow >> 1) & 3)) << 4);
@@ -751,14 +766,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         sxv = (row < p.M) ? __ldg(p.sx + row) : 0.f;
       }
       for (int step = 0; step < nsteps; ++step, ++g) {
+        if ((g & 1) != wg) continue;
         const int s = g % PS;
         const uint32_t ph = (g / PS) & 1;
         const int u = g % US;
         const uint32_t uph = (g / US) & 1;
-        if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        // widened slot first (see Layout)
         if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+        if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
         const uint8_t* pk = smem + L::oPk + s * L::kPk;
-        if (act) {
+        {
           uint32_t r[32];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -769,9 +786,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             r[8 * c + 4] = hi.x; r[8 * c + 5] = hi.y; r[8 * c + 6] = hi.z; r[8 * c + 7] = hi.w;
           }
           tmem_st_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + L::kTmemA + (uint32_t)(u * (BK / 4)), r);
-          tmem_st_wait();
-          tc_fence_before();
-        } else {
+        }
+        {
           uint8_t* un = smem + L::oUn + u * L::kUn;
           uint4 v[NPB];
 #pragma unroll
@@ -783,8 +799,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(un + dst_off[i]) = lo;
             *reinterpret_cast<uint4*>(un + (dst_off[i] ^ 16u)) = hi;
           }
-          fence_proxy_async_smem();
         }
+        tmem_st_wait();
+        tc_fence_before();
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&empty_pk[s]);
@@ -826,6 +844,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(tmem_empty);
+          else
+            mbar_arrive_remote(tmem_empty, 0);
+        }
       } else {
         // this warp's staging boxes were read by its previous TMA stores
         if (stores_pending) {
@@ -875,6 +900,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
+          if (leader)
+            mbar_arrive(tmem_empty);
+          else
+            mbar_arrive_remote(tmem_empty, 0);
           const int y = m0 + q * 32;
 #pragma unroll
           for (int b = 0; b < kCpl; ++b) {
