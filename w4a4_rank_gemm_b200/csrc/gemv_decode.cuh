@@ -1,16 +1,27 @@
 // Decode-regime SERQ linear (M <= 64 tokens): memory-bound, so the goal is
 // to stream the packed INT4 weights from HBM once at full bandwidth.
 //
-// Each CTA owns 8 output channels; its 8 warps split K.  Every thread loads
-// 16 bytes (32 nibbles) of one weight row per 128-k segment straight into
-// registers, unpacks them (nibble -> int8 x16) and feeds them, with the
-// matching activation codes, to m16n8k32 integer tensor-core MMAs: no shared
-// memory for weights, no re-read.  The segments that cover the first r
-// columns also load the same 16 bytes of the compensator R and accumulate
-// X~_{s,q} Q(R) into a second accumulator from the activation fragments
-// already in registers (SERQ notes key design 2: one matmul on the salient
-// channels).  The 8 warps' partial sums are reduced in shared memory and the
-// epilogue applies sx * (sw * acc0 + sR * acc1).
+// Work item = 16 consecutive output channels (two n8 MMA tiles, so every
+// activation fragment feeds two MMAs) over all of K.
+// The grid is persistent (items strided over the CTAs).  One producer warp
+// keeps a ring of items in shared memory with two untiled bulk copies per
+// item (its 8 weight rows and its 8 compensator rows are contiguous in HBM)
+// plus the item's 8 sw and sR,
+// and the ring is filled before the kernel waits for the grid it depends on:
+// weights are not produced by any earlier kernel, so with programmatic
+// dependent launch their streaming overlaps the previous kernel's tail.  The
+// activation codes (loaded once per CTA into shared memory when they fit,
+// else read from L2) and everything written come after that wait.
+//
+// Eight compute warps split K: each lane takes 16 bytes (32 nibbles) of one
+// weight row per 128-k segment, widens them in registers (nibble -> int8
+// x16) and feeds m16n8k32 integer MMAs with the matching activation codes;
+// the segments that cover the first r columns also take the same 16 bytes of
+// R and accumulate X~_{s,q} Q(R) into a second accumulator from the same
+// activation fragments (SERQ notes key design 2: one matmul on the salient
+// channels).  The warps' partial sums are added into shared accumulators of
+// the item's stage and the last warp to finish applies the epilogue
+// sx * (sw * acc0 + sR * acc1).
 //
 // k-order inside a segment: thread t of a quad covers the 32-code run
 // k in [128 seg + 32 t, +32).  MMA step s takes word s of the run's 16
@@ -24,8 +35,12 @@
 namespace serq {
 namespace decode {
 
-constexpr int kWarps = 8;
-constexpr int kMaxTiles = 4;  // 16-row tiles: M <= 64
+constexpr int kComputeWarps = 8;
+constexpr int kThreads = 32 * (kComputeWarps + 1);  // + one producer warp
+constexpr int kMaxTiles = 4;                        // 16-row tiles: M <= 64
+constexpr int kNT = 2;                              // n8 MMA tiles per item
+constexpr int kRows = 8 * kNT;                      // output channels per item
+constexpr int kPad = 16;                            // bytes added to every staged activation row
 
 struct Args {
   const uint8_t* Xq;
@@ -41,6 +56,28 @@ struct Args {
   int32_t* acc1;
 };
 
+// Shared-memory plan, computed on the host.
+struct Plan {
+  int kb;           // activation bytes per token row (K/2 or K)
+  int wrow, rrow;   // staged weight / compensator row bytes
+  int act_pitch;    // staged activation row pitch (activations in smem)
+  int act_bytes;    // M * act_pitch rounded up to 128, 0 when read from L2
+  int stage_bytes;  // kRows * (wrow + rrow + 8) rounded up to 128
+  int stages;
+  int items;        // N / kRows
+};
+
+// Shared accumulators of one item: [nt][mt][acc0 / acc1][fragment q][lane].
+template <int MT>
+struct Red {
+  static constexpr int kInts = kNT * MT * 2 * 4 * 32;
+};
+
+inline int smem_bytes(const Plan& pl, int mt) {
+  return 128 + pl.act_bytes + pl.stages * pl.stage_bytes + pl.stages * (Red<1>::kInts * mt + 1) * 4 + 8 +
+         (2 * pl.stages + 1) * 8 + 16;
+}
+
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -50,58 +87,51 @@ __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, ui
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ld_stream(const uint8_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ uint32_t lo_x16(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
 __device__ __forceinline__ uint32_t hi_x16(uint32_t w) { return w & 0xF0F0F0F0u; }
 
 // Operands of one 128-k segment for this thread.
 template <int MT, bool A8>
 struct Seg {
-  uint4 w, r;
+  uint4 w[kNT], r[kNT];        // weight / compensator row g of each n8 tile
   uint4 a[MT][2][A8 ? 2 : 1];  // [tile][row g / g+8][16-byte piece]
 };
 
-template <int MT, bool A8>
-__device__ __forceinline__ void load_seg(const Args& p, int seg, int g, int t, int n0, bool with_r,
-                                         Seg<MT, A8>& s) {
+template <int MT, bool A8, bool ACT_SMEM>
+__device__ __forceinline__ void load_seg(const Args& p, const Plan& pl, const uint8_t* wst, const uint8_t* rst,
+                                         const uint8_t* act, int seg, int g, int t, bool with_r, Seg<MT, A8>& s) {
   const uint4 z = make_uint4(0, 0, 0, 0);
   const int wb = seg * 64 + t * 16;  // byte offset in a packed weight row
-  s.w = (wb < (p.K >> 1)) ? ld_stream(p.Wq + (size_t)(n0 + g) * (p.K >> 1) + wb) : z;
-  s.r = (with_r && wb < (p.rpad >> 1)) ? ld_stream(p.Rq + (size_t)(n0 + g) * (p.rpad >> 1) + wb) : z;
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt) {
+    s.w[nt] = (wb < (p.K >> 1)) ? *reinterpret_cast<const uint4*>(wst + (8 * nt + g) * pl.wrow + wb) : z;
+    s.r[nt] = (with_r && wb < (p.rpad >> 1)) ? *reinterpret_cast<const uint4*>(rst + (8 * nt + g) * pl.rrow + wb) : z;
+  }
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int row = mt * 16 + g + 8 * h;
-      if (A8) {
-        const int ab = seg * 128 + t * 32;
-        const bool ok = row < p.M && ab < p.K;
-        const uint8_t* src = p.Xq + (size_t)row * p.K + ab;
-        s.a[mt][h][0] = ok ? __ldg(reinterpret_cast<const uint4*>(src)) : z;
-        s.a[mt][h][A8 ? 1 : 0] = ok ? __ldg(reinterpret_cast<const uint4*>(src + 16)) : z;
-      } else {
-        const bool ok = row < p.M && wb < (p.K >> 1);
-        s.a[mt][h][0] = ok ? __ldg(reinterpret_cast<const uint4*>(p.Xq + (size_t)row * (p.K >> 1) + wb)) : z;
+      const int ab = A8 ? seg * 128 + t * 32 : wb;
+      const bool ok = row < p.M && ab < pl.kb;
+#pragma unroll
+      for (int c = 0; c < (A8 ? 2 : 1); ++c) {
+        if (ACT_SMEM)
+          s.a[mt][h][c] = ok ? *reinterpret_cast<const uint4*>(act + row * pl.act_pitch + ab + 16 * c) : z;
+        else
+          s.a[mt][h][c] = ok ? __ldg(reinterpret_cast<const uint4*>(p.Xq + (size_t)row * pl.kb + ab + 16 * c)) : z;
       }
     }
   }
 }
 
+// One 128-k segment: every activation fragment is widened once and used by
+// the MMAs of both n8 tiles (two independent accumulator chains).
 template <int MT, bool A8>
-__device__ __forceinline__ void mma_seg(const Seg<MT, A8>& s, bool with_r, int (&acc0)[MT][4],
-                                        int (&acc1)[MT][4]) {
-  const uint32_t wv[4] = {s.w.x, s.w.y, s.w.z, s.w.w};
-  const uint32_t rv[4] = {s.r.x, s.r.y, s.r.z, s.r.w};
+__device__ __forceinline__ void mma_seg(const Seg<MT, A8>& s, bool with_r, int (&acc0)[kNT][MT][4],
+                                        int (&acc1)[kNT][MT][4]) {
 #pragma unroll
   for (int st = 0; st < 4; ++st) {
-    const uint32_t b0 = lo_x16(wv[st]), b1 = hi_x16(wv[st]);
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       uint32_t a0, a1, a2, a3;
@@ -120,94 +150,250 @@ __device__ __forceinline__ void mma_seg(const Seg<MT, A8>& s, bool with_r, int (
         a1 = lo_x16(y);
         a3 = hi_x16(y);
       }
-      mma_s8(acc0[mt], a0, a1, a2, a3, b0, b1);
-      if (with_r) mma_s8(acc1[mt], a0, a1, a2, a3, lo_x16(rv[st]), hi_x16(rv[st]));
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        const uint32_t w = (&s.w[nt].x)[st];
+        mma_s8(acc0[nt][mt], a0, a1, a2, a3, lo_x16(w), hi_x16(w));
+        if (with_r) {
+          const uint32_t r = (&s.r[nt].x)[st];
+          mma_s8(acc1[nt][mt], a0, a1, a2, a3, lo_x16(r), hi_x16(r));
+        }
+      }
     }
   }
 }
 
-template <int MT, bool A8, bool ACC_OUT>
-__global__ void __launch_bounds__(kWarps * 32) k_decode(Args p) {
-  __shared__ int red[kWarps][MT][2][4][32];
+template <int MT, bool A8, bool ACC_OUT, bool ACT_SMEM>
+__global__ void __launch_bounds__(kThreads, 1) k_decode(const Args p, const Plan pl) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* act = smem;                                          // [M][act_pitch]
+  uint8_t* ring = smem + pl.act_bytes;                          // stages of [W rows | R rows]
+  int* racc = reinterpret_cast<int*>(ring + pl.stages * pl.stage_bytes);  // [stage][mt][acc][q][lane]
+  int* cnt = racc + pl.stages * Red<MT>::kInts;                 // [stage] warps done with the item
+  uint64_t* bar = reinterpret_cast<uint64_t*>(cnt + ((pl.stages + 1) & ~1));
+  uint64_t* full = bar;                       // item landed (tx)
+  uint64_t* empty = bar + pl.stages;          // item read and its sums consumed
+  uint64_t* act_full = bar + 2 * pl.stages;   // activations landed (tx)
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(act_full + 1);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int n0 = blockIdx.x * 8;
-
-  const int nseg = (p.K + 127) >> 7;
-  const int rseg = (p.rpad + 127) >> 7;
-  const int per = nseg / kWarps, extra = nseg % kWarps;
-  const int s0 = warp * per + min(warp, extra);
-  const int s1 = s0 + per + (warp < extra ? 1 : 0);
-
-  int acc0[MT][4], acc1[MT][4];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc0[mt][j] = acc1[mt][j] = 0;
-
-  constexpr int U = (MT <= 2) ? 4 : 2;  // segments in flight per thread
-  int seg = s0;
-  for (; seg + U <= s1; seg += U) {
-    Seg<MT, A8> sv[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) load_seg<MT, A8>(p, seg + u, g, t, n0, seg + u < rseg, sv[u]);
-#pragma unroll
-    for (int u = 0; u < U; ++u) mma_seg<MT, A8>(sv[u], seg + u < rseg, acc0, acc1);
-  }
-  for (; seg < s1; ++seg) {
-    Seg<MT, A8> sv;
-    load_seg<MT, A8>(p, seg, g, t, n0, seg < rseg, sv);
-    mma_seg<MT, A8>(sv, seg < rseg, acc0, acc1);
-  }
-
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      red[warp][mt][0][j][lane] = acc0[mt][j];
-      red[warp][mt][1][j][lane] = acc1[mt][j];
+  for (int i = threadIdx.x; i < pl.stages * (Red<MT>::kInts + 1); i += blockDim.x) racc[i] = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < pl.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kComputeWarps);
     }
+    mbar_init(act_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
   __syncthreads();
+  // the next kernel in the stream may be scheduled from here on
+  grid_dep_launch();
 
-  // Accumulators carry the x16 of each unpacked INT4 operand.
-  constexpr int kShift = A8 ? 4 : 8;
-  for (int idx = threadIdx.x; idx < MT * 128; idx += blockDim.x) {
-    const int mt = idx >> 7, j = (idx >> 5) & 3, l = idx & 31;
-    int s_0 = 0, s_1 = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      s_0 += red[w][mt][0][j][l];
-      s_1 += red[w][mt][1][j][l];
+  const uint32_t wbytes = (uint32_t)p.K >> 1, rbytes = (uint32_t)p.rpad >> 1;
+
+  if (warp == kComputeWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      auto issue = [&](int item, int j) -> bool {
+        const int s = j % pl.stages;
+        const uint32_t ph = (j / pl.stages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) return false;
+        uint8_t* st = ring + s * pl.stage_bytes;
+        const size_t n0 = (size_t)item * kRows;
+        mbar_arrive_expect_tx(&full[s], kRows * (wbytes + rbytes + 8));
+        bulk_load(st, p.Wq + n0 * wbytes, kRows * wbytes, &full[s]);
+        if (rbytes) bulk_load(st + kRows * pl.wrow, p.Rq + n0 * rbytes, kRows * rbytes, &full[s]);
+        uint8_t* sc = st + kRows * (pl.wrow + pl.rrow);  // sw, sR of the item's channels (16 each)
+        bulk_load(sc, p.sw + n0, kRows * 4, &full[s]);
+        bulk_load(sc + kRows * 4, p.sr + n0, kRows * 4, &full[s]);
+        return true;
+      };
+      int item = blockIdx.x, j = 0;
+      // weights first: no earlier kernel writes them
+      for (; ok && item < pl.items && j < pl.stages; item += gridDim.x, ++j) ok = issue(item, j);
+      grid_dep_wait();
+      if (ok && ACT_SMEM) {
+        mbar_arrive_expect_tx(act_full, (uint32_t)(p.M * pl.kb));
+        for (int m = 0; m < p.M; ++m) bulk_load(act + m * pl.act_pitch, p.Xq + (size_t)m * pl.kb, pl.kb, act_full);
+      }
+      for (; ok && item < pl.items; item += gridDim.x, ++j) ok = issue(item, j);
     }
-    const int row = mt * 16 + (l >> 2) + 8 * (j >> 1);
-    const int col = n0 + 2 * (l & 3) + (j & 1);
-    if (row >= p.M) continue;
-    const int q0 = s_0 >> kShift, q1 = s_1 >> kShift;
-    if (ACC_OUT) {
-      p.acc0[(size_t)row * p.N + col] = q0;
-      p.acc1[(size_t)row * p.N + col] = q1;
-    } else {
-      const float y = p.sx[row] * fmaf(p.sw[col], (float)q0, p.sr[col] * (float)q1);
-      p.Y[(size_t)row * p.ldy + col] = __float2bfloat16_rn(y);
+  } else {
+    // ------------------------------------------------------- compute warps
+    // Each warp adds its partial sums of an item into the stage's shared
+    // accumulators; the last of the eight to finish the item (stage counter)
+    // applies the epilogue, clears the accumulators and releases the stage.
+    // No warp waits for another.
+    grid_dep_wait();  // sx and (from L2) the activation codes; Y after it
+    const int g = lane >> 2, t = lane & 3;
+    const int nseg = (p.K + 127) >> 7;
+    const int rseg = (p.rpad + 127) >> 7;
+    const int per = nseg / kComputeWarps, extra = nseg % kComputeWarps;
+    const int s0 = warp * per + min(warp, extra);
+    const int s1 = s0 + per + (warp < extra ? 1 : 0);
+    constexpr int kShift = A8 ? 4 : 8;  // the x16 of each widened INT4 operand
+    // Epilogue operands: sx in registers (loaded once), sw and sR of an
+    // item's channels in its stage.  No global load is outstanding at the
+    // shared-memory fences below, so they do not wait on HBM.
+    float sxr[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int row = mt * 16 + g + 8 * hh;
+        sxr[mt][hh] = (!ACC_OUT && row < p.M) ? __ldg(p.sx + row) : 0.f;
+      }
+    bool ok = !ACT_SMEM || mbar_wait(act_full, 0, abort_flag, kDevTimeoutUnpack);
+    int j = 0;
+    for (int item = blockIdx.x; ok && item < pl.items; item += gridDim.x, ++j) {
+      const int s = j % pl.stages;
+      const uint32_t ph = (j / pl.stages) & 1;
+      if (!mbar_wait(&full[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
+      const uint8_t* wst = ring + s * pl.stage_bytes;
+      const uint8_t* rst = wst + kRows * pl.wrow;
+      int acc0[kNT][MT][4], acc1[kNT][MT][4];
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc0[nt][mt][q] = acc1[nt][mt][q] = 0;
+      int seg = s0;
+      if (MT <= 2) {  // two segments' shared-memory loads in flight
+        for (; seg + 2 <= s1; seg += 2) {
+          Seg<MT, A8> sa, sb;
+          load_seg<MT, A8, ACT_SMEM>(p, pl, wst, rst, act, seg, g, t, seg < rseg, sa);
+          load_seg<MT, A8, ACT_SMEM>(p, pl, wst, rst, act, seg + 1, g, t, seg + 1 < rseg, sb);
+          mma_seg<MT, A8>(sa, seg < rseg, acc0, acc1);
+          mma_seg<MT, A8>(sb, seg + 1 < rseg, acc0, acc1);
+        }
+      }
+      for (; seg < s1; ++seg) {
+        Seg<MT, A8> sa;
+        load_seg<MT, A8, ACT_SMEM>(p, pl, wst, rst, act, seg, g, t, seg < rseg, sa);
+        mma_seg<MT, A8>(sa, seg < rseg, acc0, acc1);
+      }
+      int* ra = racc + s * Red<MT>::kInts;
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            atomicAdd(&ra[(((nt * MT + mt) * 2 + 0) * 4 + q) * 32 + lane], acc0[nt][mt][q]);
+            atomicAdd(&ra[(((nt * MT + mt) * 2 + 1) * 4 + q) * 32 + lane], acc1[nt][mt][q]);
+          }
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        last = (atomicAdd(&cnt[s], 1) == kComputeWarps - 1);
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence_block();
+        const float* sc = reinterpret_cast<const float*>(wst + kRows * (pl.wrow + pl.rrow));
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          const int col = item * kRows + 8 * nt + 2 * t;  // this lane's two output channels
+          const float2 sw2 = *reinterpret_cast<const float2*>(sc + 8 * nt + 2 * t);
+          const float2 sr2 = *reinterpret_cast<const float2*>(sc + kRows + 8 * nt + 2 * t);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int row = mt * 16 + g + 8 * hh;
+              int* e0 = &ra[(((nt * MT + mt) * 2 + 0) * 4 + 2 * hh) * 32 + lane];
+              int* e1 = &ra[(((nt * MT + mt) * 2 + 1) * 4 + 2 * hh) * 32 + lane];
+              const int a00 = e0[0] >> kShift, a01 = e0[32] >> kShift;  // columns col, col + 1
+              const int a10 = e1[0] >> kShift, a11 = e1[32] >> kShift;
+              e0[0] = 0; e0[32] = 0; e1[0] = 0; e1[32] = 0;
+              if (row >= p.M) continue;
+              if (ACC_OUT) {
+                *reinterpret_cast<int2*>(p.acc0 + (size_t)row * p.N + col) = make_int2(a00, a01);
+                *reinterpret_cast<int2*>(p.acc1 + (size_t)row * p.N + col) = make_int2(a10, a11);
+              } else {
+                const float sxm = sxr[mt][hh];
+                const float y0 = sxm * fmaf(sw2.x, (float)a00, sr2.x * (float)a10);
+                const float y1 = sxm * fmaf(sw2.y, (float)a01, sr2.y * (float)a11);
+                *reinterpret_cast<__nv_bfloat162*>(p.Y + (size_t)row * p.ldy + col) = __floats2bfloat162_rn(y0, y1);
+              }
+            }
+        }
+        if (lane == 0) cnt[s] = 0;
+        __threadfence_block();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // the stage (weights and sums) may be refilled
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == kComputeWarps * 32) {
+    // let bulk copies already issued land before shared memory is released
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < 100000ull) {
     }
   }
 }
 
+// Ring depth: as many items as fit next to the activations (up to 12);
+// activations go to shared memory when that leaves 2 stages.
+inline bool make_plan(const Args& p, bool a8, int mt, int max_smem, Plan& pl) {
+  pl.kb = a8 ? p.K : p.K / 2;
+  pl.wrow = p.K / 2;
+  pl.rrow = p.rpad / 2;
+  pl.stage_bytes = (kRows * (pl.wrow + pl.rrow + 8) + 127) & ~127;  // + sw, sR of the item's channels
+  pl.items = p.N / kRows;
+  pl.act_pitch = pl.kb + kPad;
+  const int per_stage = pl.stage_bytes + Red<1>::kInts * mt * 4 + 4 + 16;  // ring, sums, counter, 2 barriers
+  const int fixed = 128 + 8 + 16 + 8;
+  const int act = (p.M * pl.act_pitch + 127) & ~127;
+  auto stages_for = [&](int a) { return (max_smem - fixed - a) / per_stage; };
+  pl.act_bytes = (stages_for(act) >= 2) ? act : 0;
+  pl.stages = stages_for(pl.act_bytes);
+  if (pl.stages > 12) pl.stages = 12;
+  return pl.stages >= 1;  // one stage (K >= 14336 at W4A8) still works, unoverlapped
+}
+
+template <int MT, bool A8, bool ACC_OUT, bool ACT_SMEM>
+inline cudaError_t launch_mt(const Args& p, const Plan& pl, int sms, cudaStream_t st) {
+  auto kern = k_decode<MT, A8, ACC_OUT, ACT_SMEM>;
+  const int bytes = smem_bytes(pl, MT);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(pl.items < sms ? pl.items : sms));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, pl);
+}
+
 template <int MT, bool A8, bool ACC_OUT>
-inline cudaError_t launch_mt(const Args& p, cudaStream_t st) {
-  k_decode<MT, A8, ACC_OUT><<<p.N / 8, kWarps * 32, 0, st>>>(p);
-  return cudaGetLastError();
+inline cudaError_t launch_tiles(const Args& p, const Plan& pl, int sms, cudaStream_t st) {
+  return pl.act_bytes ? launch_mt<MT, A8, ACC_OUT, true>(p, pl, sms, st)
+                      : launch_mt<MT, A8, ACC_OUT, false>(p, pl, sms, st);
 }
 
 template <bool A8, bool ACC_OUT>
-inline cudaError_t launch(const Args& p, cudaStream_t st) {
+inline cudaError_t launch(const Args& p, int sms, int max_smem, cudaStream_t st) {
   const int tiles = (p.M + 15) / 16;
+  Plan pl;
+  if (tiles < 1 || tiles > kMaxTiles || !make_plan(p, A8, tiles, max_smem, pl)) return cudaErrorInvalidValue;
   switch (tiles) {
-    case 1: return launch_mt<1, A8, ACC_OUT>(p, st);
-    case 2: return launch_mt<2, A8, ACC_OUT>(p, st);
-    case 3: return launch_mt<3, A8, ACC_OUT>(p, st);
-    case 4: return launch_mt<4, A8, ACC_OUT>(p, st);
-    default: return cudaErrorInvalidValue;
+    case 1: return launch_tiles<1, A8, ACC_OUT>(p, pl, sms, st);
+    case 2: return launch_tiles<2, A8, ACC_OUT>(p, pl, sms, st);
+    case 3: return launch_tiles<3, A8, ACC_OUT>(p, pl, sms, st);
+    default: return launch_tiles<4, A8, ACC_OUT>(p, pl, sms, st);
   }
 }
 

@@ -193,6 +193,18 @@ int sm_count() {
   return sms;
 }
 
+// Opt-in shared memory per block of the current device.
+int max_smem() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int v = 232448;
+  cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (dev < 64) cached[dev] = v;
+  return v;
+}
+
 // ------------------------------------------------------------ GEMM launch
 template <int BN, bool A8, bool ACC, int CG>
 cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, cudaStream_t st) {
@@ -332,9 +344,11 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
     serq::decode::Args a{static_cast<const uint8_t*>(Xq), sx, M, L->K, L->N, L->rpad, L->wq, L->rq, L->sw,
                          L->sr, static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1};
     if (a8)
-      e = accum ? serq::decode::launch<true, true>(a, st) : serq::decode::launch<true, false>(a, st);
+      e = accum ? serq::decode::launch<true, true>(a, sm_count(), max_smem(), st)
+                : serq::decode::launch<true, false>(a, sm_count(), max_smem(), st);
     else
-      e = accum ? serq::decode::launch<false, true>(a, st) : serq::decode::launch<false, false>(a, st);
+      e = accum ? serq::decode::launch<false, true>(a, sm_count(), max_smem(), st)
+                : serq::decode::launch<false, false>(a, sm_count(), max_smem(), st);
   } else {
     serq::tc::Args a{M, L->K, L->N, L->rpad, (L->K + serq::tc::BK - 1) / serq::tc::BK,
                      (L->rpad + serq::tc::BK - 1) / serq::tc::BK, sx, L->sw, L->sr,
