@@ -298,6 +298,22 @@ def test_llama2_7b_decode(S, M):
     assert_y_close(Y, y_ref)
 
 
+@pytest.mark.parametrize("M,K,N,mode", [
+    (16, 11008, 512, "w4a4"),   # activations too large for shared memory next to the ring: read from L2
+    (8, 14336, 256, "w4a8"),    # an item fills half of shared memory: a one-stage ring
+    (64, 4096, 256, "w4a4"),    # four 16-token tiles
+])
+def test_decode_large_k(S, M, K, N, mode):
+    L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, 128, mode, seed=5)
+    acc0, acc1 = O.linear_accum(xq, ol)
+    g0, g1 = S.linear_accum(L, Xq, S.ALGO_DECODE)
+    Y = S.linear(L, Xq, sx, algo=S.ALGO_DECODE)
+    torch.cuda.synchronize()
+    assert np.array_equal(g0.cpu().numpy(), acc0) and np.array_equal(g1.cpu().numpy(), acc1)
+    assert_y_close(Y, O.linear_epilogue(acc0, acc1, osx, ol))
+    assert S.device_error() == 0
+
+
 def test_llama3_8b_w4a8_kv_sampled(S):
     wl = synth.llama3_8b(M=4096, only=["k_proj"])
     p = wl.projections[0]
