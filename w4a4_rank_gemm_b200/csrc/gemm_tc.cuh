@@ -205,10 +205,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   cta_sync<CG>();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_launch();  // the next kernel in the stream may be scheduled
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // Weight (or R) tiles of the first PS steps go out before the wait for
+      // the grid this launch depends on (programmatic dependent launch):
+      // no earlier kernel writes them.  Their stages are fresh, so no empty
+      // wait; the A tiles follow once the activation codes are final.
+      int npre = 0;
+      for (int t = cta_tile, step = 0; npre < PS && t < ntiles; ++npre) {
+        const int nb0 = (t / p.tiles_m) * BN + (int)rank * L::BNL;
+        const bool res = step >= p.nkb;
+        const int j = res ? step - p.nkb : step;
+        mbar_arrive_expect_tx(&full_pk[npre], L::kTxBytes);
+        tma_load_2d(smem + L::oPk + npre * L::kPk + L::kPkA, res ? &tmR : &tmB, &full_pk[npre], j * (BK / 2), nb0);
+        if (++step == nsteps) {
+          step = 0;
+          t += tile_stride;
+        }
+      }
+      grid_dep_wait();
       int g = 0;  // pipeline step across tiles
       bool ok = true;
       for (int t = cta_tile; ok && t < ntiles; t += tile_stride) {
@@ -217,13 +235,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int step = 0; step < nsteps; ++step, ++g) {
           const int s = g % PS;
           const uint32_t ph = (g / PS) & 1;
-          if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
           const bool res = step >= p.nkb;
           const int j = res ? step - p.nkb : step;
           uint8_t* stage = smem + L::oPk + s * L::kPk;
+          if (g >= npre) {
+            if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
+            tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
+          }
           tma_load_2d(stage, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
-          tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
         }
       }
     }
@@ -329,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return r;
     };
 
+    grid_dep_wait();  // sx and, in the epilogue, Y belong to the dependency chain
     bool ok = true;
     int g = 0;
     int it = 0;

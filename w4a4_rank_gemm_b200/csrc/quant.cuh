@@ -130,6 +130,9 @@ __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* _
   const int nrun = K >> 5;
   uint4 raw[RPL][4][W];
   float amax = 0.f;
+  // programmatic dependent launch: the input (written by the previous
+  // kernel) is read only after that kernel completed
+  grid_dep_wait();
 #pragma unroll
   for (int i = 0; i < RPL; ++i) {
     const int b = lane + 32 * (warp + nw * i);
@@ -210,6 +213,9 @@ __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* _
       dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
   }
+  // the next kernel may be scheduled once every CTA got here: its prologue
+  // overlaps the last rows instead of taking SMs from the earlier ones
+  grid_dep_launch();
 }
 
 // Runs per lane held in registers: 4 for bf16 input (64 registers of raw
@@ -221,8 +227,16 @@ inline cudaError_t launch_quant_rows(const Loader& ld, int M, int K, uint8_t* Xq
   const int nrun = K / 32;
   const int warps = (nrun + 32 * RPL - 1) / (32 * RPL);
   if (warps > 8) return cudaErrorInvalidValue;
-  k_quant_rows<Q, RPL, Loader><<<M, warps * 32, 0, st>>>(ld, K, Xq, sx);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M);
+  cfg.blockDim = dim3(warps * 32);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_quant_rows<Q, RPL, Loader>, ld, K, Xq, sx);
 }
 
 // --------------------------------------------------- flatten and permute

@@ -243,13 +243,15 @@ cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args&
   cfg.blockDim = dim3(serq::tc::kThreads);
   cfg.dynamicSmemBytes = Lay::kAlloc;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see the producer's first steps
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[bi], L->tmR[bi], tmY, ap);
 }
 
