@@ -349,10 +349,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       return r;
     };
 
+    // Widens pipeline step gs (this group's) into its widened slot.
+    auto widen_step = [&](int gs) -> bool {
+      const int s = gs % PS;
+      const uint32_t ph = (gs / PS) & 1;
+      const int u = gs % US;
+      const uint32_t uph = (gs / US) & 1;
+      if ((stg_mask >> u) & 1u) {
+        if (!release_staging()) return false;
+      }
+      // widened slot first: see the ring notes in Layout
+      if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) return false;
+      if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) return false;
+      const uint8_t* pk = smem + L::oPk + s * L::kPk;
+      uint8_t* un = smem + L::oUn + u * L::kUn;
+      constexpr int NB = NP < 8 ? NP : 8;  // pieces in registers at a time
+      static_assert(NP % NB == 0, "pieces come in whole batches");
+#pragma unroll
+      for (int b = 0; b < NP; b += NB) {
+        uint4 v[NB];
+#pragma unroll
+        for (int i = 0; i < NB; ++i)
+          v[i] = *reinterpret_cast<const uint4*>(pk + src0 + (b + i) * kRowStep * (BK / 2));
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          uint4 lo, hi;
+          widen_run(v[i], lo, hi);
+          const uint32_t d = dst0 + (b + i) * kRowStep * BK;
+          *reinterpret_cast<uint4*>(un + d) = lo;
+          *reinterpret_cast<uint4*>(un + (d ^ 16u)) = hi;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty_pk[s]);
+        if (leader)
+          mbar_arrive(&full_un[u]);
+        else
+          mbar_arrive_remote(&full_un[u], 0);
+      }
+      return true;
+    };
+
     grid_dep_wait();  // sx and, in the epilogue, Y belong to the dependency chain
     bool ok = true;
     int g = 0;
     int it = 0;
+    int pre_end = 0;  // steps before this were widened ahead of their tile
     for (int t = cta_tile; ok && t < ntiles; t += tile_stride, ++it) {
       const int tm = t % p.tiles_m;
       const int m0 = (tm * CG + (int)rank) * BM;
@@ -371,45 +415,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       for (int step = 0; step < nsteps; ++step, ++g) {
-        if (g % L::G != wg) continue;
-        const int s = g % PS;
-        const uint32_t ph = (g / PS) & 1;
-        const int u = g % US;
-        const uint32_t uph = (g / US) & 1;
-        if ((stg_mask >> u) & 1u) {
-          if (!release_staging()) { ok = false; break; }
-        }
-        // widened slot first: see the ring notes in Layout
-        if (!mbar_wait(&empty_un[u], uph ^ 1, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
-        if (!mbar_wait(&full_pk[s], ph, abort_flag, kDevTimeoutUnpack)) { ok = false; break; }
-        const uint8_t* pk = smem + L::oPk + s * L::kPk;
-        uint8_t* un = smem + L::oUn + u * L::kUn;
-        constexpr int NB = NP < 8 ? NP : 8;  // pieces in registers at a time
-        static_assert(NP % NB == 0, "pieces come in whole batches");
-#pragma unroll
-        for (int b = 0; b < NP; b += NB) {
-          uint4 v[NB];
-#pragma unroll
-          for (int i = 0; i < NB; ++i)
-            v[i] = *reinterpret_cast<const uint4*>(pk + src0 + (b + i) * kRowStep * (BK / 2));
-#pragma unroll
-          for (int i = 0; i < NB; ++i) {
-            uint4 lo, hi;
-            widen_run(v[i], lo, hi);
-            const uint32_t d = dst0 + (b + i) * kRowStep * BK;
-            *reinterpret_cast<uint4*>(un + d) = lo;
-            *reinterpret_cast<uint4*>(un + (d ^ 16u)) = hi;
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&empty_pk[s]);
-          if (leader)
-            mbar_arrive(&full_un[u]);
-          else
-            mbar_arrive_remote(&full_un[u], 0);
-        }
+        if (g % L::G != wg || g < pre_end) continue;
+        if (!widen_step(g)) { ok = false; break; }
+      }
+      if (!ok) break;
+      // Widen ahead: this group's steps of the next tile that go to widened
+      // slots the epilogue below does not stage into, so that the next
+      // tile's first MMAs can issue as soon as TMEM is free.
+      if (t + tile_stride < ntiles) {
+        const int ahead = min(US - L::kStgStages, nsteps);
+        for (int ga = g; ga < g + ahead; ++ga)
+          if (ga % L::G == wg && !widen_step(ga)) { ok = false; break; }
+        pre_end = g + ahead;
       }
       if (!ok) break;
 
@@ -452,11 +469,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_remote(tmem_empty, 0);
         }
       } else {
-        // scales of this warp's columns -> its private smem copy
+        // scales of this warp's columns -> its private smem copy, with the
+        // widening factor 2^kShift folded in (exact: a power of two)
+        constexpr float kUnscale = 1.f / (float)(1 << kShift);
 #pragma unroll
         for (int i = 0; i < kCpl; ++i) {
-          scl[kCpl * lane + i] = swv[i];
-          scl[kHalf + kCpl * lane + i] = srv[i];
+          scl[kCpl * lane + i] = swv[i] * kUnscale;
+          scl[kHalf + kCpl * lane + i] = srv[i] * kUnscale;
         }
         __syncwarp();
         // output staging: box b = 32 rows x 64 columns of the tile, stored
@@ -469,47 +488,81 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         const float4* sw4 = reinterpret_cast<const float4*>(scl);
         const float4* sr4 = reinterpret_cast<const float4*>(scl + kHalf);
-        for (int cc = 0; cc < kHalf; cc += 16) {
-          const int c = eh * kHalf + cc;  // tile column of this 16-column chunk
-          uint32_t r0[16], r1[16];
-          tmem_ld_32x32b_x16(tq + (uint32_t)c, r0);
-          if (has_r) tmem_ld_32x32b_x16(tq + (uint32_t)(BN + c), r1);
-          tmem_ld_wait();
-          if (!has_r) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) r1[i] = 0;
+        // 16-column chunks, double-buffered: the TMEM loads of chunk k + 1 are
+        // in flight while chunk k is converted and staged; TMEM is released
+        // as soon as the last chunk's loads have completed.
+        constexpr int kChunks = kHalf / 16;
+        auto release_tmem = [&]() {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader)
+              mbar_arrive(tmem_empty);
+            else
+              mbar_arrive_remote(tmem_empty, 0);
           }
+        };
+        auto load_chunk = [&](uint32_t(&d0)[16], uint32_t(&d1)[16], int cc) {
+          const int c = eh * kHalf + cc;
+          tmem_ld_32x32b_x16(tq + (uint32_t)c, d0);
+          if (has_r) {
+            tmem_ld_32x32b_x16(tq + (uint32_t)(BN + c), d1);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) d1[i] = 0;
+          }
+        };
+        auto convert_chunk = [&](const uint32_t(&r0)[16], const uint32_t(&r1)[16], int cc) {
+          const int c = eh * kHalf + cc;  // tile column of this 16-column chunk
           // 128-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)
           uint8_t* bp = box_ptr(eq * (BN / 64) + (c >> 6)) + lane * 128;
           const int k0 = (c & 63) >> 3;  // first 16-byte chunk of these 16 columns
+          const float2 sx2 = make_float2(sxv, sxv);
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             uint32_t pk[4];
 #pragma unroll
             for (int i = 0; i < 8; i += 4) {
+              // y = sx * (sw' * acc0 + sR' * acc1) on column pairs, with the
+              // accumulators converted as they come out of TMEM (x256 or x16;
+              // the factor is in sw', sR')
               const int e = 8 * k + i;
               const float4 w = sw4[(cc + e) >> 2];
               const float4 rr = sr4[(cc + e) >> 2];
-              const float y0 = sxv * fmaf(w.x, (float)((int)r0[e] >> kShift), rr.x * (float)((int)r1[e] >> kShift));
-              const float y1 = sxv * fmaf(w.y, (float)((int)r0[e + 1] >> kShift), rr.y * (float)((int)r1[e + 1] >> kShift));
-              const float y2 = sxv * fmaf(w.z, (float)((int)r0[e + 2] >> kShift), rr.z * (float)((int)r1[e + 2] >> kShift));
-              const float y3 = sxv * fmaf(w.w, (float)((int)r0[e + 3] >> kShift), rr.w * (float)((int)r1[e + 3] >> kShift));
-              const __nv_bfloat162 h0 = __floats2bfloat162_rn(y0, y1);
-              const __nv_bfloat162 h1 = __floats2bfloat162_rn(y2, y3);
+              const float2 f0a = make_float2((float)(int)r0[e], (float)(int)r0[e + 1]);
+              const float2 f0b = make_float2((float)(int)r0[e + 2], (float)(int)r0[e + 3]);
+              const float2 f1a = make_float2((float)(int)r1[e], (float)(int)r1[e + 1]);
+              const float2 f1b = make_float2((float)(int)r1[e + 2], (float)(int)r1[e + 3]);
+              const float2 ya = mul2(sx2, fma2(make_float2(w.x, w.y), f0a, mul2(make_float2(rr.x, rr.y), f1a)));
+              const float2 yb = mul2(sx2, fma2(make_float2(w.z, w.w), f0b, mul2(make_float2(rr.z, rr.w), f1b)));
+              const __nv_bfloat162 h0 = __floats2bfloat162_rn(ya.x, ya.y);
+              const __nv_bfloat162 h1 = __floats2bfloat162_rn(yb.x, yb.y);
               pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h0);
               pk[(i >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h1);
             }
             *reinterpret_cast<uint4*>(bp + (((k0 + k) ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
+        };
+        uint32_t ra0[16], ra1[16], rb0[16], rb1[16];
+        load_chunk(ra0, ra1, 0);
+        tmem_ld_wait_regs(ra0, ra1);
+        if (kChunks == 1) release_tmem();
+#pragma unroll
+        for (int k = 0; k < kChunks; ++k) {
+          if ((k & 1) == 0) {
+            if (k + 1 < kChunks) load_chunk(rb0, rb1, 16 * (k + 1));
+            convert_chunk(ra0, ra1, 16 * k);
+            if (k + 1 < kChunks) tmem_ld_wait_regs(rb0, rb1);
+          } else {
+            if (k + 1 < kChunks) load_chunk(ra0, ra1, 16 * (k + 1));
+            convert_chunk(rb0, rb1, 16 * k);
+            if (k + 1 < kChunks) tmem_ld_wait_regs(ra0, ra1);
+          }
+          if (k + 2 == kChunks) release_tmem();  // the last chunk's loads are complete
         }
-        tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (leader)
-            mbar_arrive(tmem_empty);
-          else
-            mbar_arrive_remote(tmem_empty, 0);
           const int y = m0 + eq * 32;
 #pragma unroll
           for (int b = 0; b < kHalf / 64; ++b) {
