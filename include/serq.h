@@ -66,8 +66,11 @@ typedef enum {
   SERQ_ALGO_PREFILL_N256 = 4,  /* PREFILL with 128 x 256 output tiles, one CTA  */
   SERQ_ALGO_PREFILL_PAIR_N256 = 5, /* PREFILL with 256 x 256 tiles on a CTA pair
                                       (tcgen05 cta_group::2)                    */
-  SERQ_ALGO_PREFILL_PAIR_TMEM_A = 6 /* W4A4 only: 256 x 192 tiles on a CTA pair with
-                                       the widened activations in tensor memory  */
+  SERQ_ALGO_PREFILL_PAIR_TMEM_A = 6, /* W4A4 only: 256 x 192 tiles on a CTA pair with
+                                        the widened activations in tensor memory  */
+  SERQ_ALGO_DECODE_TC = 7      /* M <= 32: tcgen05 GEMV with the weight rows as the
+                                  MMA's M, split-K partial sums in the layer's
+                                  workspace (one stream per layer at a time)  */
 } serq_algo;
 
 typedef struct serq_layer serq_layer;

@@ -148,7 +148,7 @@ def test_linear_accum_bit_exact(S, mode, M, K, N, r):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, r, mode)
     acc0, acc1 = O.linear_accum(xq, ol)
     algos = [S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
-        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE] if M <= 64 else [])
+        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
     for algo in algos:
         g0, g1 = S.linear_accum(L, Xq, algo)
         torch.cuda.synchronize()
@@ -164,7 +164,7 @@ def test_linear_output_within_tolerance(S, mode, M, K, N, r):
     acc0, acc1 = O.linear_accum(xq, ol)
     y_ref = O.linear_epilogue(acc0, acc1, osx, ol)
     algos = [S.ALGO_AUTO, S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
-        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE] if M <= 64 else [])
+        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
     for algo in algos:
         Y = S.linear(L, Xq, sx, algo=algo)
         torch.cuda.synchronize()
@@ -290,12 +290,13 @@ def test_llama2_7b_decode(S, M):
     inp = wl.inputs[p.input]
     (L,), (ol,) = _prepare_both(S, [p.W], inp.X_calib, wl.rank, "w4a4")
     _, Xq, sx = _gpu_act(S, L, inp.X, "bf16", "w4a4")
-    Y = S.linear(L, Xq, sx)
-    g0, g1 = S.linear_accum(L, Xq)
-    torch.cuda.synchronize()
     y_ref, xq, osx, acc0, acc1 = O.linear(O.flatten_permute(inp.X, ol.s, ol.pi, True), ol, 4)
-    assert np.array_equal(g0.cpu().numpy(), acc0) and np.array_equal(g1.cpu().numpy(), acc1)
-    assert_y_close(Y, y_ref)
+    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_TC):
+        Y = S.linear(L, Xq, sx, algo=algo)
+        g0, g1 = S.linear_accum(L, Xq, algo)
+        torch.cuda.synchronize()
+        assert np.array_equal(g0.cpu().numpy(), acc0) and np.array_equal(g1.cpu().numpy(), acc1), f"algo {algo}"
+        assert_y_close(Y, y_ref)
 
 
 @pytest.mark.parametrize("M,K,N,mode", [
@@ -306,11 +307,12 @@ def test_llama2_7b_decode(S, M):
 def test_decode_large_k(S, M, K, N, mode):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, 128, mode, seed=5)
     acc0, acc1 = O.linear_accum(xq, ol)
-    g0, g1 = S.linear_accum(L, Xq, S.ALGO_DECODE)
-    Y = S.linear(L, Xq, sx, algo=S.ALGO_DECODE)
-    torch.cuda.synchronize()
-    assert np.array_equal(g0.cpu().numpy(), acc0) and np.array_equal(g1.cpu().numpy(), acc1)
-    assert_y_close(Y, O.linear_epilogue(acc0, acc1, osx, ol))
+    for algo in [S.ALGO_DECODE] + ([S.ALGO_DECODE_TC] if M <= 32 else []):
+        g0, g1 = S.linear_accum(L, Xq, algo)
+        Y = S.linear(L, Xq, sx, algo=algo)
+        torch.cuda.synchronize()
+        assert np.array_equal(g0.cpu().numpy(), acc0) and np.array_equal(g1.cpu().numpy(), acc1), f"algo {algo}"
+        assert_y_close(Y, O.linear_epilogue(acc0, acc1, osx, ol))
     assert S.device_error() == 0
 
 

@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_decode.cuh"
+#include "gemv_tc.cuh"
 #include "prepare.cuh"
 #include "quant.cuh"
 
@@ -104,6 +105,8 @@ struct serq_layer {
   float* smooth;
   CUtensorMap tmB[3];  // box rows 128, 256, 96
   CUtensorMap tmR[3];
+  int32_t* ws;         // split-K partial sums of the tensor-core decode, zero between calls
+  int32_t* cnt;        // per 128-row tile: units done
 };
 
 namespace {
@@ -122,7 +125,9 @@ serq_status alloc_layer(int K, int N, int rank, int mode, serq_layer** out) {
   const size_t s_rq = up256((size_t)N * L->rpad / 2);
   const size_t s_n = up256((size_t)N * 4);
   const size_t s_k = up256((size_t)K * 4);
-  const size_t total = s_wq + s_rq + 2 * s_n + 2 * s_k;
+  const size_t s_ws = up256((size_t)2 * N * serq::dtc::kMaxM * 4);
+  const size_t s_cnt = up256((size_t)((N + 127) / 128) * 4);
+  const size_t total = s_wq + s_rq + 2 * s_n + 2 * s_k + s_ws + s_cnt;
   cudaError_t e = cudaMalloc(&L->block, total);
   if (e != cudaSuccess) {
     delete L;
@@ -141,6 +146,17 @@ serq_status alloc_layer(int K, int N, int rank, int mode, serq_layer** out) {
   L->perm = reinterpret_cast<int32_t*>(b);
   b += s_k;
   L->smooth = reinterpret_cast<float*>(b);
+  b += s_k;
+  L->ws = reinterpret_cast<int32_t*>(b);
+  b += s_ws;
+  L->cnt = reinterpret_cast<int32_t*>(b);
+  e = cudaMemset(L->ws, 0, s_ws + s_cnt);
+  if (e != cudaSuccess) {
+    cudaFree(L->block);
+    delete L;
+    cudaGetLastError();
+    return fail(SERQ_ERR_CUDA, "cudaMemset of the workspace failed: %s", cudaGetErrorString(e));
+  }
   *out = L;
   return SERQ_OK;
 }
@@ -295,6 +311,48 @@ cudaError_t launch_tc_ta(const serq_layer* L, const void* Xq, const serq::tc::Ar
   return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[2], L->tmR[2], tmY, ap);
 }
 
+// Tensor-core decode (weights as the MMA's M), split-K over about two units
+// per SM.
+template <int MP, bool A8, bool ACC>
+cudaError_t launch_decode_tc(const serq_layer* L, const void* Xq, serq::dtc::Args a, cudaStream_t st) {
+  using Lay = serq::dtc::Layout<MP, A8>;
+  CUtensorMap tmX;
+  bool okm = A8 ? make_map(&tmX, Xq, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, 128, MP, CU_TENSOR_MAP_SWIZZLE_128B)
+                : make_map(&tmX, Xq, (uint64_t)a.K / 2, (uint64_t)a.M, (uint64_t)a.K / 2, 64, MP, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!okm) return cudaErrorInvalidValue;
+  auto kern = serq::dtc::k_decode_tc<MP, A8, ACC>;
+  static int attr_set[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    set_smem(kern, Lay::kAlloc);
+    attr_set[dev] = 1;
+  }
+  const int tiles = (a.N + serq::dtc::BM - 1) / serq::dtc::BM;
+  int splits = (2 * sm_count() + tiles / 2) / tiles;
+  if (splits < 1) splits = 1;
+  if (splits > a.nkb) splits = a.nkb;
+  a.splits = splits;
+  a.ws = L->ws;
+  a.cnt = L->cnt;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(tiles * splits));
+  cfg.blockDim = dim3(serq::dtc::kThreads);
+  cfg.dynamicSmemBytes = Lay::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, L->tmB[0], L->tmR[0], tmX, a);
+}
+
+template <bool A8, bool ACC>
+cudaError_t dispatch_decode_tc(const serq_layer* L, const void* Xq, const serq::dtc::Args& a, cudaStream_t st) {
+  return (a.M <= 16) ? launch_decode_tc<16, A8, ACC>(L, Xq, a, st) : launch_decode_tc<32, A8, ACC>(L, Xq, a, st);
+}
+
 template <bool A8, bool ACC>
 cudaError_t dispatch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, serq_algo algo,
                         cudaStream_t st) {
@@ -334,7 +392,9 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
   if (algo == SERQ_ALGO_AUTO) algo = (M <= serq_decode_max_m()) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
   if (algo == SERQ_ALGO_DECODE && M > serq::decode::kMaxTiles * 16)
     return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "decode kernel takes M <= %d (got %d)", serq::decode::kMaxTiles * 16, M);
-  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_PREFILL_PAIR_TMEM_A) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
+  if (algo == SERQ_ALGO_DECODE_TC && M > serq::dtc::kMaxM)
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "SERQ_ALGO_DECODE_TC takes M <= %d (got %d)", serq::dtc::kMaxM, M);
+  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_DECODE_TC) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
   if (algo == SERQ_ALGO_PREFILL_PAIR_TMEM_A && L->mode != SERQ_W4A4)
     return fail(SERQ_ERR_INVALID_ARG, "SERQ_ALGO_PREFILL_PAIR_TMEM_A takes W4A4 layers");
   if ((s = check_device())) return s;
@@ -342,7 +402,15 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool a8 = (L->mode == SERQ_W4A8);
   cudaError_t e;
-  if (algo == SERQ_ALGO_DECODE) {
+  if (algo == SERQ_ALGO_DECODE_TC) {
+    serq::dtc::Args a{M, L->K, L->N, L->rpad, (L->K + serq::dtc::BK - 1) / serq::dtc::BK,
+                      (L->rpad + serq::dtc::BK - 1) / serq::dtc::BK, 1, sx, L->sw, L->sr,
+                      static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1, nullptr, nullptr};
+    if (a8)
+      e = accum ? dispatch_decode_tc<true, true>(L, Xq, a, st) : dispatch_decode_tc<true, false>(L, Xq, a, st);
+    else
+      e = accum ? dispatch_decode_tc<false, true>(L, Xq, a, st) : dispatch_decode_tc<false, false>(L, Xq, a, st);
+  } else if (algo == SERQ_ALGO_DECODE) {
     serq::decode::Args a{static_cast<const uint8_t*>(Xq), sx, M, L->K, L->N, L->rpad, L->wq, L->rq, L->sw,
                          L->sr, static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1};
     if (a8)
