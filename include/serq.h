@@ -187,6 +187,26 @@ serq_status serq_linear_accum(const serq_layer* layer, const void* Xq, int M, in
                               int32_t* acc1, serq_algo algo, void* stream);
 
 /*
+ * serq_linear_decode_static -- serq_linear (or, with acc0/acc1, the
+ * accumulator hook) through the tensor-core decode kernel
+ * (SERQ_ALGO_DECODE_TC) with its split-K partial sums and tile counters in a
+ * scratch area compiled into the library, one per device, instead of the
+ * layer's workspace: the call allocates nothing.  The pages have no
+ * counterpart; this is a deployment variant of the same arithmetic.
+ *  Xq, sx, Y, ldy  as serq_linear; M <= 32.
+ *  acc0, acc1      both null (bf16 output in Y), or both DEVICE int32 M x N
+ *                  (exact accumulators; sx and Y are then not used).
+ *  N <= 16384, else SERQ_ERR_UNSUPPORTED_SHAPE.
+ * The scratch must start at zero: the first call on a device clears it (a
+ * synchronous cudaMemset) and every completed call leaves it zero.
+ * Races: all calls on a device share the one scratch area, so they must not
+ * overlap in time (one stream, or streams ordered by events), across all
+ * layers.  A wait that times out (serq_device_error) leaves it undefined.
+ */
+serq_status serq_linear_decode_static(const serq_layer* layer, const void* Xq, const float* sx, int M,
+                                      void* Y, int ldy, int32_t* acc0, int32_t* acc1, void* stream);
+
+/*
  * serq_silu_mul_quantize -- MLP intermediate of a Llama block whose gate/up
  * were prepared with down_proj's fold: h = silu(G) * U in fp32 (silu(g) =
  * g / (1 + e^-g), e^x by Cody-Waite reduction and a degree-7 Taylor

@@ -333,8 +333,10 @@ cudaError_t launch_decode_tc(const serq_layer* L, const void* Xq, serq::dtc::Arg
   if (splits < 1) splits = 1;
   if (splits > a.nkb) splits = a.nkb;
   a.splits = splits;
-  a.ws = L->ws;
-  a.cnt = L->cnt;
+  if (!a.ws) {  // the layer's workspace unless the caller brings one
+    a.ws = L->ws;
+    a.cnt = L->cnt;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * splits));
   cfg.blockDim = dim3(serq::dtc::kThreads);
@@ -373,7 +375,8 @@ cudaError_t dispatch_tc(const serq_layer* L, const void* Xq, const serq::tc::Arg
 }
 
 serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, int M, void* Y, int ldy,
-                        int32_t* acc0, int32_t* acc1, serq_algo algo, void* stream) {
+                        int32_t* acc0, int32_t* acc1, serq_algo algo, void* stream, int32_t* scratch = nullptr,
+                        int32_t* scratch_cnt = nullptr) {
   serq_status s;
   if (!L) return fail(SERQ_ERR_INVALID_ARG, "null layer");
   const bool accum = (acc0 != nullptr);
@@ -405,7 +408,7 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
   if (algo == SERQ_ALGO_DECODE_TC) {
     serq::dtc::Args a{M, L->K, L->N, L->rpad, (L->K + serq::dtc::BK - 1) / serq::dtc::BK,
                       (L->rpad + serq::dtc::BK - 1) / serq::dtc::BK, 1, sx, L->sw, L->sr,
-                      static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1, nullptr, nullptr};
+                      static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1, scratch, scratch_cnt};
     if (a8)
       e = accum ? dispatch_decode_tc<true, true>(L, Xq, a, st) : dispatch_decode_tc<true, false>(L, Xq, a, st);
     else
@@ -439,6 +442,35 @@ serq_status check_rows(const void* X, int M, int K, int ld, int elem, const char
   if (ld < K) return fail(SERQ_ERR_INVALID_ARG, "leading dimension of %s (%d) < K (%d)", name, ld, K);
   if (!aligned16(X) || ((size_t)ld * elem) % 16)
     return fail(SERQ_ERR_INVALID_ARG, "%s rows must start 16-byte aligned", name);
+  return SERQ_OK;
+}
+
+// Scratch of serq_linear_decode_static: split-K partial sums [2][32][N] and
+// tile counters of the tensor-core decode kernel, compiled into the library
+// (one copy per device), so that the call allocates nothing.
+constexpr int kStaticMaxN = 16384;
+constexpr size_t kStaticCntOffset = (size_t)2 * serq::dtc::kMaxM * kStaticMaxN;
+constexpr size_t kStaticInts = kStaticCntOffset + kStaticMaxN / serq::dtc::BM;
+static __device__ __align__(256) int32_t g_decode_scratch[kStaticInts];
+
+// Device address of the scratch, looked up once per device; the first call
+// on a device clears it (it must start at zero; every completed call leaves
+// it zero).
+serq_status static_scratch(int32_t** out) {
+  static std::mutex mu;
+  static int32_t* addr[64] = {nullptr};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return fail(SERQ_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e == cudaSuccess) e = cudaMemset(p, 0, kStaticInts * sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "static decode scratch");
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = addr[dev];
   return SERQ_OK;
 }
 
@@ -684,6 +716,22 @@ serq_status serq_linear_accum(const serq_layer* layer, const void* Xq, int M, in
                               serq_algo algo, void* stream) {
   if (!acc0 || !acc1) return fail(SERQ_ERR_INVALID_ARG, "null acc0 or acc1");
   return linear_impl(layer, Xq, nullptr, M, nullptr, 0, acc0, acc1, algo, stream);
+}
+
+serq_status serq_linear_decode_static(const serq_layer* layer, const void* Xq, const float* sx, int M, void* Y,
+                                      int ldy, int32_t* acc0, int32_t* acc1, void* stream) {
+  if (!layer) return fail(SERQ_ERR_INVALID_ARG, "null layer");
+  if ((acc0 == nullptr) != (acc1 == nullptr)) return fail(SERQ_ERR_INVALID_ARG, "acc0 and acc1 go together");
+  if (M < 1 || M > serq::dtc::kMaxM)
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "serq_linear_decode_static takes 1 <= M <= %d (got %d)", serq::dtc::kMaxM, M);
+  if (layer->N > kStaticMaxN)
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "serq_linear_decode_static takes N <= %d (got %d)", kStaticMaxN, layer->N);
+  serq_status s = check_device();
+  if (s) return s;
+  int32_t* scratch = nullptr;
+  if ((s = static_scratch(&scratch))) return s;
+  return linear_impl(layer, Xq, sx, M, Y, ldy, acc0, acc1, SERQ_ALGO_DECODE_TC, stream, scratch,
+                     scratch + kStaticCntOffset);
 }
 
 }  // extern "C"

@@ -41,6 +41,7 @@ EXPORTS = {
     "serq_linear": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp]),
     "serq_linear_ex": (_i, [_vp, _vp, _vp, _i, _vp, _i, _i, _vp]),
     "serq_linear_accum": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp]),
+    "serq_linear_decode_static": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp]),
     "serq_silu_mul_quantize": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "serq_flatten_permute": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _i, _vp]),
     "serq_decode_max_m": (_i, []),
@@ -237,6 +238,25 @@ def linear_accum(layer: Layer, Xq: torch.Tensor, algo: int = ALGO_AUTO, stream=N
     _check(lib.serq_linear_accum(layer.handle, _ptr(Xq), M, _ptr(acc0), _ptr(acc1), algo, _stream(stream)),
            "serq_linear_accum")
     return acc0, acc1
+
+
+def linear_decode_static(layer: Layer, Xq: torch.Tensor, sx: Optional[torch.Tensor] = None,
+                         Y: Optional[torch.Tensor] = None, accum: bool = False, stream=None):
+    """serq_linear_decode_static: the tensor-core decode kernel with its
+    split-K scratch in the library's static per-device area (no allocation).
+    Returns Y (bf16), or (acc0, acc1) when accum is True."""
+    M = Xq.shape[0]
+    if accum:
+        acc0 = torch.empty((M, layer.N), dtype=torch.int32, device=Xq.device)
+        acc1 = torch.empty((M, layer.N), dtype=torch.int32, device=Xq.device)
+        _check(lib.serq_linear_decode_static(layer.handle, _ptr(Xq), None, M, None, 0, _ptr(acc0), _ptr(acc1),
+                                             _stream(stream)), "serq_linear_decode_static")
+        return acc0, acc1
+    if Y is None:
+        Y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=Xq.device)
+    _check(lib.serq_linear_decode_static(layer.handle, _ptr(Xq), _ptr(sx), M, _ptr(Y), Y.stride(0), None, None,
+                                         _stream(stream)), "serq_linear_decode_static")
+    return Y
 
 
 def device_error() -> int:
