@@ -123,15 +123,19 @@ struct LoadSiluMul {
 // codes in natural order.
 template <int Q, int RPL, class Loader>
 __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* __restrict__ Xq,
-                                                    float* __restrict__ sx) {
+                                                    float* __restrict__ sx, int early_launch) {
   constexpr int W = Loader::kWords;
   const int m = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int nrun = K >> 5;
   uint4 raw[RPL][4][W];
   float amax = 0.f;
-  // programmatic dependent launch: the input (written by the previous
-  // kernel) is read only after that kernel completed
+  // Programmatic dependent launch: the input (written by the previous
+  // kernel) is read only after that kernel completed.  A grid that is all
+  // resident at once lets the next kernel in right away (its weight prefetch
+  // overlaps this one); a larger grid only at its end, so the next kernel
+  // does not take SMs from rows still to come.
+  if (early_launch) grid_dep_launch();
   grid_dep_wait();
 #pragma unroll
   for (int i = 0; i < RPL; ++i) {
@@ -213,9 +217,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* _
       dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
   }
-  // the next kernel may be scheduled once every CTA got here: its prologue
-  // overlaps the last rows instead of taking SMs from the earlier ones
-  grid_dep_launch();
+  if (!early_launch) grid_dep_launch();
 }
 
 // Runs per lane held in registers: 4 for bf16 input (64 registers of raw
@@ -236,7 +238,11 @@ inline cudaError_t launch_quant_rows(const Loader& ld, int M, int K, uint8_t* Xq
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_quant_rows<Q, RPL, Loader>, ld, K, Xq, sx);
+  int sms = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int early = (M <= 4 * sms) ? 1 : 0;  // the whole grid is resident at once
+  return cudaLaunchKernelEx(&cfg, k_quant_rows<Q, RPL, Loader>, ld, K, Xq, sx, early);
 }
 
 // --------------------------------------------------- flatten and permute
