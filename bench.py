@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--algo", type=int, default=0,
                     help="serq_algo for every linear launch (0 = automatic choice)")
+    ap.add_argument("--no-group", action="store_true",
+                    help="one launch per projection instead of one per shared-input group")
     ap.add_argument("--profile", action="store_true",
                     help="short run for a profiler: no e2e, no CPU baseline")
     a = ap.parse_args()
@@ -201,6 +203,7 @@ class LayerWorkload:
         from w4a4_rank_gemm_b200 import synth
         self.S, self.torch, self.dev = S, torch, dev
         self.algo = args.algo
+        self.grouped = not args.no_group
         self.name = args.workload
         M = self.M = args.M
         if args.workload == "llama3_8b_w4a8":
@@ -234,9 +237,10 @@ class LayerWorkload:
         self.gemms = [(p.name, p.W.shape[0], p.W.shape[1]) for p in wl.projections]
         self.ops_step = sum(ops_of(M, K, N, r) for _, K, N in self.gemms)
         self.gemm_bytes_step = sum(linear_bytes(M, K, N, r, self.a_bits) for _, K, N in self.gemms)
-        self.launches_per_step = len(self.grp) + len(self.gemms)
-        self.weight_mb = sum(p.W.size for p in wl.projections) / 2 / 1e6
         self.decode = M <= S.decode_max_m()
+        n_gemm_launches = len(self.grp) if (self.grouped and not self.decode) else len(self.gemms)
+        self.launches_per_step = len(self.grp) + n_gemm_launches
+        self.weight_mb = sum(p.W.size for p in wl.projections) / 2 / 1e6
 
     def describe(self):
         shapes = ", ".join(f"{n} {K}x{N}" for n, K, N in self.gemms)
@@ -249,15 +253,30 @@ class LayerWorkload:
         for iname, projs in self.grp:
             if not gemm_only:
                 S.quantize_act(self.flat[iname][a], self.mode, Xq=self.Xq[iname], sx=self.sx[iname], stream=stream)
-            for p in projs:
+            for name, ps in self._launches(projs):
                 if events is not None:
                     e0 = torch.cuda.Event(enable_timing=True)
                     e1 = torch.cuda.Event(enable_timing=True)
                     e0.record(stream)
-                S.linear(self.layers[c][p.name], self.Xq[iname], self.sx[iname], Y=self.Y[p.name], algo=self.algo, stream=stream)
+                self._linear(c, iname, ps, stream)
                 if events is not None:
                     e1.record(stream)
-                    events.append((p.name, e0, e1))
+                    events.append((name, e0, e1))
+
+    def _launches(self, projs):
+        """[(name, [projection, ...]), ...]: one entry per GEMM call."""
+        if self.grouped and len(projs) > 1:
+            return [("+".join(p.name for p in projs), projs)]
+        return [(p.name, [p]) for p in projs]
+
+    def _linear(self, c, iname, ps, stream):
+        S = self.S
+        if len(ps) > 1:
+            S.linear_group([self.layers[c][p.name] for p in ps], self.Xq[iname], self.sx[iname],
+                           Ys=[self.Y[p.name] for p in ps], algo=self.algo, stream=stream)
+        else:
+            S.linear(self.layers[c][ps[0].name], self.Xq[iname], self.sx[iname], Y=self.Y[ps[0].name],
+                     algo=self.algo, stream=stream)
 
     def e2e_step(self, i, stream, host_in, host_out):
         S = self.S
@@ -266,9 +285,10 @@ class LayerWorkload:
             dev_in = self.flat[iname][1]
             dev_in.copy_(host_in[iname], non_blocking=True)
             S.quantize_act(dev_in, self.mode, Xq=self.Xq[iname], sx=self.sx[iname], stream=stream)
-            for p in projs:
-                S.linear(self.layers[c][p.name], self.Xq[iname], self.sx[iname], Y=self.Y[p.name], algo=self.algo, stream=stream)
-                host_out[p.name].copy_(self.Y[p.name], non_blocking=True)
+            for _, ps in self._launches(projs):
+                self._linear(c, iname, ps, stream)
+                for p in ps:
+                    host_out[p.name].copy_(self.Y[p.name], non_blocking=True)
 
     def host_buffers(self):
         torch = self.torch
@@ -285,6 +305,7 @@ class MLPWorkload:
         from w4a4_rank_gemm_b200 import synth
         self.S, self.torch, self.dev = S, torch, dev
         self.algo = args.algo
+        self.grouped = not args.no_group
         self.name = "mlp_block"
         M = self.M = args.M
         blk = synth.mlp_block(M=M)
@@ -314,7 +335,7 @@ class MLPWorkload:
         self.gemms = [("gate_proj", K, F), ("up_proj", K, F), ("down_proj", F, K)]
         self.ops_step = sum(ops_of(M, k, n, r) for _, k, n in self.gemms)
         self.gemm_bytes_step = sum(linear_bytes(M, k, n, r, 4) for _, k, n in self.gemms)
-        self.launches_per_step = 5
+        self.launches_per_step = 4 if self.grouped else 5
         self.weight_mb = 3 * K * F / 2 / 1e6
         self.decode = False
         torch.cuda.synchronize()
@@ -329,16 +350,24 @@ class MLPWorkload:
         Lg, Lu, Ld = self.copies[i % N_WEIGHT_COPIES]
         if not gemm_only:
             S.quantize_act(self.flat[i % N_ACT_COPIES], "w4a4", Xq=self.Xq, sx=self.sx, stream=stream)
-        for name, L, xq, sx, y, pre in (("gate_proj", Lg, self.Xq, self.sx, self.G, None),
-                                        ("up_proj", Lu, self.Xq, self.sx, self.U, None),
-                                        ("down_proj", Ld, self.Hq, self.hsx, self.Yd, "silu")):
+        if self.grouped:
+            calls = (("gate_proj+up_proj", [Lg, Lu], self.Xq, self.sx, [self.G, self.U], None),
+                     ("down_proj", [Ld], self.Hq, self.hsx, [self.Yd], "silu"))
+        else:
+            calls = (("gate_proj", [Lg], self.Xq, self.sx, [self.G], None),
+                     ("up_proj", [Lu], self.Xq, self.sx, [self.U], None),
+                     ("down_proj", [Ld], self.Hq, self.hsx, [self.Yd], "silu"))
+        for name, Ls, xq, sx, ys, pre in calls:
             if pre == "silu" and not gemm_only:
                 S.silu_mul_quantize(self.G, self.U, "w4a4", Xq=self.Hq, sx=self.hsx, stream=stream)
             if events is not None:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            S.linear(L, xq, sx, Y=y, algo=self.algo, stream=stream)
+            if len(Ls) > 1:
+                S.linear_group(Ls, xq, sx, Ys=ys, algo=self.algo, stream=stream)
+            else:
+                S.linear(Ls[0], xq, sx, Y=ys[0], algo=self.algo, stream=stream)
             if events is not None:
                 e1.record(stream)
                 events.append((name, e0, e1))
@@ -467,6 +496,7 @@ def run_gpu(args, rank, world, local_rank):
                   f"({N_WEIGHT_COPIES} x {W.weight_mb:.0f} MB packed) and {N_ACT_COPIES} activation copies alternated",
             "cuda_graphs": graphs is not None,
             "algo": args.algo,
+            "grouped_launches": W.grouped and not W.decode,
         },
         "gpu_launches": W.launches_per_step * args.steps,
         "clocks": clk.summary(),

@@ -187,6 +187,35 @@ serq_status serq_linear_accum(const serq_layer* layer, const void* Xq, int M, in
                               int32_t* acc1, serq_algo algo, void* stream);
 
 /*
+ * serq_linear_group -- serq_linear (or, with acc0/acc1, the accumulator
+ * hook) for n layers that read the same activation codes, such as a
+ * block's q/k/v projections or its gate/up pair (key design 2, applied to
+ * each layer; the pages run them as separate GEMMs).  With a prefill kernel
+ * the n products run as one launch over the union of their output tiles, so
+ * setup and the last partial wave are paid once; decode kernels and
+ * SERQ_ALGO_PREFILL_PAIR_TMEM_A run one launch per layer.  Results are
+ * identical to n serq_linear_ex calls with the same kernel.
+ *  n        1..4.
+ *  layers   HOST array of n layers with equal K and mode and ranks that
+ *           round up to the same multiple of 32 (N may differ).
+ *  Xq, sx   DEVICE, as serq_linear; the codes are read in each layer's
+ *           input order, so the layers normally come from one
+ *           serq_prepare_group call (one smoothing vector and order).
+ *  Y, ldy   HOST arrays of n DEVICE bf16 outputs (M x N_l, row stride
+ *           ldy[l] >= N_l) and their strides; may be null when acc0/acc1
+ *           are given.
+ *  acc0, acc1  both null, or HOST arrays of n DEVICE int32 M x N_l outputs
+ *           (exact accumulators; sx and Y are then not used).
+ *  algo     as serq_linear_ex (AUTO picks by M and the group's total tiles).
+ * Asynchronous.  Uses no memory beyond its arguments and the layers.
+ * Errors: SERQ_ERR_INVALID_ARG for n out of range or layers that differ in
+ * K, padded rank or mode, and every serq_linear_ex error of any member.
+ */
+serq_status serq_linear_group(int n, const serq_layer* const* layers, const void* Xq, const float* sx,
+                              int M, void* const* Y, const int* ldy, int32_t* const* acc0,
+                              int32_t* const* acc1, serq_algo algo, void* stream);
+
+/*
  * serq_linear_decode_static -- serq_linear (or, with acc0/acc1, the
  * accumulator hook) through the tensor-core decode kernel
  * (SERQ_ALGO_DECODE_TC) with its split-K partial sums and tile counters in a

@@ -58,6 +58,45 @@ struct Args {
   int tiles_m, tiles_n;  // output tiles (BM * cluster rows x BN columns)
 };
 
+// k_gemm runs one launch over the output tiles of up to kMaxGroup layers that
+// read the same activation codes (q/k/v, gate/up): per layer its width, the
+// first tile index, its scales and its output.
+constexpr int kMaxGroup = 4;
+struct LayerOut {
+  int N, tile_base;
+  const float* sw;
+  const float* sr;
+  __nv_bfloat16* Y;
+  int ldy;
+  int32_t* acc0;
+  int32_t* acc1;
+};
+struct GroupArgs {
+  int M, K, rpad;
+  int nkb, nrb;
+  const float* sx;
+  int tiles_m;
+  int nlayers, ntiles;
+  LayerOut lo[kMaxGroup];
+};
+// Per-layer tensor maps: weights and compensator (box rows BN / CG) and the
+// bf16 output (32 x 64 boxes).
+struct GroupMaps {
+  CUtensorMap b[kMaxGroup];
+  CUtensorMap r[kMaxGroup];
+  CUtensorMap y[kMaxGroup];
+};
+
+// Layer of tile t and its tile index within that layer.
+__device__ __forceinline__ int layer_of(const GroupArgs& p, int t, int& tl) {
+  int l = 0;
+#pragma unroll
+  for (int i = 1; i < kMaxGroup; ++i)
+    if (i < p.nlayers && t >= p.lo[i].tile_base) l = i;
+  tl = t - p.lo[l].tile_base;
+  return l;
+}
+
 // Shared memory: PS packed stages [A | B] written by TMA, US widened stages
 // [A | B] read by the MMAs (W4A8: A is consumed straight from the packed
 // stage, already in the MMA layout), per-warp epilogue scales, barriers.
@@ -147,8 +186,7 @@ __device__ __forceinline__ void cta_sync() {
 // -> mbarrier arrive -> MMA warp wait -> tcgen05.fence::after_thread_sync).
 template <int BN, bool A8, bool ACC_OUT, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmY, const Args p) {
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ GroupMaps mp, const GroupArgs p) {
   using L = Layout<BN, A8, CG>;
   constexpr int PS = L::PS, US = L::US;
   extern __shared__ uint8_t smem_raw[];
@@ -170,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = (rank == 0);
   const int cta_tile = (int)blockIdx.x / CG;            // this CTA (pair)'s first tile
   const int tile_stride = (int)gridDim.x / CG;
-  const int ntiles = p.tiles_m * p.tiles_n;
+  const int ntiles = p.ntiles;
   const int nsteps = p.nkb + p.nrb;
 
   if (threadIdx.x == 0) {
@@ -193,9 +231,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    tma_prefetch_desc(&tmR);
-    if (!ACC_OUT) tma_prefetch_desc(&tmY);
+    for (int l = 0; l < p.nlayers; ++l) {
+      tma_prefetch_desc(&mp.b[l]);
+      tma_prefetch_desc(&mp.r[l]);
+      if (!ACC_OUT) tma_prefetch_desc(&mp.y[l]);
+    }
   }
   if (warp == 1) {
     tmem_alloc<CG>(tmem_slot, L::kTmemCols);
@@ -216,11 +256,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // wait; the A tiles follow once the activation codes are final.
       int npre = 0;
       for (int t = cta_tile, step = 0; npre < PS && t < ntiles; ++npre) {
-        const int nb0 = (t / p.tiles_m) * BN + (int)rank * L::BNL;
+        int tl;
+        const int l = layer_of(p, t, tl);
+        const int nb0 = (tl / p.tiles_m) * BN + (int)rank * L::BNL;
         const bool res = step >= p.nkb;
         const int j = res ? step - p.nkb : step;
         mbar_arrive_expect_tx(&full_pk[npre], L::kTxBytes);
-        tma_load_2d(smem + L::oPk + npre * L::kPk + L::kPkA, res ? &tmR : &tmB, &full_pk[npre], j * (BK / 2), nb0);
+        tma_load_2d(smem + L::oPk + npre * L::kPk + L::kPkA, res ? &mp.r[l] : &mp.b[l], &full_pk[npre], j * (BK / 2),
+                    nb0);
         if (++step == nsteps) {
           step = 0;
           t += tile_stride;
@@ -230,8 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int g = 0;  // pipeline step across tiles
       bool ok = true;
       for (int t = cta_tile; ok && t < ntiles; t += tile_stride) {
-        const int m0 = ((t % p.tiles_m) * CG + (int)rank) * BM;
-        const int nb0 = (t / p.tiles_m) * BN + (int)rank * L::BNL;
+        int tl;
+        const int l = layer_of(p, t, tl);
+        const int m0 = ((tl % p.tiles_m) * CG + (int)rank) * BM;
+        const int nb0 = (tl / p.tiles_m) * BN + (int)rank * L::BNL;
         for (int step = 0; step < nsteps; ++step, ++g) {
           const int s = g % PS;
           const uint32_t ph = (g / PS) & 1;
@@ -241,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (g >= npre) {
             if (!mbar_wait(&empty_pk[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) { ok = false; break; }
             mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
-            tma_load_2d(stage + L::kPkA, res ? &tmR : &tmB, &full_pk[s], j * (BK / 2), nb0);
+            tma_load_2d(stage + L::kPkA, res ? &mp.r[l] : &mp.b[l], &full_pk[s], j * (BK / 2), nb0);
           }
           tma_load_2d(stage, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
         }
@@ -398,17 +443,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     int pre_end = 0;  // steps before this were widened ahead of their tile
     for (int t = cta_tile; ok && t < ntiles; t += tile_stride, ++it) {
-      const int tm = t % p.tiles_m;
-      const int m0 = (tm * CG + (int)rank) * BM;
-      const int n0 = (t / p.tiles_m) * BN;
+      int tl;
+      const int l = layer_of(p, t, tl);
+      const LayerOut& lo = p.lo[l];
+      const int m0 = ((tl % p.tiles_m) * CG + (int)rank) * BM;
+      const int n0 = (tl / p.tiles_m) * BN;
       // prefetch this tile's epilogue scales (consumed after the k loop)
       float swv[kCpl], srv[kCpl], sxv = 0.f;
       if (!ACC_OUT) {
 #pragma unroll
         for (int i = 0; i < kCpl; ++i) {
           const int n = n0 + eh * kHalf + kCpl * lane + i;
-          swv[i] = (n < p.N) ? __ldg(p.sw + n) : 0.f;
-          srv[i] = (n < p.N) ? __ldg(p.sr + n) : 0.f;
+          swv[i] = (n < lo.N) ? __ldg(lo.sw + n) : 0.f;
+          srv[i] = (n < lo.N) ? __ldg(lo.sr + n) : 0.f;
         }
         const int row = m0 + eq * 32 + lane;
         sxv = (row < p.M) ? __ldg(p.sx + row) : 0.f;
@@ -446,9 +493,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) r1[i] = 0;
           }
-          if (row < p.M && n0 + c < p.N) {
-            int32_t* o0 = p.acc0 + (size_t)row * p.N + n0 + c;
-            int32_t* o1 = p.acc1 + (size_t)row * p.N + n0 + c;
+          if (row < p.M && n0 + c < lo.N) {
+            int32_t* o0 = lo.acc0 + (size_t)row * lo.N + n0 + c;
+            int32_t* o1 = lo.acc1 + (size_t)row * lo.N + n0 + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
               *reinterpret_cast<int4*>(o0 + i) =
@@ -567,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int b = 0; b < kHalf / 64; ++b) {
             const int x = n0 + eh * kHalf + b * 64;
-            if (x < p.N && y < p.M) tma_store_2d(&tmY, box_ptr(eq * (BN / 64) + eh * (kHalf / 64) + b), x, y);
+            if (x < lo.N && y < p.M) tma_store_2d(&mp.y[l], box_ptr(eq * (BN / 64) + eh * (kHalf / 64) + b), x, y);
           }
           bulk_commit_group();
           bulk_wait_read_all();

@@ -222,23 +222,54 @@ int max_smem() {
 }
 
 // ------------------------------------------------------------ GEMM launch
+// Layers whose products one launch computes (they read the same activation
+// codes), with their outputs.
+struct LinearGroup {
+  int n;
+  const serq_layer* L[serq::tc::kMaxGroup];
+  __nv_bfloat16* Y[serq::tc::kMaxGroup];
+  int ldy[serq::tc::kMaxGroup];
+  int32_t* acc0[serq::tc::kMaxGroup];
+  int32_t* acc1[serq::tc::kMaxGroup];
+};
+
 template <int BN, bool A8, bool ACC, int CG>
-cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, cudaStream_t st) {
+cudaError_t launch_tc(const LinearGroup& G, const void* Xq, const float* sx, int M, cudaStream_t st) {
   using Lay = serq::tc::Layout<BN, A8, CG>;
+  const serq_layer* L0 = G.L[0];
+  const int K = L0->K;
   CUtensorMap tmA;
-  bool okm = A8 ? make_map(&tmA, Xq, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K, 128, 128,
-                           CU_TENSOR_MAP_SWIZZLE_128B)
-                : make_map(&tmA, Xq, (uint64_t)a.K / 2, (uint64_t)a.M, (uint64_t)a.K / 2, 64, 128,
-                           CU_TENSOR_MAP_SWIZZLE_NONE);
+  bool okm = A8 ? make_map(&tmA, Xq, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)
+                : make_map(&tmA, Xq, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!okm) return cudaErrorInvalidValue;
-  // output: bf16 [M][N] with row stride ldy, boxes of 32 rows x 64 columns
-  CUtensorMap tmY = tmA;
-  if (!ACC && !make_map(&tmY, a.Y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.ldy * 2, 64, 32,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
-    return cudaErrorInvalidValue;
   // weight maps by box rows: [0] 128, [1] 256 (BN / CG rows per CTA)
   const int bi = (BN / CG == 256) ? 1 : 0;
   static_assert(BN / CG == 128 || BN / CG == 256, "weight box rows");
+  serq::tc::GroupArgs ga = {};
+  serq::tc::GroupMaps mp;
+  ga.M = M;
+  ga.K = K;
+  ga.rpad = L0->rpad;
+  ga.nkb = (K + serq::tc::BK - 1) / serq::tc::BK;
+  ga.nrb = (L0->rpad + serq::tc::BK - 1) / serq::tc::BK;
+  ga.sx = sx;
+  ga.tiles_m = (M + serq::tc::BM * CG - 1) / (serq::tc::BM * CG);
+  ga.nlayers = G.n;
+  int base = 0;
+  for (int l = 0; l < serq::tc::kMaxGroup; ++l) {
+    const int li = (l < G.n) ? l : 0;  // unused slots repeat layer 0
+    const serq_layer* Ll = G.L[li];
+    mp.b[l] = Ll->tmB[bi];
+    mp.r[l] = Ll->tmR[bi];
+    mp.y[l] = tmA;
+    // output: bf16 [M][N] with row stride ldy, boxes of 32 rows x 64 columns
+    if (!ACC && !make_map(&mp.y[l], G.Y[li], (uint64_t)Ll->N, (uint64_t)M, (uint64_t)G.ldy[li] * 2, 64, 32,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+      return cudaErrorInvalidValue;
+    ga.lo[l] = serq::tc::LayerOut{Ll->N, base, Ll->sw, Ll->sr, G.Y[li], G.ldy[li], G.acc0[li], G.acc1[li]};
+    if (l < G.n) base += ga.tiles_m * ((Ll->N + BN - 1) / BN);
+  }
+  ga.ntiles = base;
   auto kern = serq::tc::k_gemm<BN, A8, ACC, CG>;
   static int attr_set[64] = {0};
   int dev = 0;
@@ -248,12 +279,8 @@ cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args&
     attr_set[dev] = 1;
   }
   // persistent: one CTA (pair) per SM (pair of SMs), tiles strided over them
-  serq::tc::Args ap = a;
-  ap.tiles_m = (a.M + serq::tc::BM * CG - 1) / (serq::tc::BM * CG);
-  ap.tiles_n = (a.N + BN - 1) / BN;
-  const long ntiles = (long)ap.tiles_m * ap.tiles_n;
   const long slots = sm_count() / CG;
-  dim3 grid((unsigned)((ntiles < slots ? ntiles : slots) * CG), 1);
+  dim3 grid((unsigned)((base < slots ? base : slots) * CG), 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(serq::tc::kThreads);
@@ -268,7 +295,7 @@ cudaError_t launch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args&
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, tmA, L->tmB[bi], L->tmR[bi], tmY, ap);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, mp, ga);
 }
 
 // W4A4 on CTA pairs with the activations in tensor memory, 256 x 192 tiles.
@@ -356,28 +383,35 @@ cudaError_t dispatch_decode_tc(const serq_layer* L, const void* Xq, const serq::
 }
 
 template <bool A8, bool ACC>
-cudaError_t dispatch_tc(const serq_layer* L, const void* Xq, const serq::tc::Args& a, serq_algo algo,
+cudaError_t dispatch_tc(const LinearGroup& G, const void* Xq, const float* sx, int M, serq_algo algo,
                         cudaStream_t st) {
   switch (algo) {
-    case SERQ_ALGO_PREFILL_N128: return launch_tc<128, A8, ACC, 1>(L, Xq, a, st);
-    case SERQ_ALGO_PREFILL_N256: return launch_tc<256, A8, ACC, 1>(L, Xq, a, st);
-    case SERQ_ALGO_PREFILL_PAIR_N256: return launch_tc<256, A8, ACC, 2>(L, Xq, a, st);
-    case SERQ_ALGO_PREFILL_PAIR_TMEM_A:
-      if (A8) return cudaErrorInvalidValue;
+    case SERQ_ALGO_PREFILL_N128: return launch_tc<128, A8, ACC, 1>(G, Xq, sx, M, st);
+    case SERQ_ALGO_PREFILL_N256: return launch_tc<256, A8, ACC, 1>(G, Xq, sx, M, st);
+    case SERQ_ALGO_PREFILL_PAIR_N256: return launch_tc<256, A8, ACC, 2>(G, Xq, sx, M, st);
+    case SERQ_ALGO_PREFILL_PAIR_TMEM_A: {
+      if (A8 || G.n != 1) return cudaErrorInvalidValue;
+      const serq_layer* L = G.L[0];
+      serq::tc::Args a{M, L->K, L->N, L->rpad, (L->K + serq::tc::BK - 1) / serq::tc::BK,
+                       (L->rpad + serq::tc::BK - 1) / serq::tc::BK, sx, L->sw, L->sr, G.Y[0], G.ldy[0],
+                       G.acc0[0], G.acc1[0]};
       return launch_tc_ta<ACC>(L, Xq, a, st);
+    }
     default: break;
   }
   // CTA pairs with 256 x 256 tiles unless that leaves most SMs idle; then
   // single-CTA 128 x 128 tiles.
-  const long ctas_pair = (long)((a.N + 255) / 256) * 2 * ((a.M + 255) / 256);
-  if (ctas_pair * 10 >= (long)sm_count() * 9) return launch_tc<256, A8, ACC, 2>(L, Xq, a, st);
-  return launch_tc<128, A8, ACC, 1>(L, Xq, a, st);
+  long ctas_pair = 0;
+  for (int l = 0; l < G.n; ++l) ctas_pair += (long)((G.L[l]->N + 255) / 256) * 2 * ((M + 255) / 256);
+  if (ctas_pair * 10 >= (long)sm_count() * 9) return launch_tc<256, A8, ACC, 2>(G, Xq, sx, M, st);
+  return launch_tc<128, A8, ACC, 1>(G, Xq, sx, M, st);
 }
 
-serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, int M, void* Y, int ldy,
-                        int32_t* acc0, int32_t* acc1, serq_algo algo, void* stream, int32_t* scratch = nullptr,
-                        int32_t* scratch_cnt = nullptr) {
+// Argument checks shared by the single-layer and grouped calls; resolves AUTO.
+serq_status check_linear(const serq_layer* L, const void* Xq, const float* sx, int M, const void* Y, int ldy,
+                         const int32_t* acc0, const int32_t* acc1, serq_algo* algo_io) {
   serq_status s;
+  serq_algo algo = *algo_io;
   if (!L) return fail(SERQ_ERR_INVALID_ARG, "null layer");
   const bool accum = (acc0 != nullptr);
   if (!Xq) return fail(SERQ_ERR_INVALID_ARG, "null Xq");
@@ -402,6 +436,16 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
     return fail(SERQ_ERR_INVALID_ARG, "SERQ_ALGO_PREFILL_PAIR_TMEM_A takes W4A4 layers");
   if ((s = check_device())) return s;
   if ((s = check_layer(L))) return s;
+  *algo_io = algo;
+  return ok();
+}
+
+serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, int M, void* Y, int ldy,
+                        int32_t* acc0, int32_t* acc1, serq_algo algo, void* stream, int32_t* scratch = nullptr,
+                        int32_t* scratch_cnt = nullptr) {
+  serq_status s;
+  if ((s = check_linear(L, Xq, sx, M, Y, ldy, acc0, acc1, &algo))) return s;
+  const bool accum = (acc0 != nullptr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool a8 = (L->mode == SERQ_W4A8);
   cudaError_t e;
@@ -423,15 +467,71 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
       e = accum ? serq::decode::launch<false, true>(a, sm_count(), max_smem(), st)
                 : serq::decode::launch<false, false>(a, sm_count(), max_smem(), st);
   } else {
-    serq::tc::Args a{M, L->K, L->N, L->rpad, (L->K + serq::tc::BK - 1) / serq::tc::BK,
-                     (L->rpad + serq::tc::BK - 1) / serq::tc::BK, sx, L->sw, L->sr,
-                     static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1};
+    LinearGroup G = {};
+    G.n = 1;
+    G.L[0] = L;
+    G.Y[0] = static_cast<__nv_bfloat16*>(Y);
+    G.ldy[0] = ldy;
+    G.acc0[0] = acc0;
+    G.acc1[0] = acc1;
     if (a8)
-      e = accum ? dispatch_tc<true, true>(L, Xq, a, algo, st) : dispatch_tc<true, false>(L, Xq, a, algo, st);
+      e = accum ? dispatch_tc<true, true>(G, Xq, sx, M, algo, st) : dispatch_tc<true, false>(G, Xq, sx, M, algo, st);
     else
-      e = accum ? dispatch_tc<false, true>(L, Xq, a, algo, st) : dispatch_tc<false, false>(L, Xq, a, algo, st);
+      e = accum ? dispatch_tc<false, true>(G, Xq, sx, M, algo, st) : dispatch_tc<false, false>(G, Xq, sx, M, algo, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "serq_linear launch");
+  return ok();
+}
+
+// Several layers over the same activation codes: prefill kernels run them as
+// one launch (one tile space, one pass of setup and tail); decode kernels and
+// the TMEM-activation variant run them one launch per layer.
+serq_status group_impl(int n, const serq_layer* const* Ls, const void* Xq, const float* sx, int M,
+                       void* const* Y, const int* ldy, int32_t* const* acc0, int32_t* const* acc1, serq_algo algo,
+                       void* stream) {
+  serq_status s;
+  if (n < 1 || n > serq::tc::kMaxGroup)
+    return fail(SERQ_ERR_INVALID_ARG, "group of %d layers (1..%d)", n, serq::tc::kMaxGroup);
+  if (!Ls) return fail(SERQ_ERR_INVALID_ARG, "null layer list");
+  if ((acc0 == nullptr) != (acc1 == nullptr)) return fail(SERQ_ERR_INVALID_ARG, "acc0 and acc1: both or neither");
+  const bool accum = (acc0 != nullptr);
+  if (!accum && (!Y || !ldy)) return fail(SERQ_ERR_INVALID_ARG, "null Y or ldy list");
+  serq_algo resolved = algo;
+  for (int l = 0; l < n; ++l) {
+    if (!Ls[l]) return fail(SERQ_ERR_INVALID_ARG, "null layer %d", l);
+    if (Ls[l]->K != Ls[0]->K || Ls[l]->rpad != Ls[0]->rpad || Ls[l]->mode != Ls[0]->mode)
+      return fail(SERQ_ERR_INVALID_ARG, "layer %d differs from layer 0 in K, rank or mode", l);
+    serq_algo a = algo;
+    if ((s = check_linear(Ls[l], Xq, sx, M, accum ? nullptr : Y[l], accum ? 0 : ldy[l], accum ? acc0[l] : nullptr,
+                          accum ? acc1[l] : nullptr, &a)))
+      return s;
+    resolved = a;
+  }
+  if (resolved == SERQ_ALGO_DECODE || resolved == SERQ_ALGO_DECODE_TC || resolved == SERQ_ALGO_PREFILL_PAIR_TMEM_A) {
+    for (int l = 0; l < n; ++l)
+      if ((s = linear_impl(Ls[l], Xq, sx, M, accum ? nullptr : Y[l], accum ? 0 : ldy[l], accum ? acc0[l] : nullptr,
+                           accum ? acc1[l] : nullptr, resolved, stream)))
+        return s;
+    return ok();
+  }
+  LinearGroup G = {};
+  G.n = n;
+  for (int l = 0; l < n; ++l) {
+    G.L[l] = Ls[l];
+    G.Y[l] = accum ? nullptr : static_cast<__nv_bfloat16*>(Y[l]);
+    G.ldy[l] = accum ? 0 : ldy[l];
+    G.acc0[l] = accum ? acc0[l] : nullptr;
+    G.acc1[l] = accum ? acc1[l] : nullptr;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (Ls[0]->mode == SERQ_W4A8)
+    e = accum ? dispatch_tc<true, true>(G, Xq, sx, M, resolved, st)
+              : dispatch_tc<true, false>(G, Xq, sx, M, resolved, st);
+  else
+    e = accum ? dispatch_tc<false, true>(G, Xq, sx, M, resolved, st)
+              : dispatch_tc<false, false>(G, Xq, sx, M, resolved, st);
+  if (e != cudaSuccess) return cuda_fail(e, "serq_linear_group launch");
   return ok();
 }
 
@@ -716,6 +816,12 @@ serq_status serq_linear_accum(const serq_layer* layer, const void* Xq, int M, in
                               serq_algo algo, void* stream) {
   if (!acc0 || !acc1) return fail(SERQ_ERR_INVALID_ARG, "null acc0 or acc1");
   return linear_impl(layer, Xq, nullptr, M, nullptr, 0, acc0, acc1, algo, stream);
+}
+
+serq_status serq_linear_group(int n, const serq_layer* const* layers, const void* Xq, const float* sx, int M,
+                              void* const* Y, const int* ldy, int32_t* const* acc0, int32_t* const* acc1,
+                              serq_algo algo, void* stream) {
+  return group_impl(n, layers, Xq, sx, M, Y, ldy, acc0, acc1, algo, stream);
 }
 
 serq_status serq_linear_decode_static(const serq_layer* layer, const void* Xq, const float* sx, int M, void* Y,

@@ -42,6 +42,8 @@ EXPORTS = {
     "serq_linear_ex": (_i, [_vp, _vp, _vp, _i, _vp, _i, _i, _vp]),
     "serq_linear_accum": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp]),
     "serq_linear_decode_static": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp]),
+    "serq_linear_group": (_i, [_i, ctypes.POINTER(_vp), _vp, _vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_i),
+                               ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp]),
     "serq_silu_mul_quantize": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "serq_flatten_permute": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _i, _vp]),
     "serq_decode_max_m": (_i, []),
@@ -238,6 +240,31 @@ def linear_accum(layer: Layer, Xq: torch.Tensor, algo: int = ALGO_AUTO, stream=N
     _check(lib.serq_linear_accum(layer.handle, _ptr(Xq), M, _ptr(acc0), _ptr(acc1), algo, _stream(stream)),
            "serq_linear_accum")
     return acc0, acc1
+
+
+def linear_group(layers, Xq: torch.Tensor, sx: Optional[torch.Tensor] = None, Ys=None,
+                 algo: int = ALGO_AUTO, accum: bool = False, stream=None):
+    """serq_linear_group: the products of up to four layers that share the
+    activation codes Xq (equal K, rank and mode), as one prefill launch.
+    Returns the list of bf16 outputs, or of (acc0, acc1) pairs when accum."""
+    n = len(layers)
+    M = Xq.shape[0]
+    hl = (_vp * n)(*[L.handle for L in layers])
+    if accum:
+        accs = [(torch.empty((M, L.N), dtype=torch.int32, device=Xq.device),
+                 torch.empty((M, L.N), dtype=torch.int32, device=Xq.device)) for L in layers]
+        a0 = (_vp * n)(*[_ptr(a[0]) for a in accs])
+        a1 = (_vp * n)(*[_ptr(a[1]) for a in accs])
+        _check(lib.serq_linear_group(n, hl, _ptr(Xq), None, M, None, None, a0, a1, algo, _stream(stream)),
+               "serq_linear_group")
+        return accs
+    if Ys is None:
+        Ys = [torch.empty((M, L.N), dtype=torch.bfloat16, device=Xq.device) for L in layers]
+    yp = (_vp * n)(*[_ptr(Y) for Y in Ys])
+    ld = (_i * n)(*[Y.stride(0) for Y in Ys])
+    _check(lib.serq_linear_group(n, hl, _ptr(Xq), _ptr(sx), M, yp, ld, None, None, algo, _stream(stream)),
+           "serq_linear_group")
+    return Ys
 
 
 def linear_decode_static(layer: Layer, Xq: torch.Tensor, sx: Optional[torch.Tensor] = None,
