@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--algo", type=int, default=0,
                     help="serq_algo for every linear launch (0 = automatic choice)")
+    ap.add_argument("--mode", choices=["w4a4", "w4a8"], default=None,
+                    help="override the workload's quantization mode (same shapes)")
     ap.add_argument("--no-group", action="store_true",
                     help="one launch per projection instead of one per shared-input group")
     ap.add_argument("--profile", action="store_true",
@@ -210,6 +212,8 @@ class LayerWorkload:
             wl = synth.llama3_8b(M=M)
         else:
             wl = synth.llama2_7b(M=M)
+        if args.mode is not None:
+            wl.mode = args.mode
         self.wl = wl
         self.mode = wl.mode
         self.a_bits = 4 if wl.mode == "w4a4" else 8

@@ -488,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t r0[32], r1[32];
           tmem_ld_32x32b_x32(tq + (uint32_t)c, r0);
           if (has_r) tmem_ld_32x32b_x32(tq + (uint32_t)(BN + c), r1);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(r0);
+          tmem_ld_wait_regs(r1);
           if (!has_r) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) r1[i] = 0;
@@ -559,6 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 16; ++i) d1[i] = 0;
           }
         };
+        // Scales of the next group of four columns are loaded while the
+        // current group is converted (carried across chunks), so their
+        // shared-memory latency stays off the conversion's dependency chain.
+        float4 wn = sw4[0], rn = sr4[0];
         auto convert_chunk = [&](const uint32_t(&r0)[16], const uint32_t(&r1)[16], int cc) {
           const int c = eh * kHalf + cc;  // tile column of this 16-column chunk
           // 128-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)
@@ -574,8 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               // accumulators converted as they come out of TMEM (x256 or x16;
               // the factor is in sw', sR')
               const int e = 8 * k + i;
-              const float4 w = sw4[(cc + e) >> 2];
-              const float4 rr = sr4[(cc + e) >> 2];
+              const float4 w = wn, rr = rn;
+              const int nx = (cc + e + 4 < kHalf) ? (cc + e + 4) >> 2 : 0;  // next group (wraps at the end)
+              wn = sw4[nx];
+              rn = sr4[nx];
               const float2 f0a = make_float2((float)(int)r0[e], (float)(int)r0[e + 1]);
               const float2 f0b = make_float2((float)(int)r0[e + 2], (float)(int)r0[e + 3]);
               const float2 f1a = make_float2((float)(int)r1[e], (float)(int)r1[e + 1]);
@@ -945,7 +952,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t r0[32], r1[32];
           tmem_ld_32x32b_x32(tq + (uint32_t)c, r0);
           if (has_r) tmem_ld_32x32b_x32(tq + (uint32_t)(BN + c), r1);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(r0);
+          tmem_ld_wait_regs(r1);
           if (!has_r) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) r1[i] = 0;
@@ -991,7 +999,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t r0[32], r1[32];
           tmem_ld_32x32b_x32(tq + (uint32_t)c, r0);
           if (has_r) tmem_ld_32x32b_x32(tq + (uint32_t)(BN + c), r1);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(r0);
+          tmem_ld_wait_regs(r1);
           if (!has_r) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) r1[i] = 0;

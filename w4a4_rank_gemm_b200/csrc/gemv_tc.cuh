@@ -263,7 +263,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(tq, a0);
         if (nres > 0) tmem_ld_32x32b_x32(tq + MP, a1);
       }
-      tmem_ld_wait();
+      if constexpr (MP == 16) {
+        tmem_ld_wait_regs(a0, a1);
+      } else {
+        tmem_ld_wait_regs(a0);
+        tmem_ld_wait_regs(a1);
+      }
       if (nres == 0) {
 #pragma unroll
         for (int m = 0; m < MP; ++m) a1[m] = 0;
