@@ -72,6 +72,29 @@ def test_host_side_argument_rejection(lib):
     assert L.serq_silu_mul_quantize(None, None, 4, 256, 256, lib.W4A4, None, None, None) == lib.ERR_INVALID_ARG
 
 
+def test_group_call_host_side_rejection(lib):
+    """serq_linear_group checks the group on the host before any device call."""
+    L = lib.lib
+    fake = ctypes.c_void_p(0x1000)
+    layers = (ctypes.c_void_p * 5)(0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    ys = (ctypes.c_void_p * 5)(0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    ld = (ctypes.c_int * 5)(256, 256, 256, 256, 256)
+    for n in (0, 5, -1):
+        assert L.serq_linear_group(n, layers, fake, fake, 16, ys, ld, None, None, 0, None) == lib.ERR_INVALID_ARG
+        assert b"group of" in L.serq_last_error_string()
+    assert L.serq_linear_group(2, None, fake, fake, 16, ys, ld, None, None, 0, None) == lib.ERR_INVALID_ARG
+    # accumulators: both or neither
+    accs = (ctypes.c_void_p * 2)(0x1000, 0x1000)
+    assert L.serq_linear_group(2, layers, fake, None, 16, None, None, accs, None, 0, None) == lib.ERR_INVALID_ARG
+    assert b"both or neither" in L.serq_last_error_string()
+    # outputs missing when no accumulators are given
+    assert L.serq_linear_group(2, layers, fake, fake, 16, None, None, None, None, 0, None) == lib.ERR_INVALID_ARG
+    # a null layer in the list (checked before the layer is read)
+    layers[0] = None
+    assert L.serq_linear_group(2, layers, fake, fake, 16, ys, ld, None, None, 0, None) == lib.ERR_INVALID_ARG
+    assert b"null layer 0" in L.serq_last_error_string()
+
+
 def test_binding_refuses_to_load_without_library(tmp_path, monkeypatch):
     """The product path fails loudly when the CUDA library is missing."""
     import importlib.util
