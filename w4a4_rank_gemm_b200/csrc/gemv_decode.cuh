@@ -164,7 +164,10 @@ __device__ __forceinline__ void mma_seg(const Seg<MT, A8>& s, bool with_r, int (
 }
 
 template <int MT, bool A8, bool ACC_OUT, bool ACT_SMEM>
-__global__ void __launch_bounds__(kThreads, 1) k_decode(const Args p, const Plan pl) {
+// Two CTAs per SM where the ring fits twice (W4A4 with one 16-token tile,
+// at 96 registers a thread; the other variants would spill and keep one):
+// the kernel is latency-bound, so more resident warps hide more of it.
+__global__ void __launch_bounds__(kThreads, (!A8 && MT == 1) ? 2 : 1) k_decode(const Args p, const Plan pl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   uint8_t* act = smem;                                          // [M][act_pitch]
@@ -368,8 +371,14 @@ inline cudaError_t launch_mt(const Args& p, const Plan& pl, int sms, cudaStream_
   const int bytes = smem_bytes(pl, MT);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
+  // persistent: as many CTAs as are resident at once (one or two per SM)
+  int per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, bytes) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  if (per_sm > 2) per_sm = 2;
+  const int ctas = pl.items < sms * per_sm ? pl.items : sms * per_sm;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(pl.items < sms ? pl.items : sms));
+  cfg.gridDim = dim3((unsigned)ctas);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = bytes;
   cfg.stream = st;
