@@ -54,9 +54,11 @@ typedef enum {
 typedef enum { SERQ_W4A4 = 0, SERQ_W4A8 = 1 } serq_mode;
 typedef enum { SERQ_F32 = 0, SERQ_BF16 = 1 } serq_dtype;
 
-/* Kernel choice for serq_linear_ex / serq_linear_accum.  AUTO picks DECODE
- * for M <= serq_decode_max_m() and PREFILL otherwise; DECODE accepts
- * M <= 64 when asked for explicitly. */
+/* Kernel choice for serq_linear_ex / serq_linear_accum / serq_linear_group.
+ * AUTO picks DECODE for M <= serq_decode_max_m() and PREFILL otherwise;
+ * DECODE accepts M <= 64 when asked for explicitly.  PREFILL picks CTA pairs
+ * with 256 x 256 tiles when the call's tiles (all layers of a group
+ * together) keep at least 90% of the SMs busy, else 128 x 128 tiles. */
 typedef enum {
   SERQ_ALGO_AUTO = 0,
   SERQ_ALGO_PREFILL = 1,       /* tcgen05 kind::i8 GEMM, TMEM accumulators; the
