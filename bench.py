@@ -242,7 +242,7 @@ class LayerWorkload:
         self.ops_step = sum(ops_of(M, K, N, r) for _, K, N in self.gemms)
         self.gemm_bytes_step = sum(linear_bytes(M, K, N, r, self.a_bits) for _, K, N in self.gemms)
         self.decode = M <= S.decode_max_m()
-        n_gemm_launches = len(self.grp) if (self.grouped and not self.decode) else len(self.gemms)
+        n_gemm_launches = len(self.grp) if self.grouped else len(self.gemms)
         self.launches_per_step = len(self.grp) + n_gemm_launches
         self.weight_mb = sum(p.W.size for p in wl.projections) / 2 / 1e6
 
@@ -521,7 +521,7 @@ def run_gpu(args, rank, world, local_rank):
                   f"({N_WEIGHT_COPIES} x {W.weight_mb:.0f} MB packed) and {N_ACT_COPIES} activation copies alternated",
             "cuda_graphs": graphs is not None,
             "algo": args.algo,
-            "grouped_launches": W.grouped and not W.decode,
+            "grouped_launches": W.grouped,
         },
         "gpu_launches": W.launches_per_step * args.steps,
         "clocks": clk.summary(),

@@ -42,10 +42,10 @@ constexpr int kNT = 2;                              // n8 MMA tiles per item
 constexpr int kRows = 8 * kNT;                      // output channels per item
 constexpr int kPad = 16;                            // bytes added to every staged activation row
 
-struct Args {
-  const uint8_t* Xq;
-  const float* sx;
-  int M, K, N, rpad;
+// Up to four layers that read the same activation codes run as one launch;
+// their items form one list (layer l's items start at item_base).
+constexpr int kMaxGroup = 4;
+struct LayerDec {
   const uint8_t* Wq;
   const uint8_t* Rq;
   const float* sw;
@@ -54,7 +54,26 @@ struct Args {
   int ldy;
   int32_t* acc0;
   int32_t* acc1;
+  int N, item_base;
 };
+
+struct Args {
+  const uint8_t* Xq;
+  const float* sx;
+  int M, K, N, rpad;  // N: all layers' channels together
+  int nlayers;
+  LayerDec lo[kMaxGroup];
+};
+
+// Layer of list item `item` and the item's index within that layer.
+__device__ __forceinline__ int layer_of(const Args& p, int item, int& li) {
+  int l = 0;
+#pragma unroll
+  for (int i = 1; i < kMaxGroup; ++i)
+    if (i < p.nlayers && item >= p.lo[i].item_base) l = i;
+  li = item - p.lo[l].item_base;
+  return l;
+}
 
 // Shared-memory plan, computed on the host.
 struct Plan {
@@ -206,13 +225,15 @@ __global__ void __launch_bounds__(kThreads, (!A8 && MT == 1) ? 2 : 1) k_decode(c
         const uint32_t ph = (j / pl.stages) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kDevTimeoutProducer)) return false;
         uint8_t* st = ring + s * pl.stage_bytes;
-        const size_t n0 = (size_t)item * kRows;
+        int li;
+        const LayerDec& lo = p.lo[layer_of(p, item, li)];
+        const size_t n0 = (size_t)li * kRows;
         mbar_arrive_expect_tx(&full[s], kRows * (wbytes + rbytes + 8));
-        bulk_load(st, p.Wq + n0 * wbytes, kRows * wbytes, &full[s]);
-        if (rbytes) bulk_load(st + kRows * pl.wrow, p.Rq + n0 * rbytes, kRows * rbytes, &full[s]);
+        bulk_load(st, lo.Wq + n0 * wbytes, kRows * wbytes, &full[s]);
+        if (rbytes) bulk_load(st + kRows * pl.wrow, lo.Rq + n0 * rbytes, kRows * rbytes, &full[s]);
         uint8_t* sc = st + kRows * (pl.wrow + pl.rrow);  // sw, sR of the item's channels (16 each)
-        bulk_load(sc, p.sw + n0, kRows * 4, &full[s]);
-        bulk_load(sc + kRows * 4, p.sr + n0, kRows * 4, &full[s]);
+        bulk_load(sc, lo.sw + n0, kRows * 4, &full[s]);
+        bulk_load(sc + kRows * 4, lo.sr + n0, kRows * 4, &full[s]);
         return true;
       };
       int item = blockIdx.x, j = 0;
@@ -300,9 +321,11 @@ __global__ void __launch_bounds__(kThreads, (!A8 && MT == 1) ? 2 : 1) k_decode(c
       if (last) {
         __threadfence_block();
         const float* sc = reinterpret_cast<const float*>(wst + kRows * (pl.wrow + pl.rrow));
+        int li;
+        const LayerDec& lo = p.lo[layer_of(p, item, li)];
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) {
-          const int col = item * kRows + 8 * nt + 2 * t;  // this lane's two output channels
+          const int col = li * kRows + 8 * nt + 2 * t;  // this lane's two output channels of its layer
           const float2 sw2 = *reinterpret_cast<const float2*>(sc + 8 * nt + 2 * t);
           const float2 sr2 = *reinterpret_cast<const float2*>(sc + kRows + 8 * nt + 2 * t);
 #pragma unroll
@@ -317,13 +340,13 @@ __global__ void __launch_bounds__(kThreads, (!A8 && MT == 1) ? 2 : 1) k_decode(c
               e0[0] = 0; e0[32] = 0; e1[0] = 0; e1[32] = 0;
               if (row >= p.M) continue;
               if (ACC_OUT) {
-                *reinterpret_cast<int2*>(p.acc0 + (size_t)row * p.N + col) = make_int2(a00, a01);
-                *reinterpret_cast<int2*>(p.acc1 + (size_t)row * p.N + col) = make_int2(a10, a11);
+                *reinterpret_cast<int2*>(lo.acc0 + (size_t)row * lo.N + col) = make_int2(a00, a01);
+                *reinterpret_cast<int2*>(lo.acc1 + (size_t)row * lo.N + col) = make_int2(a10, a11);
               } else {
                 const float sxm = sxr[mt][hh];
                 const float y0 = sxm * fmaf(sw2.x, (float)a00, sr2.x * (float)a10);
                 const float y1 = sxm * fmaf(sw2.y, (float)a01, sr2.y * (float)a11);
-                *reinterpret_cast<__nv_bfloat162*>(p.Y + (size_t)row * p.ldy + col) = __floats2bfloat162_rn(y0, y1);
+                *reinterpret_cast<__nv_bfloat162*>(lo.Y + (size_t)row * lo.ldy + col) = __floats2bfloat162_rn(y0, y1);
               }
             }
         }

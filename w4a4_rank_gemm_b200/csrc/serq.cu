@@ -407,6 +407,32 @@ cudaError_t dispatch_tc(const LinearGroup& G, const void* Xq, const float* sx, i
   return launch_tc<128, A8, ACC, 1>(G, Xq, sx, M, st);
 }
 
+// The mma.sync decode kernel over a group of layers (one launch; one layer
+// is a group of one).
+cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const float* sx, int M, bool a8, bool accum,
+                                cudaStream_t st) {
+  serq::decode::Args a = {};
+  a.Xq = static_cast<const uint8_t*>(Xq);
+  a.sx = sx;
+  a.M = M;
+  a.K = G.L[0]->K;
+  a.rpad = G.L[0]->rpad;
+  a.nlayers = G.n;
+  int items = 0;
+  for (int l = 0; l < serq::decode::kMaxGroup; ++l) {
+    const int li = (l < G.n) ? l : 0;
+    const serq_layer* L = G.L[li];
+    a.lo[l] = serq::decode::LayerDec{L->wq, L->rq, L->sw, L->sr, G.Y[li], G.ldy[li], G.acc0[li], G.acc1[li], L->N, items};
+    if (l < G.n) items += L->N / serq::decode::kRows;
+  }
+  a.N = items * serq::decode::kRows;
+  if (a8)
+    return accum ? serq::decode::launch<true, true>(a, sm_count(), max_smem(), st)
+                 : serq::decode::launch<true, false>(a, sm_count(), max_smem(), st);
+  return accum ? serq::decode::launch<false, true>(a, sm_count(), max_smem(), st)
+               : serq::decode::launch<false, false>(a, sm_count(), max_smem(), st);
+}
+
 // Argument checks shared by the single-layer and grouped calls; resolves AUTO.
 serq_status check_linear(const serq_layer* L, const void* Xq, const float* sx, int M, const void* Y, int ldy,
                          const int32_t* acc0, const int32_t* acc1, serq_algo* algo_io) {
@@ -458,14 +484,14 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
     else
       e = accum ? dispatch_decode_tc<false, true>(L, Xq, a, st) : dispatch_decode_tc<false, false>(L, Xq, a, st);
   } else if (algo == SERQ_ALGO_DECODE) {
-    serq::decode::Args a{static_cast<const uint8_t*>(Xq), sx, M, L->K, L->N, L->rpad, L->wq, L->rq, L->sw,
-                         L->sr, static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1};
-    if (a8)
-      e = accum ? serq::decode::launch<true, true>(a, sm_count(), max_smem(), st)
-                : serq::decode::launch<true, false>(a, sm_count(), max_smem(), st);
-    else
-      e = accum ? serq::decode::launch<false, true>(a, sm_count(), max_smem(), st)
-                : serq::decode::launch<false, false>(a, sm_count(), max_smem(), st);
+    LinearGroup G = {};
+    G.n = 1;
+    G.L[0] = L;
+    G.Y[0] = static_cast<__nv_bfloat16*>(Y);
+    G.ldy[0] = ldy;
+    G.acc0[0] = acc0;
+    G.acc1[0] = acc1;
+    e = launch_decode_group(G, Xq, sx, M, a8, accum, st);
   } else {
     LinearGroup G = {};
     G.n = 1;
@@ -507,7 +533,7 @@ serq_status group_impl(int n, const serq_layer* const* Ls, const void* Xq, const
       return s;
     resolved = a;
   }
-  if (resolved == SERQ_ALGO_DECODE || resolved == SERQ_ALGO_DECODE_TC || resolved == SERQ_ALGO_PREFILL_PAIR_TMEM_A) {
+  if (resolved == SERQ_ALGO_DECODE_TC || resolved == SERQ_ALGO_PREFILL_PAIR_TMEM_A) {
     for (int l = 0; l < n; ++l)
       if ((s = linear_impl(Ls[l], Xq, sx, M, accum ? nullptr : Y[l], accum ? 0 : ldy[l], accum ? acc0[l] : nullptr,
                            accum ? acc1[l] : nullptr, resolved, stream)))
@@ -525,6 +551,11 @@ serq_status group_impl(int n, const serq_layer* const* Ls, const void* Xq, const
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
+  if (resolved == SERQ_ALGO_DECODE) {
+    e = launch_decode_group(G, Xq, sx, M, Ls[0]->mode == SERQ_W4A8, accum, st);
+    if (e != cudaSuccess) return cuda_fail(e, "serq_linear_group launch");
+    return ok();
+  }
   if (Ls[0]->mode == SERQ_W4A8)
     e = accum ? dispatch_tc<true, true>(G, Xq, sx, M, resolved, st)
               : dispatch_tc<true, false>(G, Xq, sx, M, resolved, st);
