@@ -194,8 +194,9 @@ serq_status serq_linear_accum(const serq_layer* layer, const void* Xq, int M, in
  * block's q/k/v projections or its gate/up pair (key design 2, applied to
  * each layer; the pages run them as separate GEMMs).  With a prefill kernel
  * the n products run as one launch over the union of their output tiles, so
- * setup and the last partial wave are paid once; decode kernels and
- * SERQ_ALGO_PREFILL_PAIR_TMEM_A run one launch per layer.  Results are
+ * setup and the last partial wave are paid once; SERQ_ALGO_DECODE runs the
+ * union of the layers' 16-channel items as one launch; SERQ_ALGO_DECODE_TC
+ * and SERQ_ALGO_PREFILL_PAIR_TMEM_A run one launch per layer.  Results are
  * identical to n serq_linear_ex calls with the same kernel.
  *  n        1..4.
  *  layers   HOST array of n layers with equal K and mode and ranks that
