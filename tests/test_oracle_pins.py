@@ -320,3 +320,124 @@ def test_mlp_quantized_chain_tracks_full_precision():
         y = O.mlp_forward(blk.X, prep)["y"]
         rel.append(np.linalg.norm(y - ref) / np.linalg.norm(ref))
     assert rel[1] < rel[0] < 0.4, rel
+
+
+# --------------------------------------------------------------------------
+# bf16 storage rounding and the smoothing floor against hand-worked bits
+# --------------------------------------------------------------------------
+GOLD2 = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "bf16_and_floor_cases.json")))
+
+
+def _u32(h):
+    return np.array([int(h, 16)], dtype=np.uint32)
+
+
+@pytest.mark.parametrize("case", GOLD2["bf16"]["cases"], ids=lambda c: c["in"])
+def test_to_bf16_golden(case):
+    x = _u32(case["in"]).view(F32)
+    with np.errstate(over="ignore"):
+        got = O.to_bf16(x).view(np.uint32)
+    assert int(got[0]) == int(case["out"], 16), case["why"]
+
+
+def test_to_bf16_keeps_representable_values_and_halves_the_error():
+    """Every bf16 value is a fixed point, and the rounding error of any other
+    finite value is at most half a bf16 ulp (ties to even), checked on all
+    2^16 upper halves with random lower halves."""
+    rng = np.random.default_rng(2)
+    hi = np.arange(1 << 16, dtype=np.uint32)
+    exact = (hi << 16).view(F32)
+    finite = np.isfinite(exact)
+    assert np.array_equal(O.to_bf16(exact[finite]).view(np.uint32), (hi << 16)[finite])
+    lo = rng.integers(0, 1 << 16, size=hi.size, dtype=np.uint32)
+    x = ((hi << 16) | lo).view(F32)
+    ok = np.isfinite(x) & (np.abs(x) < F32(3.0e38))
+    x = x[ok]
+    y = O.to_bf16(x).astype(np.float64)
+    xe = x.astype(np.float64)
+    # ulp of the bf16 grid at |x|: 2^(exponent - 7), subnormals 2^-133
+    e = np.floor(np.log2(np.maximum(np.abs(xe), 2.0 ** -126)))
+    ulp = 2.0 ** (e - 7)
+    assert np.all(np.abs(y - xe) <= ulp / 2)
+
+
+def test_smooth_scales_floor_golden():
+    g = GOLD2["smooth_floor"]
+    s = O.smooth_scales(np.array(g["X_calib"], F32), np.array(g["W"], F32))
+    got = [f"0x{int(b):08X}" for b in s.view(np.uint32)]
+    assert got == g["s_bits"], list(zip(got, g["why"]))
+    assert O.saliency_perm(s).tolist() == g["perm"]
+
+
+# --------------------------------------------------------------------------
+# The MLP fold (key design 3): prepare_mlp / mlp_forward against a chain
+# built without any fold.  Moving down_proj's order P4 into the gate/up
+# output columns is a pure column permutation, so every per-column step
+# (row maxima, per-channel quantization, the compensator, the epilogue,
+# silu * mul) must give the permuted values of the unfolded chain bit for
+# bit, provided the unfolded up_proj has its columns divided by s4 (the
+# smoothing divisor of down_proj, which passes through up only).
+# --------------------------------------------------------------------------
+def _mlp_blk():
+    return synth.mlp_block(M=24, K=96, F=160, rank=32, seed=21, n_calib=48)
+
+
+def _fold_mismatches(prep, blk, r):
+    """Names of the checks on which `prep` differs from the unfolded chain."""
+    bad = []
+    s4, pi4, (down,) = O.prepare_group([blk.Wd], blk.H_calib, r)
+    if not (np.array_equal(prep["pi4"], pi4) and np.array_equal(prep["s4"].view(np.uint32), s4.view(np.uint32))):
+        bad.append("down order / scales")
+    Wu_div = (blk.Wu / s4[None, :]).astype(F32)
+    s_ref, pi_ref, (g_ref, u_ref) = O.prepare_group([blk.Wg, Wu_div], blk.X_calib, r)
+    if not (np.array_equal(prep["s_gu"].view(np.uint32), s_ref.view(np.uint32))
+            and np.array_equal(prep["pi_gu"], pi_ref)):
+        bad.append("gate/up smoothing")
+    for name, ref in (("gate", g_ref), ("up", u_ref)):
+        L = prep[name]
+        same = (np.array_equal(L.q_w, ref.q_w[:, pi4]) and np.array_equal(L.s_w, ref.s_w[pi4])
+                and np.array_equal(L.q_r, ref.q_r[:, pi4]) and np.array_equal(L.s_r, ref.s_r[pi4]))
+        if not same:
+            bad.append(name + " codes")
+    out = O.mlp_forward(blk.X, prep)
+    xh = O.flatten_permute(blk.X, s_ref, pi_ref, out_bf16=True)
+    g = O.to_bf16(O.linear(xh, g_ref)[0].astype(F32))[:, pi4]
+    u = O.to_bf16(O.linear(xh, u_ref)[0].astype(F32))[:, pi4]
+    if not (np.array_equal(out["g"], g) and np.array_equal(out["u"], u)):
+        bad.append("gate/up outputs")
+    h = O.silu_mul_f32(g, u)
+    if not np.array_equal(out["h"].view(np.uint32), h.view(np.uint32)):
+        bad.append("intermediate")
+    y = O.linear(h, down)[0]
+    if not np.array_equal(out["y"], y):
+        bad.append("block output")
+    return bad
+
+
+def test_prepare_mlp_is_the_permuted_unfolded_chain():
+    blk = _mlp_blk()
+    prep = O.prepare_mlp(blk.Wg, blk.Wu, blk.Wd, blk.X_calib, blk.H_calib, 32)
+    assert _fold_mismatches(prep, blk, 32) == []
+    # the folded intermediate is down_proj's flattened input: h / s4 in P4 order
+    # up to the rounding of the quantized layers (not a pin, a sanity bound)
+    assert not np.array_equal(prep["pi4"], np.arange(blk.Wd.shape[0]))
+
+
+@pytest.mark.parametrize("mistake", ["s4 also on gate", "P4 inverted", "s4 left out of up"])
+def test_prepare_mlp_check_catches_misfolds(mistake):
+    """The check above fails on plausible wrong folds (planted in a copy of
+    the oracle's preparation, on the CPU)."""
+    blk = _mlp_blk()
+    r = 32
+    s4, pi4, (down,) = O.prepare_group([blk.Wd], blk.H_calib, r)
+    inv = np.argsort(pi4).astype(np.int32)
+    assert not np.array_equal(inv, pi4)
+    if mistake == "s4 also on gate":
+        Wg_f, Wu_f = O.fold_output_columns(blk.Wg, pi4, s4), O.fold_output_columns(blk.Wu, pi4, s4)
+    elif mistake == "P4 inverted":
+        Wg_f, Wu_f = O.fold_output_columns(blk.Wg, inv, None), O.fold_output_columns(blk.Wu, inv, s4)
+    else:
+        Wg_f, Wu_f = O.fold_output_columns(blk.Wg, pi4, None), O.fold_output_columns(blk.Wu, pi4, None)
+    s_gu, pi_gu, (gate, up) = O.prepare_group([Wg_f, Wu_f], blk.X_calib, r)
+    bad = dict(s_gu=s_gu, pi_gu=pi_gu, gate=gate, up=up, s4=s4, pi4=pi4, down=down)
+    assert _fold_mismatches(bad, blk, r) != []
