@@ -51,31 +51,59 @@ def to_bf16(x: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Step 1 -- static activation flattening  ([notes] key design 1; [gist-de] 2A;
 # [radio]).  Y = X W = (X diag(s)^-1)(diag(s) W).  SmoothQuant's static
-# per-input-channel scale with migration strength 1/2:
-#     s_j = sqrt(max|X_:,j|) / sqrt(max|W_j,:|)
+# per-input-channel scale with migration strength alpha:
+#     s_j = max|X_:,j|^alpha / max|W_j,:|^(1 - alpha)
 # Reading: the pages name SmoothQuant's static scale without a formula; the
-# alpha = 1/2 form and a 1e-5 floor on both maxima are taken.  The row maxima
+# default alpha = 1/2 form (s_j = sqrt(max|X_j|) / sqrt(max|W_j|)) and a 1e-5
+# floor on both maxima are taken.  At alpha = 1/2 the two square roots and
+# the division are single fp32 operations; any other alpha is evaluated in
+# fp64 (two powers and a division) and rounded to fp32 once.  The row maxima
 # of W run over every weight that consumes the same activation (q/k/v share
 # one input, gate/up share one), so one s serves the whole group.
 # ---------------------------------------------------------------------------
-def smooth_scales(X_calib: np.ndarray, weights) -> np.ndarray:
+def weight_row_amax(weights) -> np.ndarray:
+    """max_n |W_jn| over every weight of a group (unfloored)."""
     if isinstance(weights, np.ndarray):
         weights = [weights]
+    return np.max(np.stack([np.max(np.abs(np.asarray(W, dtype=F32)), axis=1)
+                            for W in weights]), axis=0).astype(F32)
+
+
+def smooth_scales(X_calib: np.ndarray, weights, alpha: float = 0.5) -> np.ndarray:
     amax_x = np.max(np.abs(np.asarray(X_calib, dtype=F32)), axis=0)
-    amax_w = np.max(np.stack([np.max(np.abs(np.asarray(W, dtype=F32)), axis=1)
-                              for W in weights]), axis=0)
-    num = np.sqrt(np.maximum(amax_x, SMOOTH_FLOOR))
-    den = np.sqrt(np.maximum(amax_w, SMOOTH_FLOOR))
+    amax_w = weight_row_amax(weights)
+    ax = np.maximum(amax_x, SMOOTH_FLOOR)
+    aw = np.maximum(amax_w, SMOOTH_FLOOR)
+    a = float(F32(alpha))
+    if a == 0.5:
+        return (np.sqrt(ax) / np.sqrt(aw)).astype(F32)
+    num = np.power(ax.astype(np.float64), a)
+    den = np.power(aw.astype(np.float64), 1.0 - a)
     return (num / den).astype(F32)
 
 
 # ---------------------------------------------------------------------------
 # Step 2 -- saliency ranking ([notes] key design 2: after flattening, the
 # salient rows of the folded weight are identified directly by their scale;
-# [gist-de] 2B: by the activations' scale factors).  Reading: "scale" is s_j;
-# rows are ordered by descending s_j, ties kept in channel order (stable).
-# P maps position i -> original channel pi[i].
+# [gist-de] 2B: by the activations' scale factors).  Reading: "scale" is s_j
+# (metric 0, the default); metric 1 ranks by the folded row's absolute
+# maximum s_j * max_n |W_jn| (one fp32 multiply), the other plain reading of
+# "the salient rows of the folded weight".  Rows are ordered by descending
+# key, ties kept in channel order (stable).  P maps position i -> original
+# channel pi[i].
 # ---------------------------------------------------------------------------
+SALIENCY_SCALE, SALIENCY_ROW_ABSMAX = 0, 1
+
+
+def saliency_key(s: np.ndarray, weights, metric: int = SALIENCY_SCALE) -> np.ndarray:
+    s = np.asarray(s, dtype=F32)
+    if metric == SALIENCY_SCALE:
+        return s
+    if metric == SALIENCY_ROW_ABSMAX:
+        return (s * weight_row_amax(weights)).astype(F32)
+    raise ValueError(f"unknown saliency metric {metric}")
+
+
 def saliency_perm(s: np.ndarray) -> np.ndarray:
     return np.argsort(-np.asarray(s, dtype=np.float64), kind="stable").astype(np.int32)
 
@@ -211,14 +239,15 @@ def fold_output_columns(W: np.ndarray, out_perm=None, out_div=None) -> np.ndarra
     return out.astype(F32)
 
 
-def prepare_group(weights, X_calib, r: int, w_bits: int = 4):
+def prepare_group(weights, X_calib, r: int, w_bits: int = 4, alpha: float = 0.5,
+                  saliency: int = SALIENCY_SCALE):
     """SERQ offline stage for the weights that consume one activation.
 
     Returns (s, pi, [PreparedLayer per weight])."""
     if isinstance(weights, np.ndarray):
         weights = [weights]
-    s = smooth_scales(X_calib, weights)
-    pi = saliency_perm(s)
+    s = smooth_scales(X_calib, weights, alpha)
+    pi = saliency_perm(saliency_key(s, weights, saliency))
     layers = []
     for W in weights:
         W_hat = fold_weight(W, s, pi)
@@ -234,8 +263,9 @@ def prepare_group(weights, X_calib, r: int, w_bits: int = 4):
     return s, pi, layers
 
 
-def prepare(W, X_calib, r: int, w_bits: int = 4) -> PreparedLayer:
-    return prepare_group([W], X_calib, r, w_bits)[2][0]
+def prepare(W, X_calib, r: int, w_bits: int = 4, alpha: float = 0.5,
+            saliency: int = SALIENCY_SCALE) -> PreparedLayer:
+    return prepare_group([W], X_calib, r, w_bits, alpha, saliency)[2][0]
 
 
 # ---------------------------------------------------------------------------

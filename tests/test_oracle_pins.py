@@ -441,3 +441,41 @@ def test_prepare_mlp_check_catches_misfolds(mistake):
     s_gu, pi_gu, (gate, up) = O.prepare_group([Wg_f, Wu_f], blk.X_calib, r)
     bad = dict(s_gu=s_gu, pi_gu=pi_gu, gate=gate, up=up, s4=s4, pi4=pi4, down=down)
     assert _fold_mismatches(bad, blk, r) != []
+
+
+# --------------------------------------------------------------------------
+# Preparation options: SmoothQuant's migration strength alpha and the
+# saliency metric (the reading by the folded row's absolute maximum)
+# --------------------------------------------------------------------------
+def test_smooth_scales_alpha_closed_forms():
+    Xc = np.array([[16.0, -2.0, 0.0], [3.0, 1.0, 0.0]], F32)   # column maxima 16, 2, 0 (-> 1e-5)
+    W = np.array([[0.25, 0.0], [-3.0, 1.0], [0.5, 0.0]], F32)    # row maxima 0.25, 3, 0.5
+    # alpha = 3/4 by hand: 16^(3/4) / 0.25^(1/4) = 8 / 2^(-1/2) = 8 sqrt(2) = 11.3137085 -> 0x413504f3
+    s = O.smooth_scales(Xc, W, alpha=0.75)
+    assert f"0x{int(s.view(np.uint32)[0]):08x}" == "0x413504f3"
+    # alpha = 1: s = the floored activation maximum itself; alpha = 0: s = 1 / weight maximum
+    s1 = O.smooth_scales(Xc, W, alpha=1.0)
+    assert s1.tolist() == [16.0, 2.0, float(F32(1e-5))]
+    s0 = O.smooth_scales(Xc, W, alpha=0.0)
+    assert s0.tolist() == [4.0, float(F32(1.0 / 3.0)), 2.0]
+    # the general path agrees with the square-root path next to alpha = 1/2
+    rng = np.random.default_rng(4)
+    Xr = np.abs(rng.standard_normal((16, 64))).astype(F32) * F32(30)
+    Wr = (0.02 * rng.standard_normal((64, 40))).astype(F32)
+    near = O.smooth_scales(Xr, Wr, alpha=float(np.nextafter(F32(0.5), F32(1))))
+    half = O.smooth_scales(Xr, Wr, alpha=0.5)
+    np.testing.assert_allclose(near, half, rtol=1e-5)
+
+
+def test_saliency_metric_row_absmax_golden():
+    # column maxima 4, 4, 4 and row maxima 4, 1, 0.25: s = 2/2, 2/1, 2/0.5 = 1, 2, 4 (exact);
+    # folded row maxima s * amax_w = 4, 2, 1
+    Xc = np.array([[4.0, -4.0, 1.0], [0.5, 2.0, -4.0]], F32)
+    W = np.array([[-4.0, 1.0], [0.5, 1.0], [0.25, -0.125]], F32)
+    s = O.smooth_scales(Xc, W)
+    assert s.tolist() == [1.0, 2.0, 4.0]
+    assert O.saliency_perm(O.saliency_key(s, W, O.SALIENCY_SCALE)).tolist() == [2, 1, 0]
+    assert O.saliency_perm(O.saliency_key(s, W, O.SALIENCY_ROW_ABSMAX)).tolist() == [0, 1, 2]
+    # the folded weight's row maxima are what metric 1 ranks
+    W_hat = O.fold_weight(W, s, np.arange(3))
+    np.testing.assert_array_equal(np.abs(W_hat).max(1), O.saliency_key(s, W, O.SALIENCY_ROW_ABSMAX))
