@@ -40,7 +40,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 4.5 / 2.25          # nominal dense ratio (recipe)
 N_WEIGHT_COPIES = 8                  # 8 x ~100 MB of packed weights > 126 MB L2
 N_ACT_COPIES = 2
-WORKLOADS = ("llama2_7b_prefill", "llama2_7b_decode", "llama3_8b_w4a8", "mlp_block")
+WORKLOADS = ("llama2_7b_prefill", "llama2_7b_decode", "llama3_8b_w4a8", "mlp_block", "l2qer_compare")
 
 
 def parse():
@@ -65,7 +65,7 @@ def parse():
     a = ap.parse_args()
     if a.M is None:
         a.M = {"llama2_7b_prefill": 2048, "llama2_7b_decode": 16, "llama3_8b_w4a8": 4096,
-               "mlp_block": 4096}[a.workload]
+               "mlp_block": 4096, "l2qer_compare": 2048}[a.workload]
     return a
 
 
@@ -530,10 +530,10 @@ def run_gpu(args, rank, world, local_rank):
         peak = pk.get("hbm_gbs")
         achieved = W.gemm_bytes_step * roof_steps / (gemm_ms / 1e3) / 1e9
         res["roofline"] = {
-            "kernel": "serq::decode::k_decode (split-K tensor-core GEMV, main + residual accumulators)",
+            "kernel": "serq::gs::k_gemv (streaming mma.sync GEMV, main + residual accumulators)",
             "bound": "hbm", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": recorded_traffic(f"{W.name}_M{W.M}", ["gemv_decode.cuh", "common.cuh"]),
+            "traffic": recorded_traffic(f"{W.name}_M{W.M}", ["gemv_stream.cuh", "common.cuh"]),
             "peak_source": f"{pk_src}: hbm_gbs" + (" -- of measured" if pk_src != "fallback" else " -- of fallback"),
             "gemm_share_of_step": round(gemm_ms / roof_steps / max(elapsed_ms / args.steps, 1e-9), 4),
             "timing": gemm_note,
@@ -610,6 +610,117 @@ def run_e2e(args, ctx, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 3),
             "pipelining": "copies of neighbouring steps overlap compute (3 streams, 2 buffer sets)"}
+
+
+# --------------------------------------------------------------------------
+# SERQ's residual path against the two-factor comparator (L2QER)
+# --------------------------------------------------------------------------
+def run_compare(args):
+    """Per Llama-2-7B projection, three variants on the same activation codes:
+    the main 4-bit product alone (rank 0), SERQ (main + the single r x N
+    residual on the salient columns, one launch) and the comparator (the
+    same main product, plus X_q L1 -> on-the-fly quantization -> L2, three
+    launches).  The residual path's cost is each variant's time minus the
+    main product's.  Decode sizes replay each variant as a CUDA graph."""
+    import torch
+    from w4a4_rank_gemm_b200 import build as _build
+    _build.build()
+    from w4a4_rank_gemm_b200 import serq as S
+    from w4a4_rank_gemm_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    M, copies = args.M, 4
+    wl = synth.llama2_7b(M=M)
+    r = wl.rank
+    projs = []
+    for iname, ps in groups_of(wl):
+        inp = wl.inputs[iname]
+        Xc = torch.from_numpy(inp.X_calib).to(dev)
+        for p in ps:
+            W = torch.from_numpy(p.W).to(dev)
+            K, N = p.W.shape
+            L1, L2 = synth.factor_pair(K, N, r, seed=len(projs) + 31)
+            L1d, L2d = torch.from_numpy(L1).to(dev), torch.from_numpy(L2).to(dev)
+            var = []
+            for _ in range(copies):
+                L0 = S.prepare(W, Xc, 0)
+                Lr = S.prepare(W, Xc, r)
+                var.append((L0, Lr, S.L2QER(L0, L1d, L2d)))
+            Xh = S.flatten_permute(var[0][0], torch.from_numpy(inp.X).to(dev).to(torch.bfloat16))
+            Xq, sx = S.quantize_act(Xh, "w4a4")
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            projs.append(dict(name=p.name, K=K, N=N, var=var, Xq=Xq, sx=sx, Y=Y,
+                              bufs=var[0][2].buffers(M, dev)))
+            del W
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    decode = M <= S.decode_max_m()
+
+    def call(pr, v, c):
+        L0, Lr, Q = pr["var"][c]
+        # the current stream: the timing stream, or the capture stream of a graph
+        if v == 0:
+            S.linear(L0, pr["Xq"], pr["sx"], Y=pr["Y"])
+        elif v == 1:
+            S.linear(Lr, pr["Xq"], pr["sx"], Y=pr["Y"])
+        else:
+            Q.linear(pr["Xq"], pr["sx"], Y=pr["Y"], bufs=pr["bufs"])
+
+    reps = max(10, min(args.steps, 200))
+    times = {}
+    for pr in projs:
+        for v in range(3):
+            for c in range(copies):
+                call(pr, v, c)
+            torch.cuda.synchronize()
+            if decode:
+                gs = []
+                for c in range(copies):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        call(pr, v, c)
+                    gs.append(g)
+                run = lambda i, gs=gs: gs[i % copies].replay()
+            else:
+                run = lambda i, pr=pr, v=v: call(pr, v, i % copies)
+            for i in range(3):
+                run(i)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for i in range(reps):
+                run(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times[(pr["name"], v)] = e0.elapsed_time(e1) * 1e3 / reps   # us per call
+            if decode:
+                del gs
+    if S.device_error() != 0:
+        raise RuntimeError("a kernel reported a timed-out wait")
+    per = {}
+    sum_serq = sum_two = sum_main = 0.0
+    for pr in projs:
+        t0, t1, t2 = (times[(pr["name"], v)] for v in range(3))
+        per[pr["name"]] = {"main_us": round(t0, 2), "serq_us": round(t1, 2), "two_factor_us": round(t2, 2),
+                           "serq_residual_us": round(t1 - t0, 2), "two_factor_residual_us": round(t2 - t0, 2)}
+        sum_main += t0
+        sum_serq += t1 - t0
+        sum_two += t2 - t0
+    ratio = sum_two / max(sum_serq, 1e-3)
+    return {
+        "metric": "residual-path latency: two-factor comparator (L2QER) / SERQ, one Llama-2-7B layer",
+        "value": round(ratio, 3), "unit": "x", "higher_is_better": True, "n_gpus": 1,
+        "steps": reps, "warmup": 3, "ms_per_step": round((sum_main + sum_serq) / 1e3, 4),
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 (W4A4 codes, int32 accumulate)",
+        "data": "synthetic (seeded; Llama shapes, random-init weights and factors, outlier-channel activations)",
+        "config": {"workload": f"l2qer_compare: 7 projections of one Llama-2-7B layer, M = {M}, r = {r}, "
+                               f"{copies} weight copies cycled; {'CUDA graphs' if decode else 'stream launches'}",
+                   "tokens_per_gpu": M, "rank": r},
+        "residual_us": {"serq": round(sum_serq, 2), "two_factor": round(sum_two, 2), "main_only": round(sum_main, 2)},
+        "per_projection": per,
+        "gpu_launches": 7 * reps * 5,
+    }
 
 
 # --------------------------------------------------------------------------
@@ -731,6 +842,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
+    if args.workload == "l2qer_compare":
+        if world == 1:
+            print(json.dumps(run_compare(args)), flush=True)
+        return
     try:
         res, ctx = run_gpu(args, rank, world, local_rank)
         if not args.profile and not args.no_e2e:

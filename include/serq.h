@@ -63,16 +63,21 @@ typedef enum {
   SERQ_ALGO_AUTO = 0,
   SERQ_ALGO_PREFILL = 1,       /* tcgen05 kind::i8 GEMM, TMEM accumulators; the
                                   output tile width is chosen from the shape  */
-  SERQ_ALGO_DECODE = 2,        /* memory-bound split-K tensor-core GEMV, M <= 64 */
+  SERQ_ALGO_DECODE = 2,        /* memory-bound GEMV (mma.sync), M <= 64: the
+                                  streaming kernel (every SM streams an equal
+                                  share of the channels) where it fits, else
+                                  the item-ring kernel                         */
   SERQ_ALGO_PREFILL_N128 = 3,  /* PREFILL with 128 x 128 output tiles, one CTA  */
   SERQ_ALGO_PREFILL_N256 = 4,  /* PREFILL with 128 x 256 output tiles, one CTA  */
   SERQ_ALGO_PREFILL_PAIR_N256 = 5, /* PREFILL with 256 x 256 tiles on a CTA pair
                                       (tcgen05 cta_group::2)                    */
   SERQ_ALGO_PREFILL_PAIR_TMEM_A = 6, /* W4A4 only: 256 x 192 tiles on a CTA pair with
                                         the widened activations in tensor memory  */
-  SERQ_ALGO_DECODE_TC = 7      /* M <= 32: tcgen05 GEMV with the weight rows as the
+  SERQ_ALGO_DECODE_TC = 7,     /* M <= 32: tcgen05 GEMV with the weight rows as the
                                   MMA's M, split-K partial sums in the layer's
                                   workspace (one stream per layer at a time)  */
+  SERQ_ALGO_DECODE_ITEMS = 8   /* M <= 64: the memory-bound GEMV over 16-channel
+                                  items with a shared bulk-copy ring          */
 } serq_algo;
 
 typedef struct serq_layer serq_layer;
@@ -81,48 +86,102 @@ typedef struct serq_layer serq_layer;
 /* Offline preparation (untimed)                                            */
 /* ------------------------------------------------------------------------ */
 
+/* Saliency metric of step 2 below (SERQ notes, key design 2: the salient
+ * rows of the folded weight are identified by their scale). */
+typedef enum {
+  SERQ_SALIENCY_SCALE = 0,      /* by s_j (default; the pages' "scale")      */
+  SERQ_SALIENCY_ROW_ABSMAX = 1  /* by the folded row's max |s_j W_jn|        */
+} serq_saliency;
+
+/* Options of the offline stage.  Fill with serq_prepare_opts_init, then
+ * change what differs. */
+typedef struct {
+  float alpha;                /* SmoothQuant migration strength in [0, 1];
+                                 default 0.5 (the square-root form)          */
+  int rank;                   /* r, 0 <= r <= K; default 128                 */
+  serq_mode mode;             /* activation format; weights are INT4 in both;
+                                 default SERQ_W4A4                           */
+  int saliency;               /* serq_saliency; default SERQ_SALIENCY_SCALE  */
+  const int32_t* out_perm;    /* serq_prepare only: nullable HOST int32[N],
+                                 the NEXT layer's saliency order (step 5)    */
+  const float* out_colscale;  /* serq_prepare only: nullable HOST float[N],
+                                 the NEXT layer's smoothing scales, divided
+                                 into the columns (step 5); needs out_perm   */
+} serq_prepare_opts;
+
+/* Defaults: alpha 0.5, rank 128, SERQ_W4A4, SERQ_SALIENCY_SCALE, no fold. */
+void serq_prepare_opts_init(serq_prepare_opts* opts);
+
 /*
- * serq_prepare_group -- SERQ's offline stage for n_weights weights that read
- * the same activation (q/k/v share one input, gate/up share one).
+ * serq_prepare -- SERQ's offline stage for one weight, from HOST arrays.
+ * Allocates the layer, uploads W and X_calib (and the fold arrays) to the
+ * current device, runs the steps below there and returns when they have
+ * finished; the handle owns its device memory (release with
+ * serq_layer_destroy).
  *
  * Steps (SERQ notes, "overall framework" and key designs 1-3):
- *  1. static activation flattening: s_j = sqrt(max_t|Xc_tj|) / sqrt(max|W_j,:|)
- *     with both maxima floored at 1e-5 and the weight maximum taken over all
- *     n_weights weights (key design 1; SmoothQuant form with strength 1/2);
- *  2. saliency order P: channels by descending s_j, ties by channel index
- *     (key design 2: salient rows are identified by their scale);
+ *  1. static activation flattening (key design 1, SmoothQuant's static
+ *     scale): s_j = max_t|Xc_tj|^alpha / max_n|W_jn|^(1 - alpha), both maxima
+ *     floored at 1e-5; at alpha = 0.5 this is sqrt / sqrt / divide in fp32,
+ *     any other alpha is evaluated in fp64 and rounded to fp32 once;
+ *  2. saliency order P: channels by descending key (opts->saliency), ties by
+ *     channel index (key design 2);
  *  3. W^ = P diag(s) W, quantized per output channel to INT4:
  *     code = clamp(rint(W^ * (7/amax)), -7, 7), sw = amax/7;
  *  4. R = W^[0:r] - code[0:r]*sw (the main path's own error on the r salient
  *     rows, key design 2 / core idea), quantized the same way -> Rq, sR;
- *  5. optionally, before all of the above, the NEXT layer's permutation and
- *     smoothing divisor are folded into this weight's output columns:
- *     W'[:, i] = W[:, out_perm[i]] / out_div[out_perm[i]] (key design 3:
+ *  5. optionally, before all of the above, the NEXT layer's order and
+ *     smoothing scales are folded into this weight's output columns:
+ *     W'[:, i] = W[:, out_perm[i]] / out_colscale[out_perm[i]] (key design 3:
  *     down_proj's order propagates into the gate/up columns).
- * All arithmetic is IEEE fp32 with one rounding per operation.
+ * Every step but the general-alpha power is IEEE fp32 with one rounding per
+ * operation.
  *
- *  W        host array of n_weights DEVICE pointers, each K x N_i fp32,
- *           row-major (d_in x d_out; Y = X W).
- *  N        host array of n_weights output widths (multiples of 32).
- *  X_calib  DEVICE, n_calib x K fp32 calibration activations (n_calib >= 1).
- *  rank     r, 0 <= r <= K.
- *  mode     SERQ_W4A4 or SERQ_W4A8 (weights are INT4 in both).
- *  out_perm host array of n_weights nullable DEVICE int32[N_i] pointers (or
- *           NULL for none).  out_div likewise with DEVICE float[N_i]; an
- *           out_div entry requires the matching out_perm entry.
- *  layers   host array receiving n_weights new handles.  On failure every
- *           entry is set to NULL and nothing is leaked.
- * Synchronous (returns after the device work has finished).
+ *  W        HOST, K x N fp32, row-major (d_in x d_out; Y = X W); N a multiple
+ *           of 32.
+ *  X_calib  HOST, n_calib x K fp32 calibration activations (n_calib >= 1).
+ *  opts     options (NULL = the defaults above).
+ *  layer    receives the new handle (NULL on failure; nothing leaks).
+ * Errors: SERQ_ERR_INVALID_ARG (null pointers, alpha outside [0, 1], bad mode
+ * or metric, out_colscale without out_perm), SERQ_ERR_UNSUPPORTED_SHAPE
+ * (K or N not a multiple of 32, rank outside [0, K]), SERQ_ERR_ALLOC,
+ * SERQ_ERR_CUDA, SERQ_ERR_UNSUPPORTED_DEVICE.  Synchronous.
+ */
+serq_status serq_prepare(const float* W, int K, int N, const float* X_calib, int n_calib,
+                         const serq_prepare_opts* opts, serq_layer** layer);
+
+/*
+ * serq_prepare_shared -- serq_prepare for n_weights weights that read the
+ * same activation (q/k/v share one input, gate/up share one): one smoothing
+ * vector s, whose weight maximum runs over all n_weights weights, and one
+ * order P, so one set of activation codes feeds every returned layer.
+ *  W        HOST array of n_weights HOST K x N_i fp32 arrays.
+ *  N        HOST array of n_weights output widths (multiples of 32).
+ *  X_calib  HOST, n_calib x K fp32.
+ *  opts     options; opts->out_perm and opts->out_colscale must be NULL (the
+ *           folds are per weight here).
+ *  out_perm, out_colscale  NULL, or HOST arrays of n_weights nullable HOST
+ *           arrays of N_i entries (step 5 per weight).
+ *  layers   HOST array receiving n_weights new handles (all NULL on failure).
+ * Errors as serq_prepare.  Synchronous.
+ */
+serq_status serq_prepare_shared(int n_weights, const float* const* W, const int* N, int K,
+                                const float* X_calib, int n_calib, const serq_prepare_opts* opts,
+                                const int32_t* const* out_perm, const float* const* out_colscale,
+                                serq_layer** layers);
+
+/*
+ * serq_prepare_group -- serq_prepare_shared with every array on the DEVICE:
+ * W[i] (K x N_i fp32), X_calib (n_calib x K fp32), out_perm[i] (int32[N_i])
+ * and out_colscale[i] (float[N_i]) are DEVICE pointers (the pointer arrays
+ * and N themselves are host arrays).  For callers whose weights are already
+ * resident, such as a model loaded onto the GPU; nothing is uploaded.
+ * Errors as serq_prepare.  Synchronous.
  */
 serq_status serq_prepare_group(int n_weights, const float* const* W, const int* N, int K,
-                               const float* X_calib, int n_calib, int rank, serq_mode mode,
-                               const int32_t* const* out_perm, const float* const* out_div,
+                               const float* X_calib, int n_calib, const serq_prepare_opts* opts,
+                               const int32_t* const* out_perm, const float* const* out_colscale,
                                serq_layer** layers);
-
-/* One weight: serq_prepare_group with n_weights = 1. */
-serq_status serq_prepare(const float* W, int K, int N, const float* X_calib, int n_calib,
-                         int rank, serq_mode mode, const int32_t* out_perm,
-                         const float* out_div, serq_layer** layer);
 
 /* Frees the handle's device memory.  NULL is accepted.  Synchronous. */
 void serq_layer_destroy(serq_layer* layer);
@@ -130,9 +189,16 @@ void serq_layer_destroy(serq_layer* layer);
 /* Shape and configuration of a prepared layer (any pointer may be NULL). */
 serq_status serq_layer_info(const serq_layer* layer, int* K, int* N, int* rank, int* mode);
 
+/* Synchronous copies of the layer's saliency order P (int32[K]: position i
+ * holds original channel P[i]) and smoothing scales s (float[K]) into HOST
+ * buffers: what the previous layer's serq_prepare needs for its fold
+ * (opts->out_perm / out_colscale) or a caller needs to produce X^. */
+serq_status serq_layer_get_perm(const serq_layer* layer, int32_t* perm);
+serq_status serq_layer_get_smooth(const serq_layer* layer, float* smooth);
+
 /* DEVICE pointers to the layer's permutation (int32[K]) and smoothing scales
  * (float[K]); owned by the layer, valid until serq_layer_destroy.  Used by
- * the previous layer's prepare (out_perm / out_div) or by
+ * the previous layer's serq_prepare_group (out_perm / out_colscale) or by
  * serq_flatten_permute. */
 serq_status serq_layer_perm_smooth(const serq_layer* layer, const int32_t** perm,
                                    const float** smooth);
@@ -222,21 +288,94 @@ serq_status serq_linear_group(int n, const serq_layer* const* layers, const void
  * serq_linear_decode_static -- serq_linear (or, with acc0/acc1, the
  * accumulator hook) through the tensor-core decode kernel
  * (SERQ_ALGO_DECODE_TC) with its split-K partial sums and tile counters in a
- * scratch area compiled into the library, one per device, instead of the
- * layer's workspace: the call allocates nothing.  The pages have no
- * counterpart; this is a deployment variant of the same arithmetic.
- *  Xq, sx, Y, ldy  as serq_linear; M <= 32.
+ * scratch area compiled into the library (a file-scope __device__ array of
+ * 4 MB, one per device that loads the library, held until the process
+ * exits) instead of the layer's workspace, so the call allocates nothing.
+ * It is for callers that cannot call cudaMalloc on the decode path: a
+ * serving loop whose device memory is reserved up front by another pool, a
+ * caller running inside an allocator's own callbacks, or one that must not
+ * take the allocator's lock or its implicit synchronisation between tokens.
+ * The pages have no counterpart; this is a deployment variant of the same
+ * arithmetic.
+ *  Xq, sx, Y, ldy  as serq_linear; 1 <= M <= 32.
  *  acc0, acc1      both null (bf16 output in Y), or both DEVICE int32 M x N
  *                  (exact accumulators; sx and Y are then not used).
- *  N <= 16384, else SERQ_ERR_UNSUPPORTED_SHAPE.
- * The scratch must start at zero: the first call on a device clears it (a
- * synchronous cudaMemset) and every completed call leaves it zero.
- * Races: all calls on a device share the one scratch area, so they must not
- * overlap in time (one stream, or streams ordered by events), across all
- * layers.  A wait that times out (serq_device_error) leaves it undefined.
+ *  N <= 16384 and M <= 32, else SERQ_ERR_UNSUPPORTED_SHAPE.
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address and clears the array with cudaMemsetAsync on
+ * `stream`, ordered before the kernel; make that first call before any stream
+ * capture.  Every completed call leaves the scratch zero.  After
+ * serq_device_error has reported a timed-out wait, which can leave partial
+ * sums behind, the next call on that device clears it again the same way.
+ * Races: all calls on a device share the one scratch area and each call
+ * relies on the previous one having finished, so calls that overlap on the
+ * GPU race (use one stream, or order streams by events), across all layers.
  */
 serq_status serq_linear_decode_static(const serq_layer* layer, const void* Xq, const float* sx, int M,
                                       void* Y, int ldy, int32_t* acc0, int32_t* acc1, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Comparator: two-factor low-rank error reconstruction (L2QER)             */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The method SERQ is measured against (SERQ notes, "field status", "pain
+ * points" and "vs L2QER"; gist.science (ja) summary, "computation flow"):
+ * the weight's quantization error is approximated by two low-rank factors,
+ * L1 L2 ~ W^ - Q(W^), applied one after the other at inference with an
+ * on-the-fly quantization of the intermediate:
+ *     Y = X_q W_q + Q(X_q L1_q) L2_q.
+ * Built on a prepared SERQ layer so that the main product X_q W_q is the
+ * same; only the error path differs.  The factors are given (an offline
+ * step, like calibration data; the pages extract them by a scaled SVD) and
+ * quantized here per output channel to INT4 like W^ (the pages' L2QER keeps
+ * them in 8 bits; 4 bits is the cheaper choice, so the comparison isolates
+ * the serial structure).  W4A4 layers only.
+ */
+typedef struct serq_l2qer serq_l2qer;
+
+/*
+ * serq_l2qer_prepare -- quantizes and packs the factors.
+ *  layer  prepared W4A4 layer (not owned; must outlive the comparator).
+ *  L1     DEVICE, K x r fp32 row-major, rows in the layer's input order
+ *         (the flattened, permuted X^ multiplies it).
+ *  L2     DEVICE, r x N fp32 row-major.
+ *  r      a positive multiple of 32, <= K.
+ *  out    receives the handle (NULL on failure).  Synchronous.
+ */
+serq_status serq_l2qer_prepare(const serq_layer* layer, const float* L1, const float* L2, int r,
+                               serq_l2qer** out);
+
+/* Frees the comparator's device memory (not the layer).  NULL accepted. */
+void serq_l2qer_destroy(serq_l2qer* q);
+
+/* Synchronous copies to HOST buffers (any may be NULL): l1q r x K/2 bytes
+ * (L1's codes, output channel major), s_l1 float[r], l2q N x r/2 bytes,
+ * s_l2 float[N]. */
+serq_status serq_l2qer_get_packed(const serq_l2qer* q, uint8_t* l1q, float* s_l1, uint8_t* l2q, float* s_l2);
+
+/*
+ * serq_l2qer_linear -- the comparator's inference path, three launches on
+ * `stream`: Z = bf16(sx * (s_L1 * (X_q L1_q))) (the layer epilogue of a
+ * rank-0 linear), per-token quantization of Z (as serq_quantize_act,
+ * W4A4), then Y = sx * (sw * acc0) + sz * (s_L2 * acc2) with
+ * acc0 = X_q W_q and acc2 = Z_q L2_q exact in int32.
+ *  Xq, sx   DEVICE, from serq_quantize_act of the layer's X^.
+ *  Z        DEVICE bf16 M x r (written), Zq DEVICE M x r/2 bytes (written),
+ *           sz DEVICE float[M] (written): the intermediate, owned by the
+ *           caller (the call allocates nothing).
+ *  Y, ldy   DEVICE bf16 M x N output.
+ *  algo     SERQ_ALGO_AUTO, DECODE (M <= 32), PREFILL, PREFILL_N128 or
+ *           PREFILL_PAIR_N256.
+ * Asynchronous.
+ */
+serq_status serq_l2qer_linear(const serq_l2qer* q, const void* Xq, const float* sx, int M, void* Z, void* Zq,
+                              float* sz, void* Y, int ldy, serq_algo algo, void* stream);
+
+/* Test hook: the final GEMM's exact accumulators acc0 = X_q W_q and
+ * acc1 = Z_q L2_q (DEVICE int32 M x N) for given codes Xq and Zq. */
+serq_status serq_l2qer_accum(const serq_l2qer* q, const void* Xq, const void* Zq, int M, int32_t* acc0,
+                             int32_t* acc1, serq_algo algo, void* stream);
 
 /*
  * serq_silu_mul_quantize -- MLP intermediate of a Llama block whose gate/up
@@ -280,6 +419,18 @@ serq_status serq_check_device(void);
 /* Reads and clears the device-side status word that kernels set when a
  * bounded wait gives up (0 = none).  Synchronises the current device. */
 serq_status serq_device_error(int* code);
+
+/*
+ * Test hook for failure detection (no GPU fault involved): runs the
+ * streaming decode kernel (SERQ_ALGO_DECODE, M <= 32) with its activation
+ * copies withheld and the bounded wait for them shortened to wait_us
+ * microseconds (1 .. 10^6).  Every CTA gives up that wait, records the
+ * timeout in the device status word (serq_device_error then reports 2),
+ * lets its weight copies land and returns; Y is not written.  The next call
+ * on the device runs normally.
+ */
+serq_status serq_test_decode_timeout(const serq_layer* layer, const void* Xq, const float* sx, int M, void* Y,
+                                     int ldy, int wait_us, void* stream);
 
 /* Library version string. */
 const char* serq_version(void);

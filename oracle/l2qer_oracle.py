@@ -113,3 +113,14 @@ def linear(X_hat: np.ndarray, layer: L2QERLayer):
     Y = (np.asarray(sx, np.float64)[:, None] * layer.s_w.astype(np.float64)[None, :] * acc0
          + np.asarray(sz, np.float64)[:, None] * layer.s_l2.astype(np.float64)[None, :] * acc2)
     return Y, xq, sx, acc0, zq, sz, acc2
+
+
+def prepare_from_factors(serq_layer, L1: np.ndarray, L2: np.ndarray) -> L2QERLayer:
+    """The comparator on a prepared SERQ layer (its W^ codes and scales) with
+    given fp32 factors L1 (K x r, rows in the layer's input order) and L2
+    (r x N), each quantized per output channel with 4-bit codes."""
+    L1 = np.asarray(L1, F32)
+    L2 = np.asarray(L2, F32)
+    q_l1, s_l1 = O.quantize_weight(L1, 4)
+    q_l2, s_l2 = O.quantize_weight(L2, 4)
+    return L2QERLayer(serq_layer.q_w, serq_layer.s_w, L1, L2, q_l1, s_l1, q_l2, s_l2, None, L1.shape[1])

@@ -64,10 +64,51 @@ def test_host_side_argument_rejection(lib):
     W = (ctypes.c_void_p * 1)(0x1000)
     N = (ctypes.c_int * 1)(256)
     out = (ctypes.c_void_p * 1)()
-    assert L.serq_prepare_group(1, W, N, 256, fake, 8, 300, lib.W4A4, None, None, out) == lib.ERR_UNSUPPORTED_SHAPE
+    o = lib.prepare_opts(rank=300)
+    assert L.serq_prepare_group(1, W, N, 256, fake, 8, ctypes.byref(o), None, None, out) == lib.ERR_UNSUPPORTED_SHAPE
     N[0] = 100
-    assert L.serq_prepare_group(1, W, N, 256, fake, 8, 16, lib.W4A4, None, None, out) == lib.ERR_UNSUPPORTED_SHAPE
+    o = lib.prepare_opts(rank=16)
+    assert L.serq_prepare_group(1, W, N, 256, fake, 8, ctypes.byref(o), None, None, out) == lib.ERR_UNSUPPORTED_SHAPE
     assert out[0] is None
+
+
+def test_prepare_options_host_side_rejection(lib):
+    """serq_prepare / serq_prepare_shared / serq_prepare_group check their
+    options before touching a device."""
+    import numpy as np
+    L = lib.lib
+    o = lib.PrepareOpts()
+    L.serq_prepare_opts_init(ctypes.byref(o))
+    assert (abs(o.alpha - 0.5) < 1e-9, o.rank, o.mode, o.saliency, o.out_perm, o.out_colscale) == \
+        (True, 128, lib.W4A4, lib.SALIENCY_SCALE, None, None)
+    W = np.zeros((256, 64), np.float32)
+    Xc = np.zeros((4, 256), np.float32)
+    out = ctypes.c_void_p()
+    wp, xp = W.ctypes.data_as(ctypes.c_void_p), Xc.ctypes.data_as(ctypes.c_void_p)
+    for field, value, status, msg in (("alpha", 1.5, lib.ERR_INVALID_ARG, b"alpha"),
+                                      ("alpha", float("nan"), lib.ERR_INVALID_ARG, b"alpha"),
+                                      ("rank", 257, lib.ERR_UNSUPPORTED_SHAPE, b"rank"),
+                                      ("mode", 7, lib.ERR_INVALID_ARG, b"mode"),
+                                      ("saliency", 2, lib.ERR_INVALID_ARG, b"saliency")):
+        o = lib.prepare_opts(rank=32)
+        setattr(o, field, value)
+        assert L.serq_prepare(wp, 256, 64, xp, 4, ctypes.byref(o), ctypes.byref(out)) == status
+        assert msg in L.serq_last_error_string()
+        assert out.value is None
+    # a column scale without an order
+    o = lib.prepare_opts(rank=32)
+    d = np.ones(64, np.float32)
+    o.out_colscale = d.ctypes.data
+    assert L.serq_prepare(wp, 256, 64, xp, 4, ctypes.byref(o), ctypes.byref(out)) == lib.ERR_INVALID_ARG
+    assert b"without out_perm" in L.serq_last_error_string()
+    # group calls take the folds per weight, not in the options
+    Ws = (ctypes.c_void_p * 1)(W.ctypes.data)
+    Ns = (ctypes.c_int * 1)(64)
+    outs = (ctypes.c_void_p * 1)()
+    assert L.serq_prepare_shared(1, Ws, Ns, 256, xp, 4, ctypes.byref(o), None, None, outs) == lib.ERR_INVALID_ARG
+    assert b"per weight" in L.serq_last_error_string()
+    assert L.serq_prepare_shared(1, Ws, Ns, 256, xp, 4, None, None, None, outs) == lib.ERR_INVALID_ARG
+    assert outs[0] is None
     # silu: null inputs
     assert L.serq_silu_mul_quantize(None, None, 4, 256, 256, lib.W4A4, None, None, None) == lib.ERR_INVALID_ARG
 
@@ -106,3 +147,17 @@ def test_binding_refuses_to_load_without_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError, match="libserq.so not found"):
         spec.loader.exec_module(mod)
+
+
+def test_comparator_host_side_rejection(lib):
+    """The two-factor comparator's calls check their arguments on the host."""
+    L = lib.lib
+    out = ctypes.c_void_p()
+    fake = ctypes.c_void_p(0x1000)
+    assert L.serq_l2qer_prepare(None, fake, fake, 32, ctypes.byref(out)) == lib.ERR_INVALID_ARG
+    assert L.serq_l2qer_prepare(fake, None, fake, 32, ctypes.byref(out)) == lib.ERR_INVALID_ARG
+    assert out.value is None
+    assert L.serq_l2qer_linear(None, fake, fake, 4, fake, fake, fake, fake, 256, 0, None) == lib.ERR_INVALID_ARG
+    assert b"null comparator" in L.serq_last_error_string()
+    assert L.serq_l2qer_accum(None, fake, fake, 4, fake, fake, 0, None) == lib.ERR_INVALID_ARG
+    L.serq_l2qer_destroy(None)

@@ -89,18 +89,56 @@ def test_group_strided_outputs_into_one_buffer(S):
     assert torch.all(big[:, sum(Ns):] == 5.0)
 
 
-@pytest.mark.parametrize("M", [1, 7, 32])
-def test_group_decode_sizes(S, M):
-    """Decode-sized groups run one decode launch per layer."""
-    layers, olayers, Xq, sx, xq, osx = _group_case(S, M, 1024, [512, 256, 256], 128, "w4a4", seed=M)
-    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_TC):
+DECODE_GROUPS = [
+    # M, K, Ns, r, mode
+    (1, 1024, [512, 256, 256], 128, "w4a4"),
+    (7, 1024, [512, 256, 256], 128, "w4a4"),
+    (16, 1024, [512, 256, 256], 128, "w4a4"),
+    (32, 1024, [512, 256, 256], 128, "w4a4"),
+    (16, 768, [256, 96, 160, 512], 64, "w4a4"),   # four layers (the most a group takes)
+    (1, 512, [384, 128], 0, "w4a4"),              # rank 0: no compensator is read
+    (16, 512, [384, 128], 0, "w4a8"),
+    (1, 1024, [512, 128, 128], 128, "w4a8"),
+    (32, 640, [256, 128, 96, 64], 160, "w4a8"),   # four layers, rank padded to 192
+]
+
+
+@pytest.mark.parametrize("M,K,Ns,r,mode", DECODE_GROUPS)
+def test_group_decode_sizes(S, M, K, Ns, r, mode):
+    """Decode-sized groups: the mma.sync decode kernels run the whole group as
+    one launch (streaming kernel and item ring), DECODE_TC one launch per
+    layer; accumulators bit-exact, outputs within tolerance and equal to the
+    single-layer calls of the same kernel."""
+    layers, olayers, Xq, sx, xq, osx = _group_case(S, M, K, Ns, r, mode, seed=M + 3 * K + r)
+    want = [O.linear_accum(xq, ol) for ol in olayers]
+    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_TC):
         got = S.linear_group(layers, Xq, accum=True, algo=algo)
         Ys = S.linear_group(layers, Xq, sx, algo=algo)
+        singles = [S.linear(L, Xq, sx, algo=algo) for L in layers]
         torch.cuda.synchronize()
-        for (g0, g1), Y, ol in zip(got, Ys, olayers):
-            a0, a1 = O.linear_accum(xq, ol)
-            assert np.array_equal(g0.cpu().numpy(), a0) and np.array_equal(g1.cpu().numpy(), a1), f"algo {algo}"
+        for l, ((g0, g1), Y, Y1, (a0, a1), ol) in enumerate(zip(got, Ys, singles, want, olayers)):
+            assert np.array_equal(g0.cpu().numpy(), a0), f"acc0 of layer {l} differs (algo {algo})"
+            assert np.array_equal(g1.cpu().numpy(), a1), f"acc1 of layer {l} differs (algo {algo})"
+            assert torch.equal(Y.view(torch.int16), Y1.view(torch.int16)), f"layer {l} differs (algo {algo})"
             assert_y_close(Y, O.linear_epilogue(a0, a1, osx, ol))
+    assert S.device_error() == 0
+
+
+@pytest.mark.parametrize("M,mode", [(1, "w4a4"), (16, "w4a4"), (32, "w4a8")])
+def test_group_decode_strided_outputs_into_one_buffer(S, M, mode):
+    """Decode groups written side by side into one M x (sum N + 16) buffer:
+    every layer writes its own columns at the shared row stride only."""
+    Ns = [256, 128, 96]
+    layers, olayers, Xq, sx, xq, osx = _group_case(S, M, 512, Ns, 64, mode, seed=40 + M)
+    offs = np.concatenate([[0], np.cumsum(Ns)])
+    for algo in (S.ALGO_DECODE, S.ALGO_DECODE_ITEMS):
+        big = torch.full((M, sum(Ns) + 16), 5.0, dtype=torch.bfloat16, device="cuda")
+        Ys = [big[:, offs[l]:offs[l + 1]] for l in range(len(Ns))]
+        S.linear_group(layers, Xq, sx, Ys=Ys, algo=algo)
+        torch.cuda.synchronize()
+        for Y, ol in zip(Ys, olayers):
+            assert_y_close(Y, O.linear_epilogue(*O.linear_accum(xq, ol), osx, ol))
+        assert torch.all(big[:, sum(Ns):] == 5.0), f"algo {algo} wrote past the last layer"
 
 
 def test_llama2_7b_qkv_group_sampled(S):

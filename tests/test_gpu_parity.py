@@ -85,6 +85,45 @@ def test_prepare_with_output_fold(S):
     _check_prepared(L, ol)
 
 
+@pytest.mark.parametrize("alpha,saliency", [(0.5, 0), (0.5, 1), (0.8, 0), (0.3, 1), (1.0, 0)])
+def test_prepare_options_host_and_device_paths(S, alpha, saliency):
+    """serq_prepare (host arrays, one weight), serq_prepare_shared (host
+    arrays, a group) and serq_prepare_group (device arrays) with the same
+    options all give the oracle's bytes and scales bit for bit."""
+    rng = np.random.default_rng(int(alpha * 10) + 7 * saliency)
+    K, Ns, r = 512, [256, 128], 64
+    Xc = rng.standard_normal((40, K)).astype(np.float32)
+    Xc[:, rng.choice(K, 5, replace=False)] *= 40
+    Ws = [(0.02 * rng.standard_normal((K, n))).astype(np.float32) for n in Ns]
+    Ws[0][rng.choice(K, 3, replace=False)] *= 8          # rows whose folded maximum stands out
+    L1 = S.prepare_host(Ws[0], Xc, rank=r, alpha=alpha, saliency=saliency)
+    _check_prepared(L1, O.prepare(Ws[0], Xc, r, alpha=alpha, saliency=saliency))
+    _, _, ols = O.prepare_group(Ws, Xc, r, alpha=alpha, saliency=saliency)
+    Lh = S.prepare_shared_host(Ws, Xc, rank=r, alpha=alpha, saliency=saliency)
+    Ld = S.prepare_group([dev(W) for W in Ws], dev(Xc), r, "w4a4", alpha=alpha, saliency=saliency)
+    for a, b, ol in zip(Lh, Ld, ols):
+        _check_prepared(a, ol)
+        _check_prepared(b, ol)
+    perm, smooth = Lh[1].perm_smooth()
+    assert np.array_equal(perm, ols[1].pi) and np.array_equal(bits(smooth), bits(ols[1].s))
+    if saliency == 1:
+        s_only = O.saliency_perm(ols[0].s)
+        assert not np.array_equal(s_only, ols[0].pi), "the test data should tell the two metrics apart"
+
+
+def test_prepare_host_with_output_fold(S):
+    rng = np.random.default_rng(6)
+    K, N = 256, 192
+    W = (0.05 * rng.standard_normal((K, N))).astype(np.float32)
+    Xc = rng.standard_normal((32, K)).astype(np.float32)
+    P = rng.permutation(N).astype(np.int32)
+    d = rng.uniform(0.2, 5.0, N).astype(np.float32)
+    L = S.prepare_host(W, Xc, rank=32, out_perm=P, out_colscale=d)
+    _check_prepared(L, O.prepare(O.fold_output_columns(W, P, d), Xc, 32))
+    Ls = S.prepare_shared_host([W, W], Xc, rank=32, out_perm=[P, None], out_colscale=[d, None])
+    _check_prepared(Ls[1], O.prepare_group([O.fold_output_columns(W, P, d), W], Xc, 32)[2][1])
+
+
 # --------------------------------------------------- activations: quantize
 @pytest.mark.parametrize("act_dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("mode", ["w4a4", "w4a8"])
@@ -148,7 +187,7 @@ def test_linear_accum_bit_exact(S, mode, M, K, N, r):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, r, mode)
     acc0, acc1 = O.linear_accum(xq, ol)
     algos = [S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
-        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
+        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE, S.ALGO_DECODE_ITEMS] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
     for algo in algos:
         g0, g1 = S.linear_accum(L, Xq, algo)
         torch.cuda.synchronize()
@@ -164,7 +203,7 @@ def test_linear_output_within_tolerance(S, mode, M, K, N, r):
     acc0, acc1 = O.linear_accum(xq, ol)
     y_ref = O.linear_epilogue(acc0, acc1, osx, ol)
     algos = [S.ALGO_AUTO, S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
-        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
+        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE, S.ALGO_DECODE_ITEMS] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
     for algo in algos:
         Y = S.linear(L, Xq, sx, algo=algo)
         torch.cuda.synchronize()
@@ -174,7 +213,7 @@ def test_linear_output_within_tolerance(S, mode, M, K, N, r):
 def test_linear_strided_output(S):
     L, ol, Xq, sx, xq, osx = _linear_case(S, 40, 256, 128, 16, "w4a4")
     y_ref = O.linear_epilogue(*O.linear_accum(xq, ol), osx, ol)
-    for algo in (S.ALGO_PREFILL, S.ALGO_DECODE):
+    for algo in (S.ALGO_PREFILL, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS):
         big = torch.full((40, 200), 7.0, dtype=torch.bfloat16, device="cuda")
         S.linear(L, Xq, sx, Y=big[:, 8:136], algo=algo)
         torch.cuda.synchronize()
@@ -234,13 +273,28 @@ def test_mlp_block_chain(S):
     U = S.linear(Lu, Xq, sx)
     Hq, hsx = S.silu_mul_quantize(G, U, "w4a4")
     Y = S.linear(Ld, Hq, hsx)
+    d0, d1 = S.linear_accum(Ld, Hq)
     torch.cuda.synchronize()
     out = O.mlp_forward(blk.X, prep)
     # gate/up outputs within the bf16 tolerance
     assert_y_close(G, O.linear(out["xh"], prep["gate"])[0])
-    # the chain: g/u may round differently in the last bf16 place (fp32 vs
-    # fp64 epilogue), which may move a few down_proj input codes by one
+    assert_y_close(U, O.linear(out["xh"], prep["up"])[0])
+    # the intermediate codes from the GPU's own g/u are bit-exact (the oracle
+    # fed the same bf16 values)
+    g16 = G.float().cpu().numpy()
+    u16 = U.float().cpu().numpy()
+    hq_own, hsx_own = O.quantize_act(O.silu_mul_f32(g16, u16), 4)
     hq = Hq.cpu().numpy()
+    assert np.array_equal(hq, act_bytes(hq_own, 4))
+    assert np.array_equal(bits(hsx.cpu().numpy()), bits(hsx_own))
+    # down_proj on the GPU's own codes: accumulators bit-exact, the block
+    # output element by element within the tolerance
+    a0, a1 = O.linear_accum(hq_own, prep["down"])
+    assert np.array_equal(d0.cpu().numpy(), a0) and np.array_equal(d1.cpu().numpy(), a1)
+    assert_y_close(Y, O.linear_epilogue(a0, a1, hsx_own, prep["down"]))
+    # against the oracle's own chain: g/u may round differently in the last
+    # bf16 place (fp32 vs fp64 epilogue), which may move a few down_proj input
+    # codes by one
     ref_hq = act_bytes(out["hq"], 4)
     codes_g = O.unpack_int4_rows(hq).astype(int)
     codes_o = O.unpack_int4_rows(ref_hq).astype(int)
@@ -283,6 +337,33 @@ def test_llama2_7b_prefill_sampled(S, name):
     assert_y_close(Y[torch.from_numpy(rows).cuda()], O.linear_epilogue(acc0, acc1, osx, ol))
 
 
+@pytest.mark.parametrize("names", [["gate_proj", "up_proj"], ["down_proj"], ["q_proj", "k_proj", "v_proj"]])
+def test_llama3_8b_w4a8_sampled(S, names):
+    """Full Llama-3-8B projections at W4A8, M = 4096, through the calls the
+    bench makes (gate/up and q/k/v as one grouped launch): accumulators
+    bit-exact and outputs within tolerance on sampled rows."""
+    wl = synth.llama3_8b(M=4096, only=names)
+    inp = wl.inputs[wl.projections[0].input]
+    Ws = [p.W for p in wl.projections]
+    layers, olayers = _prepare_both(S, Ws, inp.X_calib, wl.rank, "w4a8")
+    for L, ol in zip(layers, olayers):
+        _check_prepared(L, ol)
+    _, Xq, sx = _gpu_act(S, layers[0], inp.X, "bf16", "w4a8")
+    Ys = S.linear_group(layers, Xq, sx)
+    accs = S.linear_group(layers, Xq, accum=True)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([[0, 255, 256, 4095], np.random.default_rng(4).choice(4096, 20, replace=False)]))
+    ol0 = olayers[0]
+    xq, osx = O.quantize_act(O.flatten_permute(inp.X[rows], ol0.s, ol0.pi, True), 8)
+    assert np.array_equal(Xq.cpu().numpy()[rows], act_bytes(xq, 8))
+    ridx = torch.from_numpy(rows).cuda()
+    for Y, (g0, g1), ol in zip(Ys, accs, olayers):
+        a0, a1 = O.linear_accum(xq, ol)
+        assert np.array_equal(g0.cpu().numpy()[rows], a0) and np.array_equal(g1.cpu().numpy()[rows], a1)
+        assert_y_close(Y[ridx], O.linear_epilogue(a0, a1, osx, ol))
+    del accs, Ys
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_llama2_7b_decode(S, M):
     wl = synth.llama2_7b(M=M, only=["gate_proj"])
@@ -291,7 +372,7 @@ def test_llama2_7b_decode(S, M):
     (L,), (ol,) = _prepare_both(S, [p.W], inp.X_calib, wl.rank, "w4a4")
     _, Xq, sx = _gpu_act(S, L, inp.X, "bf16", "w4a4")
     y_ref, xq, osx, acc0, acc1 = O.linear(O.flatten_permute(inp.X, ol.s, ol.pi, True), ol, 4)
-    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_TC):
+    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_TC):
         Y = S.linear(L, Xq, sx, algo=algo)
         g0, g1 = S.linear_accum(L, Xq, algo)
         torch.cuda.synchronize()
@@ -300,14 +381,16 @@ def test_llama2_7b_decode(S, M):
 
 
 @pytest.mark.parametrize("M,K,N,mode", [
-    (16, 11008, 512, "w4a4"),   # activations too large for shared memory next to the ring: read from L2
-    (8, 14336, 256, "w4a8"),    # an item fills half of shared memory: a one-stage ring
+    (16, 11008, 512, "w4a4"),   # item ring: activations read from L2; streaming: staged (89 KB)
+    (8, 14336, 256, "w4a8"),    # item ring: a one-stage ring; streaming: 115 KB of staged activations
+    (32, 11008, 256, "w4a4"),   # streaming: four token tiles next to 176 KB of activations (four warps)
+    (32, 14336, 128, "w4a8"),   # too large for the streaming kernel: DECODE falls back to the item ring
     (64, 4096, 256, "w4a4"),    # four 16-token tiles
 ])
 def test_decode_large_k(S, M, K, N, mode):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, 128, mode, seed=5)
     acc0, acc1 = O.linear_accum(xq, ol)
-    for algo in [S.ALGO_DECODE] + ([S.ALGO_DECODE_TC] if M <= 32 else []):
+    for algo in [S.ALGO_DECODE, S.ALGO_DECODE_ITEMS] + ([S.ALGO_DECODE_TC] if M <= 32 else []):
         g0, g1 = S.linear_accum(L, Xq, algo)
         Y = S.linear(L, Xq, sx, algo=algo)
         torch.cuda.synchronize()

@@ -6,11 +6,32 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libserq is written for sm_100a (B200); compile with -gencode arch=compute_100a,code=sm_100a"
 #endif
 
 namespace serq {
+
+// Raises a kernel's dynamic shared-memory limit on the current device to at
+// least `bytes`; the attribute is set at most once per kernel, device and
+// size, under a lock, so concurrent host threads need no coordination.
+inline cudaError_t smem_limit(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> have;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  int& cur = have[std::make_pair(kernel, dev)];
+  if (cur >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) cur = bytes;
+  return e;
+}
 
 // Status word that kernels set when a bounded wait gives up.  Read and
 // cleared by serq_device_error().
@@ -110,8 +131,8 @@ __device__ __forceinline__ void cluster_sync_all() {
 // kWaitLimitNs or, when `abort` is given, as soon as another role of the CTA
 // has raised it; on a timeout it records `who` in the device status word.
 template <bool CLUSTER = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int who) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int who,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   auto probe = [&]() { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (probe()) return true;
   const unsigned long long t0 = global_ns();
@@ -119,7 +140,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (probe()) return true;
     if ((it & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         if (abort != nullptr) *abort = 1;
         atomicCAS(&g_device_status, 0, who);
         return false;

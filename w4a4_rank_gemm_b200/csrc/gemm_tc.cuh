@@ -75,6 +75,7 @@ struct GroupArgs {
   int M, K, rpad;
   int nkb, nrb;
   const float* sx;
+  const float* sxr;  // two-source variant: per-row scale of the residual's activation codes
   int tiles_m;
   int nlayers, ntiles;
   LayerOut lo[kMaxGroup];
@@ -85,6 +86,7 @@ struct GroupMaps {
   CUtensorMap b[kMaxGroup];
   CUtensorMap r[kMaxGroup];
   CUtensorMap y[kMaxGroup];
+  CUtensorMap ar;  // activation codes of the residual steps (SERQ: the same map as the main steps)
 };
 
 // Layer of tile t and its tile index within that layer.
@@ -184,7 +186,14 @@ __device__ __forceinline__ void cta_sync() {
 // next tile waits on tmem_empty until every epilogue warp of the pair has
 // finished its TMEM reads (tcgen05.wait::ld -> tcgen05.fence::before_thread_sync
 // -> mbarrier arrive -> MMA warp wait -> tcgen05.fence::after_thread_sync).
-template <int BN, bool A8, bool ACC_OUT, int CG>
+//
+// TWO (the two-factor comparator): the residual steps read their activation
+// codes through mp.ar (a second, already quantized activation) and the
+// epilogue scales the two products by their own per-row scales,
+// y = sx * (sw * acc0) + sxr * (sR * acc1).  SERQ itself passes the main
+// activation map as mp.ar (its residual reuses the first r columns of the
+// same codes, key design 2) and TWO = false.
+template <int BN, bool A8, bool ACC_OUT, int CG, bool TWO = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ GroupMaps mp, const GroupArgs p) {
   using L = Layout<BN, A8, CG>;
@@ -231,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&mp.ar);
     for (int l = 0; l < p.nlayers; ++l) {
       tma_prefetch_desc(&mp.b[l]);
       tma_prefetch_desc(&mp.r[l]);
@@ -288,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&full_pk[s], L::kTxBytes);
             tma_load_2d(stage + L::kPkA, res ? &mp.r[l] : &mp.b[l], &full_pk[s], j * (BK / 2), nb0);
           }
-          tma_load_2d(stage, &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
+          tma_load_2d(stage, res ? &mp.ar : &tmA, &full_pk[s], j * (A8 ? BK : BK / 2), m0);
         }
       }
     }
@@ -449,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m0 = ((tl % p.tiles_m) * CG + (int)rank) * BM;
       const int n0 = (tl / p.tiles_m) * BN;
       // prefetch this tile's epilogue scales (consumed after the k loop)
-      float swv[kCpl], srv[kCpl], sxv = 0.f;
+      float swv[kCpl], srv[kCpl], sxv = 0.f, sxrv = 0.f;
       if (!ACC_OUT) {
 #pragma unroll
         for (int i = 0; i < kCpl; ++i) {
@@ -459,6 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int row = m0 + eq * 32 + lane;
         sxv = (row < p.M) ? __ldg(p.sx + row) : 0.f;
+        if (TWO) sxrv = (row < p.M) ? __ldg(p.sxr + row) : 0.f;
       }
 
       for (int step = 0; step < nsteps; ++step, ++g) {
@@ -570,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* bp = box_ptr(eq * (BN / 64) + (c >> 6)) + lane * 128;
           const int k0 = (c & 63) >> 3;  // first 16-byte chunk of these 16 columns
           const float2 sx2 = make_float2(sxv, sxv);
+          const float2 sxr2 = make_float2(sxrv, sxrv);
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             uint32_t pk[4];
@@ -587,8 +599,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float2 f0b = make_float2((float)(int)r0[e + 2], (float)(int)r0[e + 3]);
               const float2 f1a = make_float2((float)(int)r1[e], (float)(int)r1[e + 1]);
               const float2 f1b = make_float2((float)(int)r1[e + 2], (float)(int)r1[e + 3]);
-              const float2 ya = mul2(sx2, fma2(make_float2(w.x, w.y), f0a, mul2(make_float2(rr.x, rr.y), f1a)));
-              const float2 yb = mul2(sx2, fma2(make_float2(w.z, w.w), f0b, mul2(make_float2(rr.z, rr.w), f1b)));
+              float2 ya, yb;
+              if (TWO) {
+                ya = fma2(mul2(sx2, make_float2(w.x, w.y)), f0a, mul2(sxr2, mul2(make_float2(rr.x, rr.y), f1a)));
+                yb = fma2(mul2(sx2, make_float2(w.z, w.w)), f0b, mul2(sxr2, mul2(make_float2(rr.z, rr.w), f1b)));
+              } else {
+                ya = mul2(sx2, fma2(make_float2(w.x, w.y), f0a, mul2(make_float2(rr.x, rr.y), f1a)));
+                yb = mul2(sx2, fma2(make_float2(w.z, w.w), f0b, mul2(make_float2(rr.z, rr.w), f1b)));
+              }
               const __nv_bfloat162 h0 = __floats2bfloat162_rn(ya.x, ya.y);
               const __nv_bfloat162 h1 = __floats2bfloat162_rn(yb.x, yb.y);
               pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h0);

@@ -392,7 +392,7 @@ template <int MT, bool A8, bool ACC_OUT, bool ACT_SMEM>
 inline cudaError_t launch_mt(const Args& p, const Plan& pl, int sms, cudaStream_t st) {
   auto kern = k_decode<MT, A8, ACC_OUT, ACT_SMEM>;
   const int bytes = smem_bytes(pl, MT);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  cudaError_t e = serq::smem_limit(reinterpret_cast<const void*>(kern), bytes);
   if (e != cudaSuccess) return e;
   // persistent: as many CTAs as are resident at once (one or two per SM)
   int per_sm = 1;

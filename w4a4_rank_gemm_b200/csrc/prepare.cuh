@@ -61,15 +61,31 @@ __global__ void k_rowmax_abs(WeightView w, int K, float* __restrict__ amax_w) {
   }
 }
 
-// s_j = sqrt(max(amax_x, 1e-5)) / sqrt(max(amax_w, 1e-5))  (SmoothQuant form,
-// migration strength 1/2; SERQ notes key design 1).  In place over amax_x.
-__global__ void k_smooth(float* __restrict__ ax_to_s, const float* __restrict__ amax_w, int K) {
+// s_j = max(amax_x, 1e-5)^alpha / max(amax_w, 1e-5)^(1 - alpha)  (SmoothQuant's
+// static scale with migration strength alpha; SERQ notes key design 1).  At
+// the default alpha = 1/2 it is sqrt / sqrt / divide, each one fp32 rounding;
+// any other alpha is two fp64 powers and a division rounded to fp32 once.
+// In place over amax_x.
+__global__ void k_smooth(float* __restrict__ ax_to_s, const float* __restrict__ amax_w, int K, float alpha) {
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= K) return;
   const float floor_ = 1e-5f;
-  const float num = __fsqrt_rn(fmaxf(ax_to_s[j], floor_));
-  const float den = __fsqrt_rn(fmaxf(amax_w[j], floor_));
-  ax_to_s[j] = __fdiv_rn(num, den);
+  const float ax = fmaxf(ax_to_s[j], floor_), aw = fmaxf(amax_w[j], floor_);
+  if (alpha == 0.5f) {
+    ax_to_s[j] = __fdiv_rn(__fsqrt_rn(ax), __fsqrt_rn(aw));
+  } else {
+    const double a = (double)alpha;
+    ax_to_s[j] = __double2float_rn(__ddiv_rn(pow((double)ax, a), pow((double)aw, 1.0 - a)));
+  }
+}
+
+// Saliency key of channel j: s_j (metric 0) or the folded row's absolute
+// maximum s_j * max_n |W_jn| (metric 1, one fp32 multiply).
+__global__ void k_saliency_key(const float* __restrict__ s, const float* __restrict__ amax_w, int K, int metric,
+                               float* __restrict__ key) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= K) return;
+  key[j] = (metric == 1) ? __fmul_rn(s[j], amax_w[j]) : s[j];
 }
 
 // Saliency order (SERQ notes key design 2): position of channel i is the

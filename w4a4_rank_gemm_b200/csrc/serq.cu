@@ -10,11 +10,13 @@
 #include <mutex>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "../../include/serq.h"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_decode.cuh"
+#include "gemv_stream.cuh"
 #include "gemv_tc.cuh"
 #include "prepare.cuh"
 #include "quant.cuh"
@@ -193,10 +195,7 @@ serq_status check_layer(const serq_layer* L) {
   return SERQ_OK;
 }
 
-template <class K>
-void set_smem(K kernel, int bytes) {
-  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
+
 
 int sm_count() {
   static int cached[64] = {0};
@@ -233,8 +232,12 @@ struct LinearGroup {
   int32_t* acc1[serq::tc::kMaxGroup];
 };
 
-template <int BN, bool A8, bool ACC, int CG>
-cudaError_t launch_tc(const LinearGroup& G, const void* Xq, const float* sx, int M, cudaStream_t st) {
+// Xr / sxr: the two-factor comparator's second activation (codes M x rpad,
+// packed like Xq, and its per-row scales) for the residual steps; null for
+// SERQ, whose residual reads the first r columns of Xq.
+template <int BN, bool A8, bool ACC, int CG, bool TWO = false>
+cudaError_t launch_tc(const LinearGroup& G, const void* Xq, const float* sx, int M, cudaStream_t st,
+                      const void* Xr = nullptr, const float* sxr = nullptr) {
   using Lay = serq::tc::Layout<BN, A8, CG>;
   const serq_layer* L0 = G.L[0];
   const int K = L0->K;
@@ -253,7 +256,12 @@ cudaError_t launch_tc(const LinearGroup& G, const void* Xq, const float* sx, int
   ga.nkb = (K + serq::tc::BK - 1) / serq::tc::BK;
   ga.nrb = (L0->rpad + serq::tc::BK - 1) / serq::tc::BK;
   ga.sx = sx;
+  ga.sxr = sxr;
   ga.tiles_m = (M + serq::tc::BM * CG - 1) / (serq::tc::BM * CG);
+  mp.ar = tmA;
+  if (Xr && !make_map(&mp.ar, Xr, (uint64_t)L0->rpad / 2, (uint64_t)M, (uint64_t)L0->rpad / 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   ga.nlayers = G.n;
   int base = 0;
   for (int l = 0; l < serq::tc::kMaxGroup; ++l) {
@@ -270,13 +278,10 @@ cudaError_t launch_tc(const LinearGroup& G, const void* Xq, const float* sx, int
     if (l < G.n) base += ga.tiles_m * ((Ll->N + BN - 1) / BN);
   }
   ga.ntiles = base;
-  auto kern = serq::tc::k_gemm<BN, A8, ACC, CG>;
-  static int attr_set[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    set_smem(kern, Lay::kAlloc);
-    attr_set[dev] = 1;
+  auto kern = serq::tc::k_gemm<BN, A8, ACC, CG, TWO>;
+  {
+    const cudaError_t ea = serq::smem_limit(reinterpret_cast<const void*>(kern), Lay::kAlloc);
+    if (ea != cudaSuccess) return ea;
   }
   // persistent: one CTA (pair) per SM (pair of SMs), tiles strided over them
   const long slots = sm_count() / CG;
@@ -311,12 +316,9 @@ cudaError_t launch_tc_ta(const serq_layer* L, const void* Xq, const serq::tc::Ar
                         CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
     return cudaErrorInvalidValue;
   auto kern = serq::tc::k_gemm_ta<BN, ACC>;
-  static int attr_set[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    set_smem(kern, Lay::kAlloc);
-    attr_set[dev] = 1;
+  {
+    const cudaError_t ea = serq::smem_limit(reinterpret_cast<const void*>(kern), Lay::kAlloc);
+    if (ea != cudaSuccess) return ea;
   }
   serq::tc::Args ap = a;
   ap.tiles_m = (a.M + 255) / 256;
@@ -348,12 +350,9 @@ cudaError_t launch_decode_tc(const serq_layer* L, const void* Xq, serq::dtc::Arg
                 : make_map(&tmX, Xq, (uint64_t)a.K / 2, (uint64_t)a.M, (uint64_t)a.K / 2, 64, MP, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!okm) return cudaErrorInvalidValue;
   auto kern = serq::dtc::k_decode_tc<MP, A8, ACC>;
-  static int attr_set[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    set_smem(kern, Lay::kAlloc);
-    attr_set[dev] = 1;
+  {
+    const cudaError_t ea = serq::smem_limit(reinterpret_cast<const void*>(kern), Lay::kAlloc);
+    if (ea != cudaSuccess) return ea;
   }
   const int tiles = (a.N + serq::dtc::BM - 1) / serq::dtc::BM;
   int splits = (2 * sm_count() + tiles / 2) / tiles;
@@ -407,10 +406,40 @@ cudaError_t dispatch_tc(const LinearGroup& G, const void* Xq, const float* sx, i
   return launch_tc<128, A8, ACC, 1>(G, Xq, sx, M, st);
 }
 
-// The mma.sync decode kernel over a group of layers (one launch; one layer
-// is a group of one).
+// The mma.sync decode kernels over a group of layers (one launch; one layer
+// is a group of one): the streaming kernel where its shared memory fits
+// (M <= 32 and the staged activations leave room for the rings), else, or
+// when asked for by SERQ_ALGO_DECODE_ITEMS, the item-ring kernel.
+// fault_wait_ns is zero except in the failure-detection test hook.
 cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const float* sx, int M, bool a8, bool accum,
-                                cudaStream_t st) {
+                                bool items, cudaStream_t st, unsigned long long fault_wait_ns = 0) {
+  if (!items) {
+    serq::gs::Args g = {};
+    g.Xq = static_cast<const uint8_t*>(Xq);
+    g.sx = sx;
+    g.M = M;
+    g.K = G.L[0]->K;
+    g.rpad = G.L[0]->rpad;
+    g.nlayers = G.n;
+    int base = 0;
+    for (int l = 0; l < serq::gs::kMaxGroup; ++l) {
+      const int li = (l < G.n) ? l : 0;
+      const serq_layer* L = G.L[li];
+      g.lo[l] = serq::gs::Layer{L->wq, L->rq, L->sw, L->sr, G.Y[li], G.ldy[li], G.acc0[li], G.acc1[li], L->N,
+                                l < G.n ? base : 1 << 30};
+      if (l < G.n) base += L->N;
+    }
+    g.C = base;
+    const bool fit = a8 ? serq::gs::fits<true>(g, sm_count(), max_smem()) : serq::gs::fits<false>(g, sm_count(), max_smem());
+    if (fit) {
+      if (a8)
+        return accum ? serq::gs::launch<true, true>(g, sm_count(), max_smem(), st, fault_wait_ns)
+                     : serq::gs::launch<true, false>(g, sm_count(), max_smem(), st, fault_wait_ns);
+      return accum ? serq::gs::launch<false, true>(g, sm_count(), max_smem(), st, fault_wait_ns)
+                   : serq::gs::launch<false, false>(g, sm_count(), max_smem(), st, fault_wait_ns);
+    }
+    if (fault_wait_ns) return cudaErrorInvalidValue;
+  }
   serq::decode::Args a = {};
   a.Xq = static_cast<const uint8_t*>(Xq);
   a.sx = sx;
@@ -418,14 +447,14 @@ cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const floa
   a.K = G.L[0]->K;
   a.rpad = G.L[0]->rpad;
   a.nlayers = G.n;
-  int items = 0;
+  int items_n = 0;
   for (int l = 0; l < serq::decode::kMaxGroup; ++l) {
     const int li = (l < G.n) ? l : 0;
     const serq_layer* L = G.L[li];
-    a.lo[l] = serq::decode::LayerDec{L->wq, L->rq, L->sw, L->sr, G.Y[li], G.ldy[li], G.acc0[li], G.acc1[li], L->N, items};
-    if (l < G.n) items += L->N / serq::decode::kRows;
+    a.lo[l] = serq::decode::LayerDec{L->wq, L->rq, L->sw, L->sr, G.Y[li], G.ldy[li], G.acc0[li], G.acc1[li], L->N, items_n};
+    if (l < G.n) items_n += L->N / serq::decode::kRows;
   }
-  a.N = items * serq::decode::kRows;
+  a.N = items_n * serq::decode::kRows;
   if (a8)
     return accum ? serq::decode::launch<true, true>(a, sm_count(), max_smem(), st)
                  : serq::decode::launch<true, false>(a, sm_count(), max_smem(), st);
@@ -453,11 +482,11 @@ serq_status check_linear(const serq_layer* L, const void* Xq, const float* sx, i
       return fail(SERQ_ERR_INVALID_ARG, "Y must be 16-byte aligned with ldy a multiple of 8");
   }
   if (algo == SERQ_ALGO_AUTO) algo = (M <= serq_decode_max_m()) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
-  if (algo == SERQ_ALGO_DECODE && M > serq::decode::kMaxTiles * 16)
+  if ((algo == SERQ_ALGO_DECODE || algo == SERQ_ALGO_DECODE_ITEMS) && M > serq::decode::kMaxTiles * 16)
     return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "decode kernel takes M <= %d (got %d)", serq::decode::kMaxTiles * 16, M);
   if (algo == SERQ_ALGO_DECODE_TC && M > serq::dtc::kMaxM)
     return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "SERQ_ALGO_DECODE_TC takes M <= %d (got %d)", serq::dtc::kMaxM, M);
-  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_DECODE_TC) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
+  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_DECODE_ITEMS) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
   if (algo == SERQ_ALGO_PREFILL_PAIR_TMEM_A && L->mode != SERQ_W4A4)
     return fail(SERQ_ERR_INVALID_ARG, "SERQ_ALGO_PREFILL_PAIR_TMEM_A takes W4A4 layers");
   if ((s = check_device())) return s;
@@ -483,7 +512,7 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
       e = accum ? dispatch_decode_tc<true, true>(L, Xq, a, st) : dispatch_decode_tc<true, false>(L, Xq, a, st);
     else
       e = accum ? dispatch_decode_tc<false, true>(L, Xq, a, st) : dispatch_decode_tc<false, false>(L, Xq, a, st);
-  } else if (algo == SERQ_ALGO_DECODE) {
+  } else if (algo == SERQ_ALGO_DECODE || algo == SERQ_ALGO_DECODE_ITEMS) {
     LinearGroup G = {};
     G.n = 1;
     G.L[0] = L;
@@ -491,7 +520,7 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
     G.ldy[0] = ldy;
     G.acc0[0] = acc0;
     G.acc1[0] = acc1;
-    e = launch_decode_group(G, Xq, sx, M, a8, accum, st);
+    e = launch_decode_group(G, Xq, sx, M, a8, accum, algo == SERQ_ALGO_DECODE_ITEMS, st);
   } else {
     LinearGroup G = {};
     G.n = 1;
@@ -509,9 +538,10 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
   return ok();
 }
 
-// Several layers over the same activation codes: prefill kernels run them as
-// one launch (one tile space, one pass of setup and tail); decode kernels and
-// the TMEM-activation variant run them one launch per layer.
+// Several layers over the same activation codes: the prefill kernels and the
+// mma.sync decode kernels run them as one launch (one tile or channel space,
+// one pass of setup and tail); SERQ_ALGO_DECODE_TC and the TMEM-activation
+// variant run them one launch per layer.
 serq_status group_impl(int n, const serq_layer* const* Ls, const void* Xq, const float* sx, int M,
                        void* const* Y, const int* ldy, int32_t* const* acc0, int32_t* const* acc1, serq_algo algo,
                        void* stream) {
@@ -551,8 +581,8 @@ serq_status group_impl(int n, const serq_layer* const* Ls, const void* Xq, const
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (resolved == SERQ_ALGO_DECODE) {
-    e = launch_decode_group(G, Xq, sx, M, Ls[0]->mode == SERQ_W4A8, accum, st);
+  if (resolved == SERQ_ALGO_DECODE || resolved == SERQ_ALGO_DECODE_ITEMS) {
+    e = launch_decode_group(G, Xq, sx, M, Ls[0]->mode == SERQ_W4A8, accum, resolved == SERQ_ALGO_DECODE_ITEMS, st);
     if (e != cudaSuccess) return cuda_fail(e, "serq_linear_group launch");
     return ok();
   }
@@ -584,25 +614,42 @@ constexpr size_t kStaticCntOffset = (size_t)2 * serq::dtc::kMaxM * kStaticMaxN;
 constexpr size_t kStaticInts = kStaticCntOffset + kStaticMaxN / serq::dtc::BM;
 static __device__ __align__(256) int32_t g_decode_scratch[kStaticInts];
 
-// Device address of the scratch, looked up once per device; the first call
-// on a device clears it (it must start at zero; every completed call leaves
-// it zero).
-serq_status static_scratch(int32_t** out) {
-  static std::mutex mu;
-  static int32_t* addr[64] = {nullptr};
+// Device address of the scratch, looked up once per device with that device
+// current.  The scratch must start at zero and every completed call leaves it
+// zero, so it is cleared (on the call's own stream, ordered before the
+// kernel) only on the first call on a device and after a kernel reported a
+// timed-out wait, which can leave partial sums behind.
+std::mutex g_static_mu;
+int32_t* g_static_addr[64] = {nullptr};
+bool g_static_dirty[64] = {false};
+
+serq_status static_scratch(cudaStream_t st, int32_t** out) {
   int dev = 0;
-  cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(SERQ_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
     void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e == cudaSuccess) e = cudaMemset(p, 0, kStaticInts * sizeof(int32_t));
-    if (e != cudaSuccess) return cuda_fail(e, "static decode scratch");
-    addr[dev] = static_cast<int32_t*>(p);
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static decode scratch");
+    g_static_addr[dev] = static_cast<int32_t*>(p);
+    g_static_dirty[dev] = true;
   }
-  *out = addr[dev];
+  if (g_static_dirty[dev]) {
+    e = cudaMemsetAsync(g_static_addr[dev], 0, kStaticInts * sizeof(int32_t), st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the static decode scratch");
+    g_static_dirty[dev] = false;
+  }
+  *out = g_static_addr[dev];
   return SERQ_OK;
+}
+
+// After a reported timeout on `dev`, the next static call clears the scratch.
+void static_scratch_mark_dirty(int dev) {
+  if (dev < 0 || dev >= 64) return;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  g_static_dirty[dev] = true;
 }
 
 }  // namespace
@@ -629,33 +676,47 @@ serq_status serq_device_error(int* code) {
   if (e != cudaSuccess) return cuda_fail(e, "read device status");
   e = cudaMemcpyToSymbol(serq::g_device_status, &zero, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e, "clear device status");
+  if (v != 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) static_scratch_mark_dirty(dev);
+  }
   *code = v;
   return ok();
 }
 
-serq_status serq_prepare_group(int n_weights, const float* const* W, const int* N, int K,
-                               const float* X_calib, int n_calib, int rank, serq_mode mode,
-                               const int32_t* const* out_perm, const float* const* out_div,
-                               serq_layer** layers) {
-  if (!layers) return fail(SERQ_ERR_INVALID_ARG, "null layers");
-  if (n_weights < 1 || n_weights > 64) return fail(SERQ_ERR_INVALID_ARG, "n_weights = %d", n_weights);
-  for (int i = 0; i < n_weights; ++i) layers[i] = nullptr;
-  serq_status s;
-  if (!W || !N || !X_calib) return fail(SERQ_ERR_INVALID_ARG, "null W, N or X_calib");
-  if (K < 32 || K % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "K = %d must be a positive multiple of 32", K);
-  if (n_calib < 1) return fail(SERQ_ERR_INVALID_ARG, "n_calib = %d", n_calib);
-  if (rank < 0 || rank > K) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "rank %d not in [0, K=%d]", rank, K);
-  if (mode != SERQ_W4A4 && mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode %d", (int)mode);
-  for (int i = 0; i < n_weights; ++i) {
-    if (!W[i]) return fail(SERQ_ERR_INVALID_ARG, "null W[%d]", i);
-    if (N[i] < 32 || N[i] % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "N[%d] = %d must be a positive multiple of 32", i, N[i]);
-    if (out_div && out_div[i] && !(out_perm && out_perm[i]))
-      return fail(SERQ_ERR_INVALID_ARG, "out_div[%d] given without out_perm[%d]", i, i);
-  }
-  if ((s = check_device())) return s;
+void serq_prepare_opts_init(serq_prepare_opts* opts) {
+  if (!opts) return;
+  opts->alpha = 0.5f;
+  opts->rank = 128;
+  opts->mode = SERQ_W4A4;
+  opts->saliency = SERQ_SALIENCY_SCALE;
+  opts->out_perm = nullptr;
+  opts->out_colscale = nullptr;
+}
 
+}  // extern "C"
+
+namespace {
+
+// Checks the options shared by every prepare entry point.
+serq_status check_opts(const serq_prepare_opts* o, int K) {
+  if (!o) return fail(SERQ_ERR_INVALID_ARG, "null options");
+  if (!(o->alpha >= 0.f && o->alpha <= 1.f)) return fail(SERQ_ERR_INVALID_ARG, "alpha = %g not in [0, 1]", o->alpha);
+  if (o->rank < 0 || o->rank > K) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "rank %d not in [0, K=%d]", o->rank, K);
+  if (o->mode != SERQ_W4A4 && o->mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode %d", (int)o->mode);
+  if (o->saliency != SERQ_SALIENCY_SCALE && o->saliency != SERQ_SALIENCY_ROW_ABSMAX)
+    return fail(SERQ_ERR_INVALID_ARG, "bad saliency metric %d", o->saliency);
+  return SERQ_OK;
+}
+
+// The offline stage on device-resident inputs (all pointers DEVICE).
+serq_status prepare_impl(int n_weights, const float* const* W, const int* N, int K, const float* X_calib,
+                         int n_calib, const serq_prepare_opts& o, const int32_t* const* out_perm,
+                         const float* const* out_div, serq_layer** layers) {
+  serq_status s;
+  const int rank = o.rank;
   for (int i = 0; i < n_weights; ++i) {
-    s = alloc_layer(K, N[i], rank, mode, &layers[i]);
+    s = alloc_layer(K, N[i], rank, o.mode, &layers[i]);
     if (s) {
       for (int j = 0; j < i; ++j) {
         free_layer(layers[j]);
@@ -671,10 +732,18 @@ serq_status serq_prepare_group(int n_weights, const float* const* W, const int* 
     }
     return st;
   };
-
+  float* key = nullptr;
+  cudaError_t e = cudaMalloc(&key, sizeof(float) * K);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cleanup(fail(SERQ_ERR_ALLOC, "cudaMalloc of the saliency keys failed: %s", cudaGetErrorString(e)));
+  }
   cudaStream_t st;
-  cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
-  if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaStreamCreate"));
+  e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    cudaFree(key);
+    return cleanup(cuda_fail(e, "cudaStreamCreate"));
+  }
   using namespace serq::prep;
   serq_layer* L0 = layers[0];
   auto view = [&](int i) {
@@ -685,9 +754,10 @@ serq_status serq_prepare_group(int n_weights, const float* const* W, const int* 
   k_colmax_abs<<<(K + 255) / 256, 256, 0, st>>>(X_calib, n_calib, K, L0->smooth);
   cudaMemsetAsync(amax_w, 0, sizeof(float) * K, st);
   for (int i = 0; i < n_weights; ++i) k_rowmax_abs<<<K, 256, 0, st>>>(view(i), K, amax_w);
-  k_smooth<<<(K + 255) / 256, 256, 0, st>>>(L0->smooth, amax_w, K);
+  k_smooth<<<(K + 255) / 256, 256, 0, st>>>(L0->smooth, amax_w, K, o.alpha);
   // 2. saliency order
-  k_rank_perm<<<(K + 255) / 256, 256, 256 * sizeof(float), st>>>(L0->smooth, K, L0->perm);
+  k_saliency_key<<<(K + 255) / 256, 256, 0, st>>>(L0->smooth, amax_w, K, o.saliency, key);
+  k_rank_perm<<<(K + 255) / 256, 256, 256 * sizeof(float), st>>>(key, K, L0->perm);
   for (int i = 1; i < n_weights; ++i) {
     cudaMemcpyAsync(layers[i]->smooth, L0->smooth, sizeof(float) * K, cudaMemcpyDeviceToDevice, st);
     cudaMemcpyAsync(layers[i]->perm, L0->perm, sizeof(int32_t) * K, cudaMemcpyDeviceToDevice, st);
@@ -712,6 +782,7 @@ serq_status serq_prepare_group(int n_weights, const float* const* W, const int* 
   e = cudaGetLastError();
   cudaError_t e2 = cudaStreamSynchronize(st);
   cudaStreamDestroy(st);
+  cudaFree(key);
   if (e != cudaSuccess) return cleanup(cuda_fail(e, "serq_prepare launch"));
   if (e2 != cudaSuccess) return cleanup(cuda_fail(e2, "serq_prepare"));
   for (int i = 0; i < n_weights; ++i)
@@ -719,13 +790,116 @@ serq_status serq_prepare_group(int n_weights, const float* const* W, const int* 
   return ok();
 }
 
-serq_status serq_prepare(const float* W, int K, int N, const float* X_calib, int n_calib, int rank,
-                         serq_mode mode, const int32_t* out_perm, const float* out_div, serq_layer** layer) {
+// Argument checks of the group calls (host or device pointers alike).
+serq_status check_group_args(int n_weights, const float* const* W, const int* N, int K, const float* X_calib,
+                             int n_calib, const serq_prepare_opts* opts, const int32_t* const* out_perm,
+                             const float* const* out_div, serq_layer** layers) {
+  if (!layers) return fail(SERQ_ERR_INVALID_ARG, "null layers");
+  if (n_weights < 1 || n_weights > 64) return fail(SERQ_ERR_INVALID_ARG, "n_weights = %d", n_weights);
+  for (int i = 0; i < n_weights; ++i) layers[i] = nullptr;
+  serq_status s;
+  if (!W || !N || !X_calib) return fail(SERQ_ERR_INVALID_ARG, "null W, N or X_calib");
+  if (K < 32 || K % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "K = %d must be a positive multiple of 32", K);
+  if (n_calib < 1) return fail(SERQ_ERR_INVALID_ARG, "n_calib = %d", n_calib);
+  if ((s = check_opts(opts, K))) return s;
+  if (opts->out_perm || opts->out_colscale)
+    return fail(SERQ_ERR_INVALID_ARG, "group calls take the folds per weight (out_perm / out_colscale arrays), "
+                                      "not in the options");
+  for (int i = 0; i < n_weights; ++i) {
+    if (!W[i]) return fail(SERQ_ERR_INVALID_ARG, "null W[%d]", i);
+    if (N[i] < 32 || N[i] % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "N[%d] = %d must be a positive multiple of 32", i, N[i]);
+    if (out_div && out_div[i] && !(out_perm && out_perm[i]))
+      return fail(SERQ_ERR_INVALID_ARG, "out_colscale[%d] given without out_perm[%d]", i, i);
+  }
+  return check_device();
+}
+
+// Device copies of host arrays for the host-pointer prepare calls; freed
+// when the owner goes out of scope.
+struct Uploads {
+  std::vector<void*> bufs;
+  ~Uploads() {
+    for (void* b : bufs) cudaFree(b);
+  }
+  template <class T>
+  serq_status put(const T* host, size_t count, const T** out) {
+    *out = nullptr;
+    if (!host) return SERQ_OK;
+    void* d = nullptr;
+    cudaError_t e = cudaMalloc(&d, count * sizeof(T));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(SERQ_ERR_ALLOC, "cudaMalloc(%zu) for an upload failed: %s", count * sizeof(T), cudaGetErrorString(e));
+    }
+    bufs.push_back(d);
+    e = cudaMemcpy(d, host, count * sizeof(T), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy of a prepare input");
+    *out = static_cast<const T*>(d);
+    return SERQ_OK;
+  }
+};
+
+serq_status prepare_shared_host(int n_weights, const float* const* W, const int* N, int K, const float* X_calib,
+                                int n_calib, const serq_prepare_opts& o, const int32_t* const* out_perm,
+                                const float* const* out_div, serq_layer** layers) {
+  Uploads up;
+  std::vector<const float*> dW(n_weights, nullptr), dDiv(n_weights, nullptr);
+  std::vector<const int32_t*> dPerm(n_weights, nullptr);
+  const float* dX = nullptr;
+  serq_status s;
+  for (int i = 0; i < n_weights; ++i) {
+    if ((s = up.put(W[i], (size_t)K * N[i], &dW[i]))) return s;
+    if (out_perm && (s = up.put(out_perm[i], (size_t)N[i], &dPerm[i]))) return s;
+    if (out_div && (s = up.put(out_div[i], (size_t)N[i], &dDiv[i]))) return s;
+  }
+  if ((s = up.put(X_calib, (size_t)n_calib * K, &dX))) return s;
+  return prepare_impl(n_weights, dW.data(), N, K, dX, n_calib, o, dPerm.data(), dDiv.data(), layers);
+}
+
+}  // namespace
+
+extern "C" {
+
+serq_status serq_prepare_group(int n_weights, const float* const* W, const int* N, int K, const float* X_calib,
+                               int n_calib, const serq_prepare_opts* opts, const int32_t* const* out_perm,
+                               const float* const* out_colscale, serq_layer** layers) {
+  serq_status s = check_group_args(n_weights, W, N, K, X_calib, n_calib, opts, out_perm, out_colscale, layers);
+  if (s) return s;
+  return prepare_impl(n_weights, W, N, K, X_calib, n_calib, *opts, out_perm, out_colscale, layers);
+}
+
+serq_status serq_prepare_shared(int n_weights, const float* const* W, const int* N, int K, const float* X_calib,
+                                int n_calib, const serq_prepare_opts* opts, const int32_t* const* out_perm,
+                                const float* const* out_colscale, serq_layer** layers) {
+  serq_status s = check_group_args(n_weights, W, N, K, X_calib, n_calib, opts, out_perm, out_colscale, layers);
+  if (s) return s;
+  return prepare_shared_host(n_weights, W, N, K, X_calib, n_calib, *opts, out_perm, out_colscale, layers);
+}
+
+serq_status serq_prepare(const float* W, int K, int N, const float* X_calib, int n_calib,
+                         const serq_prepare_opts* opts, serq_layer** layer) {
+  serq_prepare_opts o;
+  serq_prepare_opts_init(&o);
+  if (opts) o = *opts;
   const float* Ws[1] = {W};
   const int Ns[1] = {N};
-  const int32_t* ps[1] = {out_perm};
-  const float* ds[1] = {out_div};
-  return serq_prepare_group(1, Ws, Ns, K, X_calib, n_calib, rank, mode, ps, ds, layer);
+  const int32_t* ps[1] = {o.out_perm};
+  const float* ds[1] = {o.out_colscale};
+  o.out_perm = nullptr;
+  o.out_colscale = nullptr;
+  serq_status s = check_group_args(1, Ws, Ns, K, X_calib, n_calib, &o, ps, ds, layer);
+  if (s) return s;
+  return prepare_shared_host(1, Ws, Ns, K, X_calib, n_calib, o, ps, ds, layer);
+}
+
+serq_status serq_layer_get_perm(const serq_layer* L, int32_t* host_out) {
+  if (!host_out) return fail(SERQ_ERR_INVALID_ARG, "null output");
+  return serq_layer_get_packed(L, nullptr, nullptr, nullptr, nullptr, host_out, nullptr);
+}
+
+serq_status serq_layer_get_smooth(const serq_layer* L, float* host_out) {
+  if (!host_out) return fail(SERQ_ERR_INVALID_ARG, "null output");
+  return serq_layer_get_packed(L, nullptr, nullptr, nullptr, nullptr, nullptr, host_out);
 }
 
 void serq_layer_destroy(serq_layer* layer) { free_layer(layer); }
@@ -855,6 +1029,24 @@ serq_status serq_linear_group(int n, const serq_layer* const* layers, const void
   return group_impl(n, layers, Xq, sx, M, Y, ldy, acc0, acc1, algo, stream);
 }
 
+serq_status serq_test_decode_timeout(const serq_layer* layer, const void* Xq, const float* sx, int M, void* Y,
+                                     int ldy, int wait_us, void* stream) {
+  if (wait_us < 1 || wait_us > 1000000) return fail(SERQ_ERR_INVALID_ARG, "wait_us = %d not in [1, 1e6]", wait_us);
+  serq_algo algo = SERQ_ALGO_DECODE;
+  serq_status s;
+  if ((s = check_linear(layer, Xq, sx, M, Y, ldy, nullptr, nullptr, &algo))) return s;
+  if (M > 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "the streaming decode kernel takes M <= 32");
+  LinearGroup G = {};
+  G.n = 1;
+  G.L[0] = layer;
+  G.Y[0] = static_cast<__nv_bfloat16*>(Y);
+  G.ldy[0] = ldy;
+  cudaError_t e = launch_decode_group(G, Xq, sx, M, layer->mode == SERQ_W4A8, false, false,
+                                      static_cast<cudaStream_t>(stream), (unsigned long long)wait_us * 1000ull);
+  if (e != cudaSuccess) return cuda_fail(e, "serq_test_decode_timeout launch");
+  return ok();
+}
+
 serq_status serq_linear_decode_static(const serq_layer* layer, const void* Xq, const float* sx, int M, void* Y,
                                       int ldy, int32_t* acc0, int32_t* acc1, void* stream) {
   if (!layer) return fail(SERQ_ERR_INVALID_ARG, "null layer");
@@ -866,9 +1058,246 @@ serq_status serq_linear_decode_static(const serq_layer* layer, const void* Xq, c
   serq_status s = check_device();
   if (s) return s;
   int32_t* scratch = nullptr;
-  if ((s = static_scratch(&scratch))) return s;
+  if ((s = static_scratch(static_cast<cudaStream_t>(stream), &scratch))) return s;
   return linear_impl(layer, Xq, sx, M, Y, ldy, acc0, acc1, SERQ_ALGO_DECODE_TC, stream, scratch,
                      scratch + kStaticCntOffset);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------
+// The two-factor comparator (L2QER): X_q W_q + Q(X_q L1_q) L2_q on the
+// kernels above.  L1 runs as a layer of r output channels (rank 0), its bf16
+// output is quantized per token by the activation quantizer, and the final
+// GEMM reads those codes in its residual steps with L2 in place of R.
+// ------------------------------------------------------------------------
+struct serq_l2qer {
+  int K, N, r;
+  serq_layer* f1;    // L1: r x K/2 packed codes, per-channel scales (owned)
+  serq_layer view;   // the base layer with R / sR replaced by L2's codes / scales
+  void* block;       // L2's codes (N x r/2) and scales (N)
+};
+
+namespace {
+
+// scale = amax / 7 in place (the symmetric INT4 scale, one fp32 division)
+__global__ void k_amax_to_scale(float* a, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) a[i] = __fdiv_rn(a[i], 7.f);
+}
+
+// Per-column INT4 quantization and packing of a plain K x N fp32 matrix
+// (no smoothing, identity order) into codes (N x K/2) and scales (N).
+serq_status quantize_columns(const float* W, int K, int N, uint8_t* codes, float* scales, const float* ones,
+                             const int32_t* ident, cudaStream_t st) {
+  using namespace serq::prep;
+  const WeightView v{W, N, nullptr, nullptr};
+  const int rows_per_block = 64;
+  cudaMemsetAsync(scales, 0, sizeof(float) * N, st);
+  k_colmax_what<<<dim3((N + 255) / 256, (K + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(
+      v, ones, ident, K, rows_per_block, scales);
+  k_quant_pack_w<<<dim3((N + 127) / 128, K / 32), 128, 0, st>>>(v, ones, ident, K, scales, codes);
+  k_amax_to_scale<<<(N + 255) / 256, 256, 0, st>>>(scales, N);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SERQ_OK : cuda_fail(e, "quantizing a factor");
+}
+
+__global__ void k_fill_ones_iota(float* ones, int32_t* ident, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    ones[i] = 1.f;
+    ident[i] = i;
+  }
+}
+
+void free_l2qer(serq_l2qer* q) {
+  if (!q) return;
+  free_layer(q->f1);
+  if (q->block) cudaFree(q->block);
+  delete q;
+}
+
+template <bool ACC>
+cudaError_t dispatch_two(const LinearGroup& G, const void* Xq, const float* sx, int M, serq_algo algo,
+                         const void* Zq, const float* sz, cudaStream_t st) {
+  if (algo == SERQ_ALGO_PREFILL_N128) return launch_tc<128, false, ACC, 1, !ACC>(G, Xq, sx, M, st, Zq, sz);
+  if (algo == SERQ_ALGO_PREFILL_PAIR_N256) return launch_tc<256, false, ACC, 2, !ACC>(G, Xq, sx, M, st, Zq, sz);
+  const long ctas_pair = (long)((G.L[0]->N + 255) / 256) * 2 * ((M + 255) / 256);
+  if (ctas_pair * 10 >= (long)sm_count() * 9) return launch_tc<256, false, ACC, 2, !ACC>(G, Xq, sx, M, st, Zq, sz);
+  return launch_tc<128, false, ACC, 1, !ACC>(G, Xq, sx, M, st, Zq, sz);
+}
+
+// Final GEMM of the comparator (main product + L2 on the intermediate codes).
+serq_status l2qer_final(const serq_l2qer* q, const void* Xq, const float* sx, int M, const void* Zq, const float* sz,
+                        void* Y, int ldy, int32_t* acc0, int32_t* acc1, serq_algo algo, cudaStream_t st) {
+  const bool accum = acc0 != nullptr;
+  if (!aligned16(Zq)) return fail(SERQ_ERR_INVALID_ARG, "Zq must be 16-byte aligned");
+  if (!accum && !aligned16(sz)) return fail(SERQ_ERR_INVALID_ARG, "null or misaligned sz");
+  cudaError_t e;
+  if (algo == SERQ_ALGO_DECODE) {
+    serq::gs::Args g = {};
+    g.Xq = static_cast<const uint8_t*>(Xq);
+    g.sx = sx;
+    g.Xr = static_cast<const uint8_t*>(Zq);
+    g.sxr = accum ? nullptr : sz;
+    g.M = M;
+    g.K = q->K;
+    g.rpad = q->view.rpad;
+    g.nlayers = 1;
+    const serq_layer* L = &q->view;
+    for (int l = 0; l < serq::gs::kMaxGroup; ++l)
+      g.lo[l] = serq::gs::Layer{L->wq, L->rq, L->sw, L->sr, static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1, L->N,
+                                l == 0 ? 0 : 1 << 30};
+    g.C = L->N;
+    if (!serq::gs::fits<false>(g, sm_count(), max_smem()))
+      return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "the comparator's decode GEMM does not fit shared memory at M = %d", M);
+    e = accum ? serq::gs::launch<false, true>(g, sm_count(), max_smem(), st)
+              : serq::gs::launch<false, false>(g, sm_count(), max_smem(), st);
+  } else {
+    LinearGroup G = {};
+    G.n = 1;
+    G.L[0] = &q->view;
+    G.Y[0] = static_cast<__nv_bfloat16*>(Y);
+    G.ldy[0] = ldy;
+    G.acc0[0] = acc0;
+    G.acc1[0] = acc1;
+    e = accum ? dispatch_two<true>(G, Xq, sx, M, algo, Zq, nullptr, st) : dispatch_two<false>(G, Xq, sx, M, algo, Zq, sz, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "comparator GEMM launch");
+  return ok();
+}
+
+serq_status check_two_algo(const serq_l2qer* q, int M, serq_algo* algo) {
+  if (!q) return fail(SERQ_ERR_INVALID_ARG, "null comparator");
+  if (M < 1 || M > 65535 * 128) return fail(SERQ_ERR_INVALID_ARG, "M = %d out of range", M);
+  serq_algo a = *algo;
+  if (a == SERQ_ALGO_AUTO) a = (M <= serq_decode_max_m()) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
+  if (a != SERQ_ALGO_DECODE && a != SERQ_ALGO_PREFILL && a != SERQ_ALGO_PREFILL_N128 &&
+      a != SERQ_ALGO_PREFILL_PAIR_N256)
+    return fail(SERQ_ERR_INVALID_ARG, "the comparator runs SERQ_ALGO_AUTO, DECODE, PREFILL, PREFILL_N128 or "
+                                      "PREFILL_PAIR_N256 (got %d)", (int)*algo);
+  if (a == SERQ_ALGO_DECODE && M > 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "decode takes M <= 32 (got %d)", M);
+  serq_status s;
+  if ((s = check_device())) return s;
+  if ((s = check_layer(q->f1))) return s;
+  *algo = a;
+  return SERQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+serq_status serq_l2qer_prepare(const serq_layer* layer, const float* L1, const float* L2, int r, serq_l2qer** out) {
+  if (!out) return fail(SERQ_ERR_INVALID_ARG, "null out");
+  *out = nullptr;
+  if (!layer || !L1 || !L2) return fail(SERQ_ERR_INVALID_ARG, "null layer, L1 or L2");
+  if (layer->mode != SERQ_W4A4) return fail(SERQ_ERR_INVALID_ARG, "the comparator takes W4A4 layers");
+  if (r < 32 || r % 32 || r > layer->K)
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "rank %d must be a positive multiple of 32 and <= K = %d", r, layer->K);
+  serq_status s;
+  if ((s = check_device())) return s;
+  if ((s = check_layer(layer))) return s;
+  serq_l2qer* q = new (std::nothrow) serq_l2qer();
+  if (!q) return fail(SERQ_ERR_ALLOC, "host allocation failed");
+  q->K = layer->K;
+  q->N = layer->N;
+  q->r = r;
+  q->f1 = nullptr;
+  q->block = nullptr;
+  if ((s = alloc_layer(layer->K, r, 0, SERQ_W4A4, &q->f1))) {
+    delete q;
+    return s;
+  }
+  const size_t s_codes = up256((size_t)layer->N * r / 2), s_sc = up256((size_t)layer->N * 4);
+  const int tmpn = layer->K > r ? layer->K : r;
+  const size_t s_tmp = up256((size_t)tmpn * 4);
+  cudaError_t e = cudaMalloc(&q->block, s_codes + s_sc + 2 * s_tmp);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    free_l2qer(q);
+    return fail(SERQ_ERR_ALLOC, "cudaMalloc for the comparator failed: %s", cudaGetErrorString(e));
+  }
+  uint8_t* b = static_cast<uint8_t*>(q->block);
+  uint8_t* l2q = b;
+  float* s_l2 = reinterpret_cast<float*>(b + s_codes);
+  float* ones = reinterpret_cast<float*>(b + s_codes + s_sc);
+  int32_t* ident = reinterpret_cast<int32_t*>(b + s_codes + s_sc + s_tmp);
+  cudaStream_t st;
+  e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    free_l2qer(q);
+    return cuda_fail(e, "cudaStreamCreate");
+  }
+  k_fill_ones_iota<<<(tmpn + 255) / 256, 256, 0, st>>>(ones, ident, tmpn);
+  s = quantize_columns(L1, layer->K, r, q->f1->wq, q->f1->sw, ones, ident, st);
+  if (!s) {
+    cudaMemsetAsync(q->f1->sr, 0, sizeof(float) * r, st);
+    s = quantize_columns(L2, r, layer->N, l2q, s_l2, ones, ident, st);
+  }
+  e = cudaStreamSynchronize(st);
+  cudaStreamDestroy(st);
+  if (!s && e != cudaSuccess) s = cuda_fail(e, "serq_l2qer_prepare");
+  if (s) {
+    free_l2qer(q);
+    return s;
+  }
+  q->view = *layer;
+  q->view.rank = r;
+  q->view.rpad = r;
+  q->view.rq = l2q;
+  q->view.sr = s_l2;
+  if (!build_weight_maps(q->f1) || !build_weight_maps(&q->view)) {
+    free_l2qer(q);
+    return fail(SERQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the comparator");
+  }
+  *out = q;
+  return ok();
+}
+
+void serq_l2qer_destroy(serq_l2qer* q) { free_l2qer(q); }
+
+serq_status serq_l2qer_get_packed(const serq_l2qer* q, uint8_t* l1q, float* s_l1, uint8_t* l2q, float* s_l2) {
+  if (!q) return fail(SERQ_ERR_INVALID_ARG, "null comparator");
+  serq_status s = check_layer(q->f1);
+  if (s) return s;
+  cudaError_t e = cudaSuccess;
+  auto cp = [&](void* dst, const void* src, size_t n) {
+    if (dst && e == cudaSuccess) e = cudaMemcpy(dst, src, n, cudaMemcpyDeviceToHost);
+  };
+  cp(l1q, q->f1->wq, (size_t)q->r * q->K / 2);
+  cp(s_l1, q->f1->sw, sizeof(float) * q->r);
+  cp(l2q, q->view.rq, (size_t)q->N * q->r / 2);
+  cp(s_l2, q->view.sr, sizeof(float) * q->N);
+  if (e != cudaSuccess) return cuda_fail(e, "serq_l2qer_get_packed");
+  return ok();
+}
+
+serq_status serq_l2qer_linear(const serq_l2qer* q, const void* Xq, const float* sx, int M, void* Z, void* Zq,
+                              float* sz, void* Y, int ldy, serq_algo algo, void* stream) {
+  serq_status s;
+  if ((s = check_two_algo(q, M, &algo))) return s;
+  if (!Xq || !sx || !Z || !Zq || !sz || !Y) return fail(SERQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(Z) || !aligned16(Zq) || !aligned16(Y) || (ldy % 8) || ldy < q->N)
+    return fail(SERQ_ERR_INVALID_ARG, "Z, Zq, Y must be 16-byte aligned, ldy >= N and a multiple of 8");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // 1. Z = X_q L1_q (bf16, M x r)
+  const serq_algo a1 = (algo == SERQ_ALGO_DECODE) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
+  if ((s = linear_impl(q->f1, Xq, sx, M, Z, q->r, nullptr, nullptr, a1, stream))) return s;
+  // 2. on-the-fly quantization of the intermediate
+  if ((s = serq_quantize_act(Z, SERQ_BF16, M, q->r, q->r, SERQ_W4A4, Zq, sz, stream))) return s;
+  // 3. X_q W_q + Z_q L2_q
+  return l2qer_final(q, Xq, sx, M, Zq, sz, Y, ldy, nullptr, nullptr, algo, st);
+}
+
+serq_status serq_l2qer_accum(const serq_l2qer* q, const void* Xq, const void* Zq, int M, int32_t* acc0,
+                             int32_t* acc1, serq_algo algo, void* stream) {
+  serq_status s;
+  if ((s = check_two_algo(q, M, &algo))) return s;
+  if (!Xq || !Zq || !acc0 || !acc1) return fail(SERQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(Xq) || !aligned16(acc0) || !aligned16(acc1))
+    return fail(SERQ_ERR_INVALID_ARG, "Xq, acc0, acc1 must be 16-byte aligned");
+  return l2qer_final(q, Xq, nullptr, M, Zq, nullptr, nullptr, 0, acc0, acc1, algo, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

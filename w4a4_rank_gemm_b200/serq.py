@@ -24,15 +24,29 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_UNSUPPORTED_DEVICE, ERR_ALLOC, E
 W4A4, W4A8 = 0, 1
 F32, BF16 = 0, 1
 (ALGO_AUTO, ALGO_PREFILL, ALGO_DECODE, ALGO_PREFILL_N128, ALGO_PREFILL_N256, ALGO_PREFILL_PAIR_N256,
- ALGO_PREFILL_PAIR_TMEM_A, ALGO_DECODE_TC) = 0, 1, 2, 3, 4, 5, 6, 7
+ ALGO_PREFILL_PAIR_TMEM_A, ALGO_DECODE_TC, ALGO_DECODE_ITEMS) = 0, 1, 2, 3, 4, 5, 6, 7, 8
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
+SALIENCY_SCALE, SALIENCY_ROW_ABSMAX = 0, 1
+
+
+class PrepareOpts(ctypes.Structure):
+    """serq_prepare_opts."""
+    _fields_ = [("alpha", ctypes.c_float), ("rank", _i), ("mode", _i), ("saliency", _i),
+                ("out_perm", _vp), ("out_colscale", _vp)]
+
 
 EXPORTS = {
-    "serq_prepare_group": (_i, [_i, ctypes.POINTER(_vp), ctypes.POINTER(_i), _i, _vp, _i, _i, _i,
+    "serq_prepare_opts_init": (None, [ctypes.POINTER(PrepareOpts)]),
+    "serq_prepare_group": (_i, [_i, ctypes.POINTER(_vp), ctypes.POINTER(_i), _i, _vp, _i, ctypes.POINTER(PrepareOpts),
                                 ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
-    "serq_prepare": (_i, [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp, ctypes.POINTER(_vp)]),
+    "serq_prepare_shared": (_i, [_i, ctypes.POINTER(_vp), ctypes.POINTER(_i), _i, _vp, _i,
+                                 ctypes.POINTER(PrepareOpts), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                 ctypes.POINTER(_vp)]),
+    "serq_prepare": (_i, [_vp, _i, _i, _vp, _i, ctypes.POINTER(PrepareOpts), ctypes.POINTER(_vp)]),
+    "serq_layer_get_perm": (_i, [_vp, _vp]),
+    "serq_layer_get_smooth": (_i, [_vp, _vp]),
     "serq_layer_destroy": (None, [_vp]),
     "serq_layer_info": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "serq_layer_perm_smooth": (_i, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
@@ -44,8 +58,14 @@ EXPORTS = {
     "serq_linear_decode_static": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp]),
     "serq_linear_group": (_i, [_i, ctypes.POINTER(_vp), _vp, _vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_i),
                                ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp]),
+    "serq_l2qer_prepare": (_i, [_vp, _vp, _vp, _i, ctypes.POINTER(_vp)]),
+    "serq_l2qer_destroy": (None, [_vp]),
+    "serq_l2qer_get_packed": (_i, [_vp, _vp, _vp, _vp, _vp]),
+    "serq_l2qer_linear": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp]),
+    "serq_l2qer_accum": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp]),
     "serq_silu_mul_quantize": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "serq_flatten_permute": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _i, _vp]),
+    "serq_test_decode_timeout": (_i, [_vp, _vp, _vp, _i, _vp, _i, _i, _vp]),
     "serq_decode_max_m": (_i, []),
     "serq_last_error_string": (ctypes.c_char_p, []),
     "serq_check_device": (_i, []),
@@ -131,10 +151,15 @@ class Layer:
         _check(lib.serq_layer_perm_smooth(self._h, ctypes.byref(p), ctypes.byref(s)), "serq_layer_perm_smooth")
         return p.value, s.value
 
-    def perm_smooth(self) -> Tuple[torch.Tensor, torch.Tensor]:
-        """Device copies of the saliency order (int32[K]) and scales (f32[K])."""
-        d = self.get_packed()
-        return d["perm"], d["smooth"]
+    def perm_smooth(self) -> Tuple["np.ndarray", "np.ndarray"]:
+        """Host copies of the saliency order (int32[K]) and scales (f32[K])
+        (serq_layer_get_perm / serq_layer_get_smooth)."""
+        import numpy as np
+        perm = np.empty(self.K, np.int32)
+        smooth = np.empty(self.K, np.float32)
+        _check(lib.serq_layer_get_perm(self._h, perm.ctypes.data_as(_vp)), "serq_layer_get_perm")
+        _check(lib.serq_layer_get_smooth(self._h, smooth.ctypes.data_as(_vp)), "serq_layer_get_smooth")
+        return perm, smooth
 
     def get_packed(self) -> dict:
         """Host copies of everything prepare produced."""
@@ -153,10 +178,20 @@ class Layer:
                     sw=sw, sr=sr, perm=perm, smooth=smooth)
 
 
+def prepare_opts(rank: int = 128, mode="w4a4", alpha: float = 0.5, saliency: int = SALIENCY_SCALE) -> PrepareOpts:
+    o = PrepareOpts()
+    lib.serq_prepare_opts_init(ctypes.byref(o))
+    o.rank, o.mode, o.alpha, o.saliency = rank, _mode_code(mode), alpha, saliency
+    return o
+
+
 def prepare_group(weights: Sequence[torch.Tensor], X_calib: torch.Tensor, rank: int, mode="w4a4",
                   out_perm: Optional[Sequence[Optional[torch.Tensor]]] = None,
-                  out_div: Optional[Sequence[Optional[torch.Tensor]]] = None) -> List[Layer]:
-    """serq_prepare_group: weights are CUDA fp32 K x N tensors sharing one input."""
+                  out_div: Optional[Sequence[Optional[torch.Tensor]]] = None,
+                  alpha: float = 0.5, saliency: int = SALIENCY_SCALE) -> List[Layer]:
+    """serq_prepare_group: weights are CUDA fp32 K x N tensors sharing one
+    input; out_perm / out_div are the next layer's order and smoothing scales
+    per weight (CUDA tensors or None)."""
     n = len(weights)
     K = weights[0].shape[0]
     for w in weights:
@@ -171,14 +206,72 @@ def prepare_group(weights: Sequence[torch.Tensor], X_calib: torch.Tensor, rank: 
     ps = (_vp * n)(*[(p.data_ptr() if p is not None else None) for p in (out_perm or [None] * n)])
     ds = (_vp * n)(*[(d.data_ptr() if d is not None else None) for d in (out_div or [None] * n)])
     outs = (_vp * n)()
-    _check(lib.serq_prepare_group(n, Ws, Ns, K, _ptr(X_calib), X_calib.shape[0], rank, _mode_code(mode), ps, ds,
-                                  outs), "serq_prepare_group")
+    o = prepare_opts(rank, mode, alpha, saliency)
+    _check(lib.serq_prepare_group(n, Ws, Ns, K, _ptr(X_calib), X_calib.shape[0], ctypes.byref(o), ps, ds, outs),
+           "serq_prepare_group")
     return [Layer(_vp(outs[i])) for i in range(n)]
 
 
 def prepare(W: torch.Tensor, X_calib: torch.Tensor, rank: int, mode="w4a4", out_perm=None,
-            out_div=None) -> Layer:
-    return prepare_group([W], X_calib, rank, mode, [out_perm], [out_div])[0]
+            out_div=None, alpha: float = 0.5, saliency: int = SALIENCY_SCALE) -> Layer:
+    return prepare_group([W], X_calib, rank, mode, [out_perm], [out_div], alpha, saliency)[0]
+
+
+def _host_f32(a, name):
+    import numpy as np
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    if a.ndim not in (1, 2):
+        raise ValueError(f"{name} must be a 1-D or 2-D array")
+    return a
+
+
+def prepare_host(W, X_calib, rank: int = 128, mode="w4a4", alpha: float = 0.5,
+                 saliency: int = SALIENCY_SCALE, out_perm=None, out_colscale=None) -> Layer:
+    """serq_prepare: W (K x N) and X_calib (n x K) are host (numpy) arrays;
+    the library uploads them."""
+    import numpy as np
+    W = _host_f32(W, "W")
+    Xc = _host_f32(X_calib, "X_calib")
+    o = prepare_opts(rank, mode, alpha, saliency)
+    keep = []
+    if out_perm is not None:
+        keep.append(np.ascontiguousarray(out_perm, dtype=np.int32))
+        o.out_perm = keep[-1].ctypes.data
+    if out_colscale is not None:
+        keep.append(np.ascontiguousarray(out_colscale, dtype=np.float32))
+        o.out_colscale = keep[-1].ctypes.data
+    out = _vp()
+    _check(lib.serq_prepare(W.ctypes.data_as(_vp), W.shape[0], W.shape[1], Xc.ctypes.data_as(_vp), Xc.shape[0],
+                            ctypes.byref(o), ctypes.byref(out)), "serq_prepare")
+    return Layer(out)
+
+
+def prepare_shared_host(weights, X_calib, rank: int = 128, mode="w4a4", alpha: float = 0.5,
+                        saliency: int = SALIENCY_SCALE, out_perm=None, out_colscale=None) -> List[Layer]:
+    """serq_prepare_shared: host (numpy) weights sharing one input."""
+    import numpy as np
+    Ws = [_host_f32(w, "W") for w in weights]
+    n = len(Ws)
+    Xc = _host_f32(X_calib, "X_calib")
+    o = prepare_opts(rank, mode, alpha, saliency)
+    keep = list(Ws)
+    def arr(seq, dt):
+        if seq is None:
+            return None
+        ptrs = []
+        for a in seq:
+            if a is None:
+                ptrs.append(None)
+            else:
+                keep.append(np.ascontiguousarray(a, dtype=dt))
+                ptrs.append(keep[-1].ctypes.data)
+        return (_vp * n)(*ptrs)
+    outs = (_vp * n)()
+    _check(lib.serq_prepare_shared(n, (_vp * n)(*[w.ctypes.data for w in Ws]), (_i * n)(*[w.shape[1] for w in Ws]),
+                                   Ws[0].shape[0], Xc.ctypes.data_as(_vp), Xc.shape[0], ctypes.byref(o),
+                                   arr(out_perm, np.int32), arr(out_colscale, np.float32), outs),
+           "serq_prepare_shared")
+    return [Layer(_vp(outs[i])) for i in range(n)]
 
 
 def act_bytes_per_row(K: int, mode) -> int:
@@ -284,6 +377,66 @@ def linear_decode_static(layer: Layer, Xq: torch.Tensor, sx: Optional[torch.Tens
     _check(lib.serq_linear_decode_static(layer.handle, _ptr(Xq), _ptr(sx), M, _ptr(Y), Y.stride(0), None, None,
                                          _stream(stream)), "serq_linear_decode_static")
     return Y
+
+
+class L2QER:
+    """Owner of a two-factor comparator built on a prepared layer."""
+
+    def __init__(self, layer: Layer, L1: torch.Tensor, L2: torch.Tensor):
+        K, r = L1.shape
+        if L2.shape != (r, layer.N) or K != layer.K:
+            raise ValueError("L1 must be K x r and L2 r x N")
+        for t, n in ((L1, "L1"), (L2, "L2")):
+            if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous fp32 CUDA tensor")
+        self.layer, self.K, self.N, self.r = layer, K, layer.N, r
+        h = _vp()
+        _check(lib.serq_l2qer_prepare(layer.handle, _ptr(L1), _ptr(L2), r, ctypes.byref(h)), "serq_l2qer_prepare")
+        self._h = h
+
+    def close(self):
+        if self._h:
+            lib.serq_l2qer_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def get_packed(self) -> dict:
+        import numpy as np
+        l1q = np.empty(self.r * self.K // 2, np.uint8)
+        s1 = np.empty(self.r, np.float32)
+        l2q = np.empty(self.N * self.r // 2, np.uint8)
+        s2 = np.empty(self.N, np.float32)
+        c = lambda a: a.ctypes.data_as(_vp)
+        _check(lib.serq_l2qer_get_packed(self._h, c(l1q), c(s1), c(l2q), c(s2)), "serq_l2qer_get_packed")
+        return dict(l1q=l1q.reshape(self.r, self.K // 2), s_l1=s1, l2q=l2q.reshape(self.N, self.r // 2), s_l2=s2)
+
+    def buffers(self, M: int, device):
+        """Caller-owned intermediate buffers (Z bf16, Zq, sz) for M tokens."""
+        return (torch.empty((M, self.r), dtype=torch.bfloat16, device=device),
+                torch.empty((M, self.r // 2), dtype=torch.uint8, device=device),
+                torch.empty(M, dtype=torch.float32, device=device))
+
+    def linear(self, Xq: torch.Tensor, sx: torch.Tensor, Y=None, bufs=None, algo: int = ALGO_AUTO, stream=None):
+        M = Xq.shape[0]
+        if Y is None:
+            Y = torch.empty((M, self.N), dtype=torch.bfloat16, device=Xq.device)
+        Z, Zq, sz = bufs if bufs is not None else self.buffers(M, Xq.device)
+        _check(lib.serq_l2qer_linear(self._h, _ptr(Xq), _ptr(sx), M, _ptr(Z), _ptr(Zq), _ptr(sz), _ptr(Y),
+                                     Y.stride(0), algo, _stream(stream)), "serq_l2qer_linear")
+        return Y, (Z, Zq, sz)
+
+    def accum(self, Xq: torch.Tensor, Zq: torch.Tensor, algo: int = ALGO_AUTO, stream=None):
+        M = Xq.shape[0]
+        acc0 = torch.empty((M, self.N), dtype=torch.int32, device=Xq.device)
+        acc1 = torch.empty((M, self.N), dtype=torch.int32, device=Xq.device)
+        _check(lib.serq_l2qer_accum(self._h, _ptr(Xq), _ptr(Zq), M, _ptr(acc0), _ptr(acc1), algo, _stream(stream)),
+               "serq_l2qer_accum")
+        return acc0, acc1
 
 
 def device_error() -> int:

@@ -235,3 +235,14 @@ def mlp_block(M: int = 4096, K: int = 4096, F: int = 11008, rank: int = 128,
     xc = inp.X_calib.astype(np.float64)
     h = _silu_f64(xc @ Wg.astype(np.float64)) * (xc @ Wu.astype(np.float64))
     return MLPBlock(M, rank, inp.X, inp.X_calib, Wg, Wu, Wd, h.astype(np.float32))
+
+
+def factor_pair(K: int, N: int, r: int, seed: int = 11, err_std: float = 3e-3):
+    """Two seeded low-rank factors shaped like the scaled-SVD factors of a
+    4-bit weight's quantization error (L1: K x r, entries ~ N(0, 1/K);
+    L2: r x N, entries ~ N(0, err_std^2 K / r)), as inputs of the two-factor
+    comparator's preparation."""
+    rng = np.random.default_rng(seed)
+    L1 = (rng.standard_normal((K, r)) / np.sqrt(K)).astype(np.float32)
+    L2 = (err_std * np.sqrt(K / r) * rng.standard_normal((r, N))).astype(np.float32)
+    return L1, L2
