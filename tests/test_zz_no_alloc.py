@@ -48,3 +48,18 @@ def test_static_scratch_limits(S):
     with pytest.raises(S.SerqError) as e:
         S.linear_decode_static(big, xq_big, sx_big)
     assert e.value.status == 2  # N > 16384
+
+
+def test_static_scratch_after_a_reported_timeout(S):
+    """After serq_device_error has reported a timed-out wait, the next static
+    call clears the scratch again (on its own stream) and is still exact."""
+    L, ol, Xq, sx, xq, osx = _linear_case(S, 8, 1024, 512, 128, "w4a4", seed=13)
+    acc0, acc1 = O.linear_accum(xq, ol)
+    Y = torch.empty((8, 512), dtype=torch.bfloat16, device="cuda")
+    assert S.lib.serq_test_decode_timeout(L.handle, S._ptr(Xq), S._ptr(sx), 8, S._ptr(Y), 512, 1000, None) == S.OK
+    assert S.device_error() == 2
+    for _ in range(2):
+        g0, g1 = S.linear_decode_static(L, Xq, accum=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(g0.cpu().numpy(), acc0) and np.array_equal(g1.cpu().numpy(), acc1)
+    assert S.device_error() == 0
