@@ -3,22 +3,24 @@
 //
 // Work split.  The output channels of the launch (the layers of a group
 // concatenated) are cut into one contiguous range per CTA at a granularity
-// of two channels, so every SM streams the same number of weight bytes
-// (o_proj at 4096 channels: 27 or 28 channels per SM instead of one or two
+// of four channels, so every SM streams the same number of weight bytes
+// (o_proj at 4096 channels: 24 or 28 channels per SM instead of one or two
 // 16-channel items).  Inside a CTA the range is covered by 16-channel tiles
-// (rows past the range are never read and never written) and every tile by
-// "units" of 256 k: 16 rows x 128 bytes of packed weights (2 KB), first the
-// residual's units (R, k < r) and then the main product's.  The CTA's units,
-// tile by tile, are dealt round-robin to its warps.
+// and every tile by "units" of 256 k: 16 rows x 128 bytes of packed weights
+// (2 KB), first the residual's units (R, k < r) and then the main
+// product's.  The CTA's unit list, tile by tile, is cut into one contiguous
+// run per warp, so a warp moves to another tile (and hands its partial sums
+// over) at most a few times.
 //
-// Each warp streams its own units through a private ring of kDepth slots
-// with 16-byte cp.async copies (each lane copies exactly the 64 bytes it
-// will read back, so a lane waits only for its own copies and no barrier is
-// involved); the first kDepth units are requested before the kernel waits
-// for the grid it depends on, since no earlier kernel writes the weights.
-// The activation codes of all tokens are staged once per CTA (one bulk copy
-// per token row, on an mbarrier) at a row pitch that makes every fragment
-// load conflict-free.
+// Each warp streams its run through a private ring of kDepth slots: one
+// lane issues a unit as up to four TMA boxes of 4 rows x 128 bytes (boxes
+// past the CTA's range are skipped; bytes past a row's end are zero-filled)
+// completing on the slot's mbarrier, so the copy engine, not the load/store
+// unit, carries the stream.  The first kDepth units are requested before
+// the kernel waits for the grid it depends on, since no earlier kernel
+// writes the weights.  The activation codes of all tokens and the CTA's
+// sw / sR are staged once per CTA by bulk copies, the codes at a row pitch
+// that makes every fragment load conflict-free.
 //
 // Arithmetic: mma.sync m16n8k32 s8 with the weight rows as the 16-row A
 // operand and the tokens as the 8-column B operand (one n8 tile per eight
@@ -29,15 +31,17 @@
 // activation fragment of the same lane and step covers the same codes, so
 // every product pairs equal k.  Nibbles are widened to int8 x16 by two mask
 // operations (INT8 activations are used as they are), hence the final
-// shift by 8 (W4A4) or 4 (W4A8).  The residual units accumulate
-// X~_{s,q} Q(R) into a second accumulator from the same activation codes
-// (SERQ notes, key design 2: one matmul on the salient channels).
+// shift by 8 (W4A4) or 4 (W4A8).  Codes past K (or r) meet zero-filled
+// weights, so the staged activation rows need no padding of their own.  The
+// residual units accumulate X~_{s,q} Q(R) into a second accumulator from
+// the same activation codes (SERQ notes, key design 2: one matmul on the
+// salient channels).
 //
 // A warp adds its partial sums of a tile into the tile's shared
-// accumulators whenever it moves on to another tile, then adds the number
-// of units it covered to the tile's counter; the warp that completes the
-// count applies the epilogue sx * (sw * acc0 + sR * acc1) for the tile's
-// channels and every token.  No warp waits for another.
+// accumulators when it moves on to another tile, then adds the number of
+// units it covered to the tile's counter; the warp that completes the count
+// applies the epilogue sx * (sw * acc0 + sR * acc1) for the tile's channels
+// and every token.  No warp waits for another.
 #pragma once
 #include "common.cuh"
 
@@ -47,7 +51,12 @@ namespace gs {
 constexpr int kDepth = 4;         // ring slots per warp
 constexpr int kUnitK = 256;       // k per unit
 constexpr int kUnitBytes = 2048;  // 16 rows x 128 bytes
-constexpr int kMaxWarps = 16;
+constexpr int kBoxRows = 4;       // rows per TMA box (the channel granularity of the CTA ranges)
+constexpr int kBoxBytes = kBoxRows * 128;
+#ifndef SERQ_GS_WARPS
+#define SERQ_GS_WARPS 16
+#endif
+constexpr int kMaxWarps = SERQ_GS_WARPS;  // warps per CTA when shared memory allows
 constexpr int kMaxGroup = 4;
 constexpr int kMaxTokenTiles = 4;  // n8 tiles: M <= 32
 
@@ -78,6 +87,13 @@ struct Args {
   Layer lo[kMaxGroup];
 };
 
+// Per layer: the weight and the compensator as 2-D byte tensors (rows =
+// output channels) read in 128-byte x 4-row boxes.
+struct Maps {
+  CUtensorMap w[kMaxGroup];
+  CUtensorMap r[kMaxGroup];
+};
+
 // Computed on the host.
 struct Plan {
   int warps;       // warps per CTA
@@ -89,6 +105,7 @@ struct Plan {
   int units_main;  // 256-k units of W per tile
   int units_res;   // 256-k units of R per tile
   int tmax;        // most tiles one CTA covers
+  int cmax;        // most channels one CTA covers
   int smem;        // dynamic shared memory bytes
   // Failure-detection test only (zero in every other launch): the activation
   // copies are not issued, so the bounded wait for them runs out after
@@ -103,7 +120,7 @@ struct AccLayout {
 };
 
 __host__ __device__ inline int chan_begin(int c, int C, int grid) {
-  return 2 * (int)(((long long)c * (C >> 1)) / grid);
+  return kBoxRows * (int)(((long long)c * (C / kBoxRows)) / grid);
 }
 
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -121,11 +138,10 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// Generic-proxy reads of shared memory before async-proxy (TMA) writes to it.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 __device__ __forceinline__ int layer_of(const Args& p, int ch) {
   int l = 0;
@@ -135,40 +151,45 @@ __device__ __forceinline__ int layer_of(const Args& p, int ch) {
   return l;
 }
 
-// Requests unit v of this CTA into ring slot `slot` (this lane's 4 pieces).
-__device__ __forceinline__ void issue_unit(const Args& p, const Plan& pl, uint8_t* slot_base, int c0, int c1,
-                                           int v, int g, int t, int lane) {
-  const int ut = pl.units_res + pl.units_main;
-  const int tile = v / ut, ku = v - tile * ut;
-  const bool res = ku < pl.units_res;
-  const int kunit = res ? ku : ku - pl.units_res;
-  const int rowbytes = res ? (p.rpad >> 1) : (p.K >> 1);
-#pragma unroll
-  for (int hs = 0; hs < 2; ++hs) {
-    const int ch = c0 + tile * 16 + g + 8 * hs;
-    const uint8_t* src = p.lo[0].Wq;
-    bool row_ok = ch < c1;
-    if (row_ok) {
-      const Layer& lo = p.lo[layer_of(p, ch)];
-      src = (res ? lo.Rq : lo.Wq) + (size_t)(ch - lo.base) * rowbytes;
+// A warp's position in its CTA's unit list (tile-major; within a tile the
+// residual units come first).
+struct Cursor {
+  int tile, ku;
+  __device__ __forceinline__ void next(int ut) {
+    if (++ku == ut) {
+      ku = 0;
+      ++tile;
     }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int kb = (kunit * 2 + h) * 64 + 16 * t;
-      const bool ok = row_ok && kb < rowbytes;
-      cp_async16_zfill(slot_base + (h * 2 + hs) * 512 + lane * 16, ok ? src + kb : p.lo[0].Wq, ok ? 16u : 0u);
-    }
+  }
+};
+
+// Issues the unit at cursor c into `slot` (called by one lane): up to four
+// 4-row boxes, skipping those past the CTA's range, all completing on bar.
+__device__ __forceinline__ void issue_unit(const Args& p, const Maps& mp, const Plan& pl, uint8_t* slot,
+                                           uint64_t* bar, const Cursor& c, int c0, int c1) {
+  const bool res = c.ku < pl.units_res;
+  const int x = (res ? c.ku : c.ku - pl.units_res) * 128;
+  const int r0 = c0 + c.tile * 16;
+  const int nbox = min(4, (c1 - r0) / kBoxRows);
+  mbar_arrive_expect_tx(bar, (uint32_t)(nbox * kBoxBytes));
+  for (int b = 0; b < nbox; ++b) {
+    const int ch = r0 + b * kBoxRows;
+    const int l = layer_of(p, ch);
+    tma_load_2d(slot + b * kBoxBytes, res ? &mp.r[l] : &mp.w[l], bar, x, ch - p.lo[l].base);
   }
 }
 
-// The MMAs of one unit: w = this lane's pieces [chunk h][row g / g + 8].
+// The MMAs of one unit.  The slot holds 16 rows x 128 bytes; lane (g, t)
+// reads rows g and g + 8 at run t of each 128-k chunk.
 template <int NTT, bool A8>
-__device__ __forceinline__ void unit_mma(const uint4 (&w)[4], const uint8_t* xs, int xpitch, int xc0, int nch,
-                                         int g, int t, int (&acc)[NTT][4]) {
+__device__ __forceinline__ void unit_mma(const uint8_t* slot, const uint8_t* xs, int xpitch, int xc0, int nch, int g,
+                                         int t, int (&acc)[NTT][4]) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     if (h < nch) {
       const int xc = xc0 + h;
+      const uint4 wg = *reinterpret_cast<const uint4*>(slot + g * 128 + h * 64 + 16 * t);
+      const uint4 wg8 = *reinterpret_cast<const uint4*>(slot + (g + 8) * 128 + h * 64 + 16 * t);
       uint4 xa[NTT], xb[NTT];
 #pragma unroll
       for (int nt = 0; nt < NTT; ++nt) {
@@ -183,7 +204,7 @@ __device__ __forceinline__ void unit_mma(const uint4 (&w)[4], const uint8_t* xs,
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t u = word(w[h * 2 + 0], i), v = word(w[h * 2 + 1], i);
+        const uint32_t u = word(wg, i), v = word(wg8, i);
         const uint32_t a0 = lo_x16(u), a1 = lo_x16(v), a2 = hi_x16(u), a3 = hi_x16(v);
 #pragma unroll
         for (int nt = 0; nt < NTT; ++nt) {
@@ -204,7 +225,7 @@ __device__ __forceinline__ void unit_mma(const uint4 (&w)[4], const uint8_t* xs,
 
 // Epilogue of one tile by one warp: every (token, channel) of the tile.
 // The scales come from shared memory: ssw / ssr hold sw and sR of the CTA's
-// channels (staged at the start), ssx / ssxr the tokens' scales.
+// channels, ssx / ssxr the tokens' scales.
 template <int NTT, bool A8, bool ACC>
 __device__ __forceinline__ void tile_epilogue(const Args& p, const int* acc, int ch0, int c0, int c1,
                                               const float* ssw, const float* ssr, const float* ssx,
@@ -234,19 +255,21 @@ __device__ __forceinline__ void tile_epilogue(const Args& p, const int* acc, int
 }
 
 template <int NTT, bool A8, bool ACC>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv(const __grid_constant__ Args p, const Plan pl) {
+__global__ void __launch_bounds__(kMaxWarps * 32, 1)
+    k_gemv(const __grid_constant__ Args p, const __grid_constant__ Maps mp, const Plan pl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  uint8_t* xs = sm;                                                  // [xrows][xpitch]
-  uint8_t* xr = xs + pl.xrows * pl.xpitch;                           // [xrows][xrpitch] (comparator only)
-  uint8_t* ring = xr + pl.xrows * pl.xrpitch;                        // [warp][slot][4 pieces][32 lanes][16 B]
-  int* acc = reinterpret_cast<int*>(ring + pl.warps * kDepth * kUnitBytes);  // [tile][AccLayout]
-  int* cnt = acc + pl.tmax * AccLayout<NTT>::kInts;                  // [tile] units added
-  float* ssw = reinterpret_cast<float*>(cnt + ((pl.tmax + 1) & ~1));  // [tmax * 16] sw of the CTA's channels
-  float* ssr = ssw + pl.tmax * 16;                                   // [tmax * 16] sR
-  float* ssx = ssr + pl.tmax * 16;                                   // [xrows] sx
-  float* ssxr = ssx + pl.xrows;                                      // [xrows] residual scale (comparator)
-  uint64_t* xbar = reinterpret_cast<uint64_t*>(ssxr + pl.xrows);
+  uint8_t* ring = sm;                                                 // [warp][slot][16 rows][128 B]
+  uint8_t* xs = ring + pl.warps * kDepth * kUnitBytes;                // [xrows][xpitch]
+  uint8_t* xr = xs + pl.xrows * pl.xpitch;                            // [xrows][xrpitch] (comparator only)
+  int* acc = reinterpret_cast<int*>(xr + pl.xrows * pl.xrpitch);      // [tile][AccLayout]
+  int* cnt = acc + pl.tmax * AccLayout<NTT>::kInts;                   // [tile] units added
+  float* ssw = reinterpret_cast<float*>(cnt + ((pl.tmax + 3) & ~3));  // [cmax] sw of the CTA's channels
+  float* ssr = ssw + pl.cmax;                                         // [cmax] sR
+  float* ssx = ssr + pl.cmax;                                         // [xrows] sx
+  float* ssxr = ssx + pl.xrows;                                       // [xrows] residual scale (comparator)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ssxr + pl.xrows);      // [warp][slot] unit landed
+  uint64_t* xbar = bars + pl.warps * kDepth;                          // activations and scales landed
   volatile int* abort_flag = reinterpret_cast<volatile int*>(xbar + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -255,54 +278,54 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv(const __grid_constan
   const int tiles = (c1 - c0 + 15) >> 4;
   const int ut = pl.units_res + pl.units_main;
   const int units = tiles * ut;
-  const int nw = (warp < units) ? (units - warp + pl.warps - 1) / pl.warps : 0;  // this warp's units
+  // this warp's contiguous run of the CTA's units
+  const int u0 = (int)(((long long)units * warp) / pl.warps);
+  const int nw = (int)(((long long)units * (warp + 1)) / pl.warps) - u0;
   uint8_t* my_ring = ring + warp * kDepth * kUnitBytes;
+  uint64_t* my_bars = bars + warp * kDepth;
 
-  // Weights first: no earlier kernel writes them.
-#pragma unroll
-  for (int s = 0; s < kDepth; ++s) {
-    if (s < nw) issue_unit(p, pl, my_ring + s * kUnitBytes, c0, c1, warp + s * pl.warps, g, t, lane);
-    cp_async_commit();
-  }
-
-  // Shared accumulators, counters, the activation rows' zero padding.
-  for (int i = threadIdx.x; i < tiles * AccLayout<NTT>::kInts; i += blockDim.x) acc[i] = 0;
-  for (int i = threadIdx.x; i < tiles; i += blockDim.x) cnt[i] = 0;
-  if (!ACC) {
-    // sw and sR of this CTA's channels (static data: read before the wait)
-    for (int i = threadIdx.x; i < c1 - c0; i += blockDim.x) {
-      const Layer& lo = p.lo[layer_of(p, c0 + i)];
-      ssw[i] = __ldg(lo.sw + (c0 + i - lo.base));
-      ssr[i] = __ldg(lo.sr + (c0 + i - lo.base));
+  if (lane == 0) {
+    for (int s = 0; s < kDepth; ++s) mbar_init(&my_bars[s], 1);
+    if (warp == 0) {
+      mbar_init(xbar, 1);
+      *abort_flag = 0;
     }
-  }
-  {
-    const int tail = pl.xpitch - pl.xbytes;  // bytes after each copied row
-    const int words_row = pl.xpitch >> 2;
-    for (int i = threadIdx.x; i < pl.xrows * words_row; i += blockDim.x) {
-      const int m = i / words_row, b = (i - m * words_row) * 4;
-      if (m >= p.M || b >= pl.xpitch - tail) reinterpret_cast<uint32_t*>(xs)[i] = 0u;
-    }
-    const int rbytes = p.rpad >> 1, words_r = pl.xrpitch >> 2;
-    for (int i = threadIdx.x; i < pl.xrows * words_r; i += blockDim.x) {
-      const int m = i / words_r, b = (i - m * words_r) * 4;
-      if (m >= p.M || b >= rbytes) reinterpret_cast<uint32_t*>(xr)[i] = 0u;
-    }
-  }
-  if (threadIdx.x == 0) {
-    mbar_init(xbar, 1);
-    *abort_flag = 0;
     fence_mbar_init();
   }
-  __syncthreads();
+  __syncwarp();
+  // Weights first: no earlier kernel writes them.  The issue cursor runs
+  // kDepth units ahead of the compute cursor.
+  Cursor ic{u0 / ut, u0 % ut};
+  if (lane == 0) {
+    for (int s = 0; s < kDepth && s < nw; ++s) {
+      issue_unit(p, mp, pl, my_ring + s * kUnitBytes, &my_bars[s], ic, c0, c1);
+      ic.next(ut);
+    }
+  }
+  // Shared accumulators and counters.
+  for (int i = threadIdx.x; i < tiles * AccLayout<NTT>::kInts; i += blockDim.x) acc[i] = 0;
+  for (int i = threadIdx.x; i < tiles; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();    // barriers initialised, accumulators zero
   grid_dep_launch();  // the next kernel in the stream may be scheduled
   grid_dep_wait();    // activations, sx and the outputs come after the grid this one depends on
   if (threadIdx.x == 0 && !pl.withhold_x) {
     const uint32_t rbytes = (uint32_t)(p.rpad >> 1);
-    mbar_arrive_expect_tx(xbar, (uint32_t)(p.M * pl.xbytes) + (pl.xrpitch ? (uint32_t)p.M * rbytes : 0u));
+    uint32_t tx = (uint32_t)(p.M * pl.xbytes) + (pl.xrpitch ? (uint32_t)p.M * rbytes : 0u);
+    if (!ACC) tx += 8u * (uint32_t)(c1 - c0);
+    mbar_arrive_expect_tx(xbar, tx);
     for (int m = 0; m < p.M; ++m) bulk_load(xs + m * pl.xpitch, p.Xq + (size_t)m * pl.xbytes, pl.xbytes, xbar);
     if (pl.xrpitch)
       for (int m = 0; m < p.M; ++m) bulk_load(xr + m * pl.xrpitch, p.Xr + (size_t)m * rbytes, rbytes, xbar);
+    if (!ACC) {
+      // sw and sR of the CTA's channels, one piece per layer they touch
+      // (channel ranges and layer bases are multiples of 4: 16-byte pieces)
+      for (int l = 0; l < p.nlayers; ++l) {
+        const int a = max(c0, p.lo[l].base), b = min(c1, p.lo[l].base + p.lo[l].N);
+        if (a >= b) continue;
+        bulk_load(ssw + (a - c0), p.lo[l].sw + (a - p.lo[l].base), 4u * (uint32_t)(b - a), xbar);
+        bulk_load(ssr + (a - c0), p.lo[l].sr + (a - p.lo[l].base), 4u * (uint32_t)(b - a), xbar);
+      }
+    }
   }
   if (!ACC) {
     for (int i = threadIdx.x; i < p.M; i += blockDim.x) {
@@ -348,48 +371,49 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) k_gemv(const __grid_constan
       had0 = had1 = false;
     };
 
-    for (int j = 0; j < nw; ++j) {
-      const int v = warp + j * pl.warps;
-      const int tile = v / ut, ku = v - tile * ut;
-      if (tile != cur) {
+    Cursor cc{u0 / ut, u0 % ut};
+    bool live = true;
+    for (int j = 0; j < nw; ++j, cc.next(ut)) {
+      if (cc.tile != cur) {
         if (cur >= 0) flush();
-        cur = tile;
+        cur = cc.tile;
       }
-      cp_async_wait_group<kDepth - 1>();  // this lane's copies of unit j have landed
-      const uint8_t* slot = my_ring + (j % kDepth) * kUnitBytes;
-      uint4 w[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) w[q] = *reinterpret_cast<const uint4*>(slot + q * 512 + lane * 16);
-      __syncwarp();  // orders this lane's reads of the slot before its refill
-      if (j + kDepth < nw)
-        issue_unit(p, pl, my_ring + (j % kDepth) * kUnitBytes, c0, c1, v + kDepth * pl.warps, g, t, lane);
-      cp_async_commit();
-      const bool res = ku < pl.units_res;
-      const int kunit = res ? ku : ku - pl.units_res;
+      const int s = j % kDepth;
+      if (!mbar_wait(&my_bars[s], (uint32_t)(j / kDepth) & 1u, abort_flag, kDevTimeoutUnpack)) {
+        live = false;
+        break;
+      }
+      const uint8_t* slot = my_ring + s * kUnitBytes;
+      const bool res = cc.ku < pl.units_res;
+      const int kunit = res ? cc.ku : cc.ku - pl.units_res;
       const int left = (res ? kl_res : kl_main) - kunit * kUnitK;
       const int nch = left >= 256 ? 2 : (left + 127) >> 7;
       if (res) {
         if (pl.xrpitch)
-          unit_mma<NTT, A8>(w, xr, pl.xrpitch, kunit * 2, nch, g, t, acc1);
+          unit_mma<NTT, A8>(slot, xr, pl.xrpitch, kunit * 2, nch, g, t, acc1);
         else
-          unit_mma<NTT, A8>(w, xs, pl.xpitch, kunit * 2, nch, g, t, acc1);
+          unit_mma<NTT, A8>(slot, xs, pl.xpitch, kunit * 2, nch, g, t, acc1);
         had1 = true;
       } else {
-        unit_mma<NTT, A8>(w, xs, pl.xpitch, kunit * 2, nch, g, t, acc0);
+        unit_mma<NTT, A8>(slot, xs, pl.xpitch, kunit * 2, nch, g, t, acc0);
         had0 = true;
       }
       ++cur_units;
-    }
-    if (cur >= 0) flush();
-  }
-  cp_async_wait_all();
-  __syncthreads();
-  if (*abort_flag) {
-    if (threadIdx.x == 0) {
-      // let the activation copies already issued land before shared memory is released
-      const unsigned long long t0 = global_ns();
-      while (global_ns() - t0 < 100000ull) {
+      // refill this slot with the unit kDepth ahead once every lane has read it
+      __syncwarp();
+      if (j + kDepth < nw && lane == 0) {
+        fence_proxy_async_shared();
+        issue_unit(p, mp, pl, my_ring + s * kUnitBytes, &my_bars[s], ic, c0, c1);
+        ic.next(ut);
       }
+    }
+    if (live && cur >= 0) flush();
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // let the copies already issued land before shared memory is released
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < 100000ull) {
     }
   }
 }
@@ -401,7 +425,7 @@ inline bool make_plan(const Args& p, int sms, int max_smem, Plan& pl) {
   pl.xbytes = A8 ? p.K : p.K / 2;
   pl.units_main = (p.K + kUnitK - 1) / kUnitK;
   pl.units_res = (p.rpad + kUnitK - 1) / kUnitK;
-  const int xrow = pl.units_main * (A8 ? 256 : 128);  // whole units, zero past K
+  const int xrow = pl.units_main * (A8 ? 256 : 128);  // whole units (bytes past K meet zero weights)
   pl.xpitch = xrow + (A8 ? 16 : 64);                   // rows g, g + 1 in opposite bank halves
   pl.xrows = 8 * NTT;
   // comparator's residual codes: whole units, rows g, g + 1 in opposite bank halves
@@ -415,11 +439,12 @@ inline bool make_plan(const Args& p, int sms, int max_smem, Plan& pl) {
     const int n = chan_begin(c + 1, p.C, grid) - chan_begin(c, p.C, grid);
     if (n > most) most = n;
   }
+  pl.cmax = most;
   pl.tmax = (most + 15) / 16;
   const int fixed = 128 + pl.xrows * (pl.xpitch + pl.xrpitch) + pl.tmax * AccLayout<NTT>::kInts * 4 +
-                    ((pl.tmax + 1) & ~1) * 4 + pl.tmax * 16 * 8 + pl.xrows * 8 + 16;
+                    ((pl.tmax + 3) & ~3) * 4 + pl.cmax * 8 + pl.xrows * 8 + 8 + 16;
   for (int w = kMaxWarps; w >= 4; w -= 4) {
-    const int bytes = fixed + w * kDepth * kUnitBytes;
+    const int bytes = fixed + w * (kDepth * kUnitBytes + kDepth * 8);
     if (bytes <= max_smem) {
       pl.warps = w;
       pl.smem = bytes;
@@ -430,8 +455,9 @@ inline bool make_plan(const Args& p, int sms, int max_smem, Plan& pl) {
 }
 
 template <int NTT, bool A8, bool ACC>
-inline cudaError_t launch_ntt(const Args& p, int sms, int max_smem, cudaStream_t st, unsigned long long fault_wait_ns) {
-  Plan pl;
+inline cudaError_t launch_ntt(const Args& p, const Maps& mp, int sms, int max_smem, cudaStream_t st,
+                              unsigned long long fault_wait_ns) {
+  Plan pl = {};
   if (!make_plan<NTT, A8>(p, sms, max_smem, pl)) return cudaErrorInvalidValue;
   pl.withhold_x = fault_wait_ns ? 1 : 0;
   pl.wait_ns = fault_wait_ns;
@@ -448,7 +474,7 @@ inline cudaError_t launch_ntt(const Args& p, int sms, int max_smem, cudaStream_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p, pl);
+  return cudaLaunchKernelEx(&cfg, kern, p, mp, pl);
 }
 
 // Whether the streaming kernel takes this launch (else the caller uses the
@@ -468,13 +494,14 @@ inline bool fits(const Args& p, int sms, int max_smem) {
 // fault_wait_ns: zero, or (failure-detection test) withhold the activation
 // copies and give the wait for them this limit.
 template <bool A8, bool ACC>
-inline cudaError_t launch(const Args& p, int sms, int max_smem, cudaStream_t st, unsigned long long fault_wait_ns = 0) {
+inline cudaError_t launch(const Args& p, const Maps& mp, int sms, int max_smem, cudaStream_t st,
+                          unsigned long long fault_wait_ns = 0) {
   const int ntt = (p.M + 7) / 8;
   switch (ntt) {
-    case 1: return launch_ntt<1, A8, ACC>(p, sms, max_smem, st, fault_wait_ns);
-    case 2: return launch_ntt<2, A8, ACC>(p, sms, max_smem, st, fault_wait_ns);
+    case 1: return launch_ntt<1, A8, ACC>(p, mp, sms, max_smem, st, fault_wait_ns);
+    case 2: return launch_ntt<2, A8, ACC>(p, mp, sms, max_smem, st, fault_wait_ns);
     case 3:
-    case 4: return launch_ntt<4, A8, ACC>(p, sms, max_smem, st, fault_wait_ns);
+    case 4: return launch_ntt<4, A8, ACC>(p, mp, sms, max_smem, st, fault_wait_ns);
     default: return cudaErrorInvalidValue;
   }
 }

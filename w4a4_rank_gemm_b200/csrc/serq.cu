@@ -107,6 +107,7 @@ struct serq_layer {
   float* smooth;
   CUtensorMap tmB[3];  // box rows 128, 256, 96
   CUtensorMap tmR[3];
+  CUtensorMap tmW4, tmR4;  // 128-byte x 4-row boxes (streaming decode kernel)
   int32_t* ws;         // split-K partial sums of the tensor-core decode, zero between calls
   int32_t* cnt;        // per 128-row tile: units done
 };
@@ -182,6 +183,16 @@ bool build_weight_maps(serq_layer* L) {
     } else {
       L->tmR[i] = L->tmB[i];  // never read when r = 0
     }
+  }
+  if (!make_map(&L->tmW4, L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 128, 4,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  if (L->rpad) {
+    if (!make_map(&L->tmR4, L->rq, (uint64_t)L->rpad / 2, (uint64_t)L->N, (uint64_t)L->rpad / 2, 128, 4,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  } else {
+    L->tmR4 = L->tmW4;  // never read when r = 0
   }
   return true;
 }
@@ -415,6 +426,7 @@ cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const floa
                                 bool items, cudaStream_t st, unsigned long long fault_wait_ns = 0) {
   if (!items) {
     serq::gs::Args g = {};
+    serq::gs::Maps mp;
     g.Xq = static_cast<const uint8_t*>(Xq);
     g.sx = sx;
     g.M = M;
@@ -427,16 +439,18 @@ cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const floa
       const serq_layer* L = G.L[li];
       g.lo[l] = serq::gs::Layer{L->wq, L->rq, L->sw, L->sr, G.Y[li], G.ldy[li], G.acc0[li], G.acc1[li], L->N,
                                 l < G.n ? base : 1 << 30};
+      mp.w[l] = L->tmW4;
+      mp.r[l] = L->tmR4;
       if (l < G.n) base += L->N;
     }
     g.C = base;
     const bool fit = a8 ? serq::gs::fits<true>(g, sm_count(), max_smem()) : serq::gs::fits<false>(g, sm_count(), max_smem());
     if (fit) {
       if (a8)
-        return accum ? serq::gs::launch<true, true>(g, sm_count(), max_smem(), st, fault_wait_ns)
-                     : serq::gs::launch<true, false>(g, sm_count(), max_smem(), st, fault_wait_ns);
-      return accum ? serq::gs::launch<false, true>(g, sm_count(), max_smem(), st, fault_wait_ns)
-                   : serq::gs::launch<false, false>(g, sm_count(), max_smem(), st, fault_wait_ns);
+        return accum ? serq::gs::launch<true, true>(g, mp, sm_count(), max_smem(), st, fault_wait_ns)
+                     : serq::gs::launch<true, false>(g, mp, sm_count(), max_smem(), st, fault_wait_ns);
+      return accum ? serq::gs::launch<false, true>(g, mp, sm_count(), max_smem(), st, fault_wait_ns)
+                   : serq::gs::launch<false, false>(g, mp, sm_count(), max_smem(), st, fault_wait_ns);
     }
     if (fault_wait_ns) return cudaErrorInvalidValue;
   }
@@ -1145,14 +1159,18 @@ serq_status l2qer_final(const serq_l2qer* q, const void* Xq, const float* sx, in
     g.rpad = q->view.rpad;
     g.nlayers = 1;
     const serq_layer* L = &q->view;
-    for (int l = 0; l < serq::gs::kMaxGroup; ++l)
+    serq::gs::Maps mp;
+    for (int l = 0; l < serq::gs::kMaxGroup; ++l) {
       g.lo[l] = serq::gs::Layer{L->wq, L->rq, L->sw, L->sr, static_cast<__nv_bfloat16*>(Y), ldy, acc0, acc1, L->N,
                                 l == 0 ? 0 : 1 << 30};
+      mp.w[l] = L->tmW4;
+      mp.r[l] = L->tmR4;
+    }
     g.C = L->N;
     if (!serq::gs::fits<false>(g, sm_count(), max_smem()))
       return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "the comparator's decode GEMM does not fit shared memory at M = %d", M);
-    e = accum ? serq::gs::launch<false, true>(g, sm_count(), max_smem(), st)
-              : serq::gs::launch<false, false>(g, sm_count(), max_smem(), st);
+    e = accum ? serq::gs::launch<false, true>(g, mp, sm_count(), max_smem(), st)
+              : serq::gs::launch<false, false>(g, mp, sm_count(), max_smem(), st);
   } else {
     LinearGroup G = {};
     G.n = 1;
