@@ -88,10 +88,14 @@ struct Args {
 };
 
 // Per layer: the weight and the compensator as 2-D byte tensors (rows =
-// output channels) read in 128-byte x 4-row boxes.
+// output channels) read in 128-byte x 16-row boxes (a whole unit) and in
+// 128-byte x 4-row boxes (the last, partial tile of a CTA's range, or a
+// tile across a layer boundary).
 struct Maps {
   CUtensorMap w[kMaxGroup];
   CUtensorMap r[kMaxGroup];
+  CUtensorMap w16[kMaxGroup];
+  CUtensorMap r16[kMaxGroup];
 };
 
 // Computed on the host.
@@ -163,13 +167,20 @@ struct Cursor {
   }
 };
 
-// Issues the unit at cursor c into `slot` (called by one lane): up to four
-// 4-row boxes, skipping those past the CTA's range, all completing on bar.
+// Issues the unit at cursor c into `slot` (called by one lane), completing
+// on bar: one 16-row box when the tile lies within the CTA's range and one
+// layer, else 4-row boxes up to the end of the range.
 __device__ __forceinline__ void issue_unit(const Args& p, const Maps& mp, const Plan& pl, uint8_t* slot,
                                            uint64_t* bar, const Cursor& c, int c0, int c1) {
   const bool res = c.ku < pl.units_res;
   const int x = (res ? c.ku : c.ku - pl.units_res) * 128;
   const int r0 = c0 + c.tile * 16;
+  const int l0 = layer_of(p, r0);
+  if (r0 + 16 <= c1 && r0 + 16 <= p.lo[l0].base + p.lo[l0].N) {
+    mbar_arrive_expect_tx(bar, (uint32_t)kUnitBytes);
+    tma_load_2d(slot, res ? &mp.r16[l0] : &mp.w16[l0], bar, x, r0 - p.lo[l0].base);
+    return;
+  }
   const int nbox = min(4, (c1 - r0) / kBoxRows);
   mbar_arrive_expect_tx(bar, (uint32_t)(nbox * kBoxBytes));
   for (int b = 0; b < nbox; ++b) {
@@ -291,6 +302,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       *abort_flag = 0;
     }
     fence_mbar_init();
+  } else if (warp == 0 && lane <= p.nlayers * 4) {
+    // descriptors of the layers' maps into the TMA unit's cache
+    const int l = (lane - 1) >> 2, k = (lane - 1) & 3;
+    tma_prefetch_desc(k == 0 ? &mp.w16[l] : k == 1 ? &mp.r16[l] : k == 2 ? &mp.w[l] : &mp.r[l]);
   }
   __syncwarp();
   // Weights first: no earlier kernel writes them.  The issue cursor runs

@@ -107,7 +107,8 @@ struct serq_layer {
   float* smooth;
   CUtensorMap tmB[3];  // box rows 128, 256, 96
   CUtensorMap tmR[3];
-  CUtensorMap tmW4, tmR4;  // 128-byte x 4-row boxes (streaming decode kernel)
+  CUtensorMap tmW4, tmR4;    // 128-byte x 4-row boxes (streaming decode kernel)
+  CUtensorMap tmW16, tmR16;  // 128-byte x 16-row boxes (streaming decode kernel)
   int32_t* ws;         // split-K partial sums of the tensor-core decode, zero between calls
   int32_t* cnt;        // per 128-row tile: units done
 };
@@ -185,14 +186,19 @@ bool build_weight_maps(serq_layer* L) {
     }
   }
   if (!make_map(&L->tmW4, L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 128, 4,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&L->tmW16, L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 128, 16,
                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   if (L->rpad) {
     if (!make_map(&L->tmR4, L->rq, (uint64_t)L->rpad / 2, (uint64_t)L->N, (uint64_t)L->rpad / 2, 128, 4,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&L->tmR16, L->rq, (uint64_t)L->rpad / 2, (uint64_t)L->N, (uint64_t)L->rpad / 2, 128, 16,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
       return false;
   } else {
     L->tmR4 = L->tmW4;  // never read when r = 0
+    L->tmR16 = L->tmW16;
   }
   return true;
 }
@@ -441,6 +447,8 @@ cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const floa
                                 l < G.n ? base : 1 << 30};
       mp.w[l] = L->tmW4;
       mp.r[l] = L->tmR4;
+      mp.w16[l] = L->tmW16;
+      mp.r16[l] = L->tmR16;
       if (l < G.n) base += L->N;
     }
     g.C = base;
@@ -1165,6 +1173,8 @@ serq_status l2qer_final(const serq_l2qer* q, const void* Xq, const float* sx, in
                                 l == 0 ? 0 : 1 << 30};
       mp.w[l] = L->tmW4;
       mp.r[l] = L->tmR4;
+      mp.w16[l] = L->tmW16;
+      mp.r16[l] = L->tmR16;
     }
     g.C = L->N;
     if (!serq::gs::fits<false>(g, sm_count(), max_smem()))
