@@ -123,8 +123,9 @@ struct AccLayout {
   static constexpr int kInts = 2 * NTT * 4 * 32;  // [acc0 / acc1][token tile][fragment q][lane]
 };
 
+// c * (C / 4) stays below 2^31 for grid <= 1024 and C <= 2^21.
 __host__ __device__ inline int chan_begin(int c, int C, int grid) {
-  return kBoxRows * (int)(((long long)c * (C / kBoxRows)) / grid);
+  return kBoxRows * ((c * (C / kBoxRows)) / grid);
 }
 
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -290,8 +291,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   const int ut = pl.units_res + pl.units_main;
   const int units = tiles * ut;
   // this warp's contiguous run of the CTA's units
-  const int u0 = (int)(((long long)units * warp) / pl.warps);
-  const int nw = (int)(((long long)units * (warp + 1)) / pl.warps) - u0;
+  const int u0 = (units * warp) / pl.warps;
+  const int nw = (units * (warp + 1)) / pl.warps - u0;
   uint8_t* my_ring = ring + warp * kDepth * kUnitBytes;
   uint64_t* my_bars = bars + warp * kDepth;
 
@@ -317,23 +318,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       ic.next(ut);
     }
   }
-  // Shared accumulators and counters.
-  for (int i = threadIdx.x; i < tiles * AccLayout<NTT>::kInts; i += blockDim.x) acc[i] = 0;
-  for (int i = threadIdx.x; i < tiles; i += blockDim.x) cnt[i] = 0;
-  __syncthreads();    // barriers initialised, accumulators zero
-  grid_dep_launch();  // the next kernel in the stream may be scheduled
-  grid_dep_wait();    // activations, sx and the outputs come after the grid this one depends on
+  const uint32_t rbytes = (uint32_t)(p.rpad >> 1);
   if (threadIdx.x == 0 && !pl.withhold_x) {
-    const uint32_t rbytes = (uint32_t)(p.rpad >> 1);
     uint32_t tx = (uint32_t)(p.M * pl.xbytes) + (pl.xrpitch ? (uint32_t)p.M * rbytes : 0u);
     if (!ACC) tx += 8u * (uint32_t)(c1 - c0);
     mbar_arrive_expect_tx(xbar, tx);
-    for (int m = 0; m < p.M; ++m) bulk_load(xs + m * pl.xpitch, p.Xq + (size_t)m * pl.xbytes, pl.xbytes, xbar);
-    if (pl.xrpitch)
-      for (int m = 0; m < p.M; ++m) bulk_load(xr + m * pl.xrpitch, p.Xr + (size_t)m * rbytes, rbytes, xbar);
     if (!ACC) {
-      // sw and sR of the CTA's channels, one piece per layer they touch
-      // (channel ranges and layer bases are multiples of 4: 16-byte pieces)
+      // sw and sR of the CTA's channels (static: before the wait), one piece
+      // per layer they touch (channel ranges and layer bases are multiples
+      // of 4: 16-byte pieces)
       for (int l = 0; l < p.nlayers; ++l) {
         const int a = max(c0, p.lo[l].base), b = min(c1, p.lo[l].base + p.lo[l].N);
         if (a >= b) continue;
@@ -341,6 +334,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
         bulk_load(ssr + (a - c0), p.lo[l].sr + (a - p.lo[l].base), 4u * (uint32_t)(b - a), xbar);
       }
     }
+  }
+  // Shared accumulators and counters.
+  for (int i = threadIdx.x; i < tiles * AccLayout<NTT>::kInts; i += blockDim.x) acc[i] = 0;
+  for (int i = threadIdx.x; i < tiles; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();    // barriers initialised, accumulators zero
+  grid_dep_launch();  // the next kernel in the stream may be scheduled
+  grid_dep_wait();    // activations, sx and the outputs come after the grid this one depends on
+  if (threadIdx.x == 0 && !pl.withhold_x) {
+    for (int m = 0; m < p.M; ++m) bulk_load(xs + m * pl.xpitch, p.Xq + (size_t)m * pl.xbytes, pl.xbytes, xbar);
+    if (pl.xrpitch)
+      for (int m = 0; m < p.M; ++m) bulk_load(xr + m * pl.xrpitch, p.Xr + (size_t)m * rbytes, rbytes, xbar);
   }
   if (!ACC) {
     for (int i = threadIdx.x; i < p.M; i += blockDim.x) {
@@ -445,6 +449,7 @@ inline bool make_plan(const Args& p, int sms, int max_smem, Plan& pl) {
   pl.xrows = 8 * NTT;
   // comparator's residual codes: whole units, rows g, g + 1 in opposite bank halves
   pl.xrpitch = (p.Xr && !A8) ? pl.units_res * 128 + 64 : 0;
+  if (p.C > (1 << 21)) return false;  // keeps chan_begin in 32-bit arithmetic
   int grid = (p.C + 15) / 16;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
