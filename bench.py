@@ -147,7 +147,7 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index, period=0.02):
+    def __init__(self, index, period=0.002):
         self.ok = False
         self.samples = []
         self.reasons = set()
@@ -163,17 +163,20 @@ class ClockSampler:
             self.max_mhz = None
         self._stop = threading.Event()
 
-    def _run(self):
+    def _sample(self):
         nv = self.nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, b in self.REASONS.items():
+                if bits & b and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, b in self.REASONS.items():
-                    if bits & b and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):

@@ -64,9 +64,9 @@ typedef enum {
   SERQ_ALGO_PREFILL = 1,       /* tcgen05 kind::i8 GEMM, TMEM accumulators; the
                                   output tile width is chosen from the shape  */
   SERQ_ALGO_DECODE = 2,        /* memory-bound GEMV (mma.sync), M <= 64: the
-                                  streaming kernel (every SM streams an equal
-                                  share of the channels) where it fits, else
-                                  the item-ring kernel                         */
+                                  streaming kernel when every SM's share of the
+                                  weights is >= 96 KB and it fits, else the
+                                  item-ring kernel                             */
   SERQ_ALGO_PREFILL_N128 = 3,  /* PREFILL with 128 x 128 output tiles, one CTA  */
   SERQ_ALGO_PREFILL_N256 = 4,  /* PREFILL with 128 x 256 output tiles, one CTA  */
   SERQ_ALGO_PREFILL_PAIR_N256 = 5, /* PREFILL with 256 x 256 tiles on a CTA pair
@@ -76,8 +76,12 @@ typedef enum {
   SERQ_ALGO_DECODE_TC = 7,     /* M <= 32: tcgen05 GEMV with the weight rows as the
                                   MMA's M, split-K partial sums in the layer's
                                   workspace (one stream per layer at a time)  */
-  SERQ_ALGO_DECODE_ITEMS = 8   /* M <= 64: the memory-bound GEMV over 16-channel
+  SERQ_ALGO_DECODE_ITEMS = 8,  /* M <= 64: the memory-bound GEMV over 16-channel
                                   items with a shared bulk-copy ring          */
+  SERQ_ALGO_DECODE_STREAM = 9  /* M <= 64: the streaming GEMV (equal channel
+                                  shares per SM, TMA rings per warp) where its
+                                  shared memory fits (M <= 32), else the item
+                                  ring                                         */
 } serq_algo;
 
 typedef struct serq_layer serq_layer;

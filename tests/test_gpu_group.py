@@ -111,7 +111,7 @@ def test_group_decode_sizes(S, M, K, Ns, r, mode):
     single-layer calls of the same kernel."""
     layers, olayers, Xq, sx, xq, osx = _group_case(S, M, K, Ns, r, mode, seed=M + 3 * K + r)
     want = [O.linear_accum(xq, ol) for ol in olayers]
-    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_TC):
+    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_STREAM, S.ALGO_DECODE_TC):
         got = S.linear_group(layers, Xq, accum=True, algo=algo)
         Ys = S.linear_group(layers, Xq, sx, algo=algo)
         singles = [S.linear(L, Xq, sx, algo=algo) for L in layers]
@@ -131,7 +131,7 @@ def test_group_decode_strided_outputs_into_one_buffer(S, M, mode):
     Ns = [256, 128, 96]
     layers, olayers, Xq, sx, xq, osx = _group_case(S, M, 512, Ns, 64, mode, seed=40 + M)
     offs = np.concatenate([[0], np.cumsum(Ns)])
-    for algo in (S.ALGO_DECODE, S.ALGO_DECODE_ITEMS):
+    for algo in (S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_STREAM):
         big = torch.full((M, sum(Ns) + 16), 5.0, dtype=torch.bfloat16, device="cuda")
         Ys = [big[:, offs[l]:offs[l + 1]] for l in range(len(Ns))]
         S.linear_group(layers, Xq, sx, Ys=Ys, algo=algo)

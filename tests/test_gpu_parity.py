@@ -187,7 +187,7 @@ def test_linear_accum_bit_exact(S, mode, M, K, N, r):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, r, mode)
     acc0, acc1 = O.linear_accum(xq, ol)
     algos = [S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
-        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE, S.ALGO_DECODE_ITEMS] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
+        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_STREAM] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
     for algo in algos:
         g0, g1 = S.linear_accum(L, Xq, algo)
         torch.cuda.synchronize()
@@ -203,7 +203,7 @@ def test_linear_output_within_tolerance(S, mode, M, K, N, r):
     acc0, acc1 = O.linear_accum(xq, ol)
     y_ref = O.linear_epilogue(acc0, acc1, osx, ol)
     algos = [S.ALGO_AUTO, S.ALGO_PREFILL_N128, S.ALGO_PREFILL_N256, S.ALGO_PREFILL_PAIR_N256] + \
-        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE, S.ALGO_DECODE_ITEMS] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
+        ([S.ALGO_PREFILL_PAIR_TMEM_A] if mode == "w4a4" else []) + ([S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_STREAM] if M <= 64 else []) + ([S.ALGO_DECODE_TC] if M <= 32 else [])
     for algo in algos:
         Y = S.linear(L, Xq, sx, algo=algo)
         torch.cuda.synchronize()
@@ -213,7 +213,7 @@ def test_linear_output_within_tolerance(S, mode, M, K, N, r):
 def test_linear_strided_output(S):
     L, ol, Xq, sx, xq, osx = _linear_case(S, 40, 256, 128, 16, "w4a4")
     y_ref = O.linear_epilogue(*O.linear_accum(xq, ol), osx, ol)
-    for algo in (S.ALGO_PREFILL, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS):
+    for algo in (S.ALGO_PREFILL, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_STREAM):
         big = torch.full((40, 200), 7.0, dtype=torch.bfloat16, device="cuda")
         S.linear(L, Xq, sx, Y=big[:, 8:136], algo=algo)
         torch.cuda.synchronize()
@@ -372,7 +372,7 @@ def test_llama2_7b_decode(S, M):
     (L,), (ol,) = _prepare_both(S, [p.W], inp.X_calib, wl.rank, "w4a4")
     _, Xq, sx = _gpu_act(S, L, inp.X, "bf16", "w4a4")
     y_ref, xq, osx, acc0, acc1 = O.linear(O.flatten_permute(inp.X, ol.s, ol.pi, True), ol, 4)
-    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_TC):
+    for algo in (S.ALGO_AUTO, S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_STREAM, S.ALGO_DECODE_TC):
         Y = S.linear(L, Xq, sx, algo=algo)
         g0, g1 = S.linear_accum(L, Xq, algo)
         torch.cuda.synchronize()
@@ -390,7 +390,7 @@ def test_llama2_7b_decode(S, M):
 def test_decode_large_k(S, M, K, N, mode):
     L, ol, Xq, sx, xq, osx = _linear_case(S, M, K, N, 128, mode, seed=5)
     acc0, acc1 = O.linear_accum(xq, ol)
-    for algo in [S.ALGO_DECODE, S.ALGO_DECODE_ITEMS] + ([S.ALGO_DECODE_TC] if M <= 32 else []):
+    for algo in [S.ALGO_DECODE, S.ALGO_DECODE_ITEMS, S.ALGO_DECODE_STREAM] + ([S.ALGO_DECODE_TC] if M <= 32 else []):
         g0, g1 = S.linear_accum(L, Xq, algo)
         Y = S.linear(L, Xq, sx, algo=algo)
         torch.cuda.synchronize()

@@ -424,13 +424,19 @@ cudaError_t dispatch_tc(const LinearGroup& G, const void* Xq, const float* sx, i
 }
 
 // The mma.sync decode kernels over a group of layers (one launch; one layer
-// is a group of one): the streaming kernel where its shared memory fits
-// (M <= 32 and the staged activations leave room for the rings), else, or
-// when asked for by SERQ_ALGO_DECODE_ITEMS, the item-ring kernel.
-// fault_wait_ns is zero except in the failure-detection test hook.
+// is a group of one).  kind: 0 = automatic (the streaming kernel when every
+// SM's share of the weights is at least 96 KB and its shared memory fits,
+// else the item ring: for a share of one or two 16-channel items per SM its
+// simpler start-up is measured faster), 1 = item ring, 2 = streaming where
+// it fits.  fault_wait_ns is zero except in the failure-detection test hook.
 cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const float* sx, int M, bool a8, bool accum,
-                                bool items, cudaStream_t st, unsigned long long fault_wait_ns = 0) {
-  if (!items) {
+                                int kind, cudaStream_t st, unsigned long long fault_wait_ns = 0) {
+  if (kind == 0) {
+    double bytes = 0;
+    for (int l = 0; l < G.n; ++l) bytes += (double)G.L[l]->N * (G.L[l]->K / 2 + G.L[l]->rpad / 2);
+    kind = (bytes >= 96.0 * 1024 * sm_count() || fault_wait_ns) ? 2 : 1;
+  }
+  if (kind == 2) {
     serq::gs::Args g = {};
     serq::gs::Maps mp;
     g.Xq = static_cast<const uint8_t*>(Xq);
@@ -484,6 +490,10 @@ cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const floa
                : serq::decode::launch<false, false>(a, sm_count(), max_smem(), st);
 }
 
+int decode_kind(serq_algo a) {
+  return a == SERQ_ALGO_DECODE_ITEMS ? 1 : a == SERQ_ALGO_DECODE_STREAM ? 2 : 0;
+}
+
 // Argument checks shared by the single-layer and grouped calls; resolves AUTO.
 serq_status check_linear(const serq_layer* L, const void* Xq, const float* sx, int M, const void* Y, int ldy,
                          const int32_t* acc0, const int32_t* acc1, serq_algo* algo_io) {
@@ -504,11 +514,12 @@ serq_status check_linear(const serq_layer* L, const void* Xq, const float* sx, i
       return fail(SERQ_ERR_INVALID_ARG, "Y must be 16-byte aligned with ldy a multiple of 8");
   }
   if (algo == SERQ_ALGO_AUTO) algo = (M <= serq_decode_max_m()) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
-  if ((algo == SERQ_ALGO_DECODE || algo == SERQ_ALGO_DECODE_ITEMS) && M > serq::decode::kMaxTiles * 16)
+  if ((algo == SERQ_ALGO_DECODE || algo == SERQ_ALGO_DECODE_ITEMS || algo == SERQ_ALGO_DECODE_STREAM) &&
+      M > serq::decode::kMaxTiles * 16)
     return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "decode kernel takes M <= %d (got %d)", serq::decode::kMaxTiles * 16, M);
   if (algo == SERQ_ALGO_DECODE_TC && M > serq::dtc::kMaxM)
     return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "SERQ_ALGO_DECODE_TC takes M <= %d (got %d)", serq::dtc::kMaxM, M);
-  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_DECODE_ITEMS) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
+  if (algo < SERQ_ALGO_PREFILL || algo > SERQ_ALGO_DECODE_STREAM) return fail(SERQ_ERR_INVALID_ARG, "bad algo %d", (int)algo);
   if (algo == SERQ_ALGO_PREFILL_PAIR_TMEM_A && L->mode != SERQ_W4A4)
     return fail(SERQ_ERR_INVALID_ARG, "SERQ_ALGO_PREFILL_PAIR_TMEM_A takes W4A4 layers");
   if ((s = check_device())) return s;
@@ -534,7 +545,7 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
       e = accum ? dispatch_decode_tc<true, true>(L, Xq, a, st) : dispatch_decode_tc<true, false>(L, Xq, a, st);
     else
       e = accum ? dispatch_decode_tc<false, true>(L, Xq, a, st) : dispatch_decode_tc<false, false>(L, Xq, a, st);
-  } else if (algo == SERQ_ALGO_DECODE || algo == SERQ_ALGO_DECODE_ITEMS) {
+  } else if (algo == SERQ_ALGO_DECODE || algo == SERQ_ALGO_DECODE_ITEMS || algo == SERQ_ALGO_DECODE_STREAM) {
     LinearGroup G = {};
     G.n = 1;
     G.L[0] = L;
@@ -542,7 +553,7 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
     G.ldy[0] = ldy;
     G.acc0[0] = acc0;
     G.acc1[0] = acc1;
-    e = launch_decode_group(G, Xq, sx, M, a8, accum, algo == SERQ_ALGO_DECODE_ITEMS, st);
+    e = launch_decode_group(G, Xq, sx, M, a8, accum, decode_kind(algo), st);
   } else {
     LinearGroup G = {};
     G.n = 1;
@@ -603,8 +614,8 @@ serq_status group_impl(int n, const serq_layer* const* Ls, const void* Xq, const
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (resolved == SERQ_ALGO_DECODE || resolved == SERQ_ALGO_DECODE_ITEMS) {
-    e = launch_decode_group(G, Xq, sx, M, Ls[0]->mode == SERQ_W4A8, accum, resolved == SERQ_ALGO_DECODE_ITEMS, st);
+  if (resolved == SERQ_ALGO_DECODE || resolved == SERQ_ALGO_DECODE_ITEMS || resolved == SERQ_ALGO_DECODE_STREAM) {
+    e = launch_decode_group(G, Xq, sx, M, Ls[0]->mode == SERQ_W4A8, accum, decode_kind(resolved), st);
     if (e != cudaSuccess) return cuda_fail(e, "serq_linear_group launch");
     return ok();
   }
@@ -1063,7 +1074,7 @@ serq_status serq_test_decode_timeout(const serq_layer* layer, const void* Xq, co
   G.L[0] = layer;
   G.Y[0] = static_cast<__nv_bfloat16*>(Y);
   G.ldy[0] = ldy;
-  cudaError_t e = launch_decode_group(G, Xq, sx, M, layer->mode == SERQ_W4A8, false, false,
+  cudaError_t e = launch_decode_group(G, Xq, sx, M, layer->mode == SERQ_W4A8, false, 2,
                                       static_cast<cudaStream_t>(stream), (unsigned long long)wait_us * 1000ull);
   if (e != cudaSuccess) return cuda_fail(e, "serq_test_decode_timeout launch");
   return ok();

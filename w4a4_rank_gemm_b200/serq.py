@@ -24,7 +24,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_UNSUPPORTED_DEVICE, ERR_ALLOC, E
 W4A4, W4A8 = 0, 1
 F32, BF16 = 0, 1
 (ALGO_AUTO, ALGO_PREFILL, ALGO_DECODE, ALGO_PREFILL_N128, ALGO_PREFILL_N256, ALGO_PREFILL_PAIR_N256,
- ALGO_PREFILL_PAIR_TMEM_A, ALGO_DECODE_TC, ALGO_DECODE_ITEMS) = 0, 1, 2, 3, 4, 5, 6, 7, 8
+ ALGO_PREFILL_PAIR_TMEM_A, ALGO_DECODE_TC, ALGO_DECODE_ITEMS, ALGO_DECODE_STREAM) = 0, 1, 2, 3, 4, 5, 6, 7, 8, 9
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
