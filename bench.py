@@ -533,10 +533,11 @@ def run_gpu(args, rank, world, local_rank):
         peak = pk.get("hbm_gbs")
         achieved = W.gemm_bytes_step * roof_steps / (gemm_ms / 1e3) / 1e9
         res["roofline"] = {
-            "kernel": "serq::gs::k_gemv (streaming mma.sync GEMV, main + residual accumulators)",
+            "kernel": ("decode GEMVs, main + residual accumulators: serq::gs::k_gemv (streaming; q/k/v, gate/up, "
+                       "down) and serq::decode::k_decode (item ring; o_proj)"),
             "bound": "hbm", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": recorded_traffic(f"{W.name}_M{W.M}", ["gemv_stream.cuh", "common.cuh"]),
+            "traffic": recorded_traffic(f"{W.name}_M{W.M}", ["gemv_stream.cuh", "gemv_decode.cuh", "common.cuh"]),
             "peak_source": f"{pk_src}: hbm_gbs" + (" -- of measured" if pk_src != "fallback" else " -- of fallback"),
             "gemm_share_of_step": round(gemm_ms / roof_steps / max(elapsed_ms / args.steps, 1e-9), 4),
             "timing": gemm_note,
