@@ -48,7 +48,8 @@ typedef enum {
   SERQ_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100           */
   SERQ_ERR_ALLOC = 4,              /* cudaMalloc failed (prepare only)       */
   SERQ_ERR_CUDA = 5,               /* a CUDA call or kernel launch failed    */
-  SERQ_ERR_TIMEOUT = 6             /* a kernel gave up a bounded wait        */
+  SERQ_ERR_TIMEOUT = 6,            /* a kernel gave up a bounded wait        */
+  SERQ_ERR_NUMERIC = 7             /* GPTQ: a Cholesky pivot was not positive */
 } serq_status;
 
 typedef enum { SERQ_W4A4 = 0, SERQ_W4A8 = 1 } serq_mode;
@@ -97,6 +98,12 @@ typedef enum {
   SERQ_SALIENCY_ROW_ABSMAX = 1  /* by the folded row's max |s_j W_jn|        */
 } serq_saliency;
 
+/* Quantizer of the main weight in step 3 below. */
+typedef enum {
+  SERQ_QUANT_RTN = 0,  /* round-to-nearest (default; the pages' RTN)          */
+  SERQ_QUANT_GPTQ = 1  /* GPTQ past the r salient rows ("SERQ(GPTQ)")         */
+} serq_quantizer;
+
 /* Options of the offline stage.  Fill with serq_prepare_opts_init, then
  * change what differs. */
 typedef struct {
@@ -111,9 +118,11 @@ typedef struct {
   const float* out_colscale;  /* serq_prepare only: nullable HOST float[N],
                                  the NEXT layer's smoothing scales, divided
                                  into the columns (step 5); needs out_perm   */
+  int quantizer;              /* serq_quantizer; default SERQ_QUANT_RTN      */
 } serq_prepare_opts;
 
-/* Defaults: alpha 0.5, rank 128, SERQ_W4A4, SERQ_SALIENCY_SCALE, no fold. */
+/* Defaults: alpha 0.5, rank 128, SERQ_W4A4, SERQ_SALIENCY_SCALE, no fold,
+ * SERQ_QUANT_RTN. */
 void serq_prepare_opts_init(serq_prepare_opts* opts);
 
 /*
@@ -132,6 +141,15 @@ void serq_prepare_opts_init(serq_prepare_opts* opts);
  *     channel index (key design 2);
  *  3. W^ = P diag(s) W, quantized per output channel to INT4:
  *     code = clamp(rint(W^ * (7/amax)), -7, 7), sw = amax/7;
+ *     With opts->quantizer = SERQ_QUANT_GPTQ ("SERQ(GPTQ)" in the SERQ notes'
+ *     main results; gist.science (de) 2B names RTN or GPTQ for the main
+ *     weight), rows r.. are quantized by GPTQ instead: with U the upper
+ *     Cholesky factor of the inverse of H = sum_t xh_t xh_t^T + 0.01 *
+ *     mean(diag) * I over the flattened, permuted calibration activations
+ *     xh (serq_gptq_factor), row by row in order, e_i = (w_i - code_i*sw) /
+ *     u_ii (fp32, U rounded to fp32) and w_j -= u_ij * e_i for j > i; the
+ *     salient rows 0..r-1 keep round-to-nearest and move nothing (R below
+ *     corrects them); amax and sw are the column's before any update;
  *  4. R = W^[0:r] - code[0:r]*sw (the main path's own error on the r salient
  *     rows, key design 2 / core idea), quantized the same way -> Rq, sR;
  *  5. optionally, before all of the above, the NEXT layer's order and
@@ -146,10 +164,12 @@ void serq_prepare_opts_init(serq_prepare_opts* opts);
  *  X_calib  HOST, n_calib x K fp32 calibration activations (n_calib >= 1).
  *  opts     options (NULL = the defaults above).
  *  layer    receives the new handle (NULL on failure; nothing leaks).
- * Errors: SERQ_ERR_INVALID_ARG (null pointers, alpha outside [0, 1], bad mode
- * or metric, out_colscale without out_perm), SERQ_ERR_UNSUPPORTED_SHAPE
- * (K or N not a multiple of 32, rank outside [0, K]), SERQ_ERR_ALLOC,
- * SERQ_ERR_CUDA, SERQ_ERR_UNSUPPORTED_DEVICE.  Synchronous.
+ * Errors: SERQ_ERR_INVALID_ARG (null pointers, alpha outside [0, 1], bad mode,
+ * metric or quantizer, out_colscale without out_perm),
+ * SERQ_ERR_UNSUPPORTED_SHAPE (K or N not a multiple of 32, rank outside
+ * [0, K]), SERQ_ERR_ALLOC, SERQ_ERR_CUDA, SERQ_ERR_UNSUPPORTED_DEVICE,
+ * SERQ_ERR_NUMERIC (GPTQ only: the damped Hessian or its inverse was not
+ * positive definite in floating point).  Synchronous.
  */
 serq_status serq_prepare(const float* W, int K, int N, const float* X_calib, int n_calib,
                          const serq_prepare_opts* opts, serq_layer** layer);
@@ -186,6 +206,29 @@ serq_status serq_prepare_group(int n_weights, const float* const* W, const int* 
                                const float* X_calib, int n_calib, const serq_prepare_opts* opts,
                                const int32_t* const* out_perm, const float* const* out_colscale,
                                serq_layer** layers);
+
+/*
+ * serq_gptq_factor -- the inverse-Hessian factor GPTQ uses (serq_prepare's
+ * step 3 with SERQ_QUANT_GPTQ computes it internally; this call exposes it).
+ *   H = sum_t xh_t xh_t^T over the n_calib rows of Xh, in token order (fp64),
+ *   H_ii += 0.01 * (H_00 + ... + H_K-1,K-1) / K   (H = I if that sum is 0),
+ *   H = L L^T (Cholesky), V = L^-1, H^-1 = V^T V = L2 L2^T, U = L2^T,
+ * so H^-1 = U^T U with U upper triangular (GPTQ, Frantar et al. 2022).
+ * Every fp64 entry receives its terms in the order of the textbook
+ * unblocked loops (sums from +0 in increasing index; Cholesky and forward
+ * substitution subtracting their products in increasing index), one
+ * rounding per product, sum, difference, quotient and square root, so the
+ * result does not depend on the blocking.
+ *  Xh  DEVICE, n_calib x K fp32, row-major: the flattened, permuted
+ *      calibration activations (X[:, P] / s[P]).
+ *  U   DEVICE, K x K fp64, row-major; receives U (zeros below the diagonal).
+ *  K a positive multiple of 32, n_calib >= 1.  Uses 2 K^2 fp64 of
+ *  temporary device memory.
+ * Errors: SERQ_ERR_INVALID_ARG, SERQ_ERR_UNSUPPORTED_SHAPE, SERQ_ERR_ALLOC,
+ * SERQ_ERR_CUDA, SERQ_ERR_NUMERIC (a pivot that is not positive; U is then
+ * not meaningful).  Synchronous.
+ */
+serq_status serq_gptq_factor(const float* Xh, int n_calib, int K, double* U);
 
 /* Frees the handle's device memory.  NULL is accepted.  Synchronous. */
 void serq_layer_destroy(serq_layer* layer);

@@ -79,8 +79,8 @@ def test_prepare_options_host_side_rejection(lib):
     L = lib.lib
     o = lib.PrepareOpts()
     L.serq_prepare_opts_init(ctypes.byref(o))
-    assert (abs(o.alpha - 0.5) < 1e-9, o.rank, o.mode, o.saliency, o.out_perm, o.out_colscale) == \
-        (True, 128, lib.W4A4, lib.SALIENCY_SCALE, None, None)
+    assert (abs(o.alpha - 0.5) < 1e-9, o.rank, o.mode, o.saliency, o.out_perm, o.out_colscale, o.quantizer) == \
+        (True, 128, lib.W4A4, lib.SALIENCY_SCALE, None, None, lib.QUANT_RTN)
     W = np.zeros((256, 64), np.float32)
     Xc = np.zeros((4, 256), np.float32)
     out = ctypes.c_void_p()
@@ -89,7 +89,8 @@ def test_prepare_options_host_side_rejection(lib):
                                       ("alpha", float("nan"), lib.ERR_INVALID_ARG, b"alpha"),
                                       ("rank", 257, lib.ERR_UNSUPPORTED_SHAPE, b"rank"),
                                       ("mode", 7, lib.ERR_INVALID_ARG, b"mode"),
-                                      ("saliency", 2, lib.ERR_INVALID_ARG, b"saliency")):
+                                      ("saliency", 2, lib.ERR_INVALID_ARG, b"saliency"),
+                                      ("quantizer", 2, lib.ERR_INVALID_ARG, b"quantizer")):
         o = lib.prepare_opts(rank=32)
         setattr(o, field, value)
         assert L.serq_prepare(wp, 256, 64, xp, 4, ctypes.byref(o), ctypes.byref(out)) == status
@@ -111,6 +112,12 @@ def test_prepare_options_host_side_rejection(lib):
     assert outs[0] is None
     # silu: null inputs
     assert L.serq_silu_mul_quantize(None, None, 4, 256, 256, lib.W4A4, None, None, None) == lib.ERR_INVALID_ARG
+    # the GPTQ factor: null pointers, K not a multiple of 32, no calibration rows
+    buf = ctypes.c_void_p(1 << 20)
+    assert L.serq_gptq_factor(None, 4, 256, buf) == lib.ERR_INVALID_ARG
+    assert L.serq_gptq_factor(buf, 4, 256, None) == lib.ERR_INVALID_ARG
+    assert L.serq_gptq_factor(buf, 4, 100, buf) == lib.ERR_UNSUPPORTED_SHAPE
+    assert L.serq_gptq_factor(buf, 0, 256, buf) == lib.ERR_INVALID_ARG
 
 
 def test_group_call_host_side_rejection(lib):

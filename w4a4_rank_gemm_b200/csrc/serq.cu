@@ -19,6 +19,7 @@
 #include "gemv_stream.cuh"
 #include "gemv_tc.cuh"
 #include "prepare.cuh"
+#include "gptq.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -725,6 +726,7 @@ void serq_prepare_opts_init(serq_prepare_opts* opts) {
   opts->saliency = SERQ_SALIENCY_SCALE;
   opts->out_perm = nullptr;
   opts->out_colscale = nullptr;
+  opts->quantizer = SERQ_QUANT_RTN;
 }
 
 }  // extern "C"
@@ -739,6 +741,109 @@ serq_status check_opts(const serq_prepare_opts* o, int K) {
   if (o->mode != SERQ_W4A4 && o->mode != SERQ_W4A8) return fail(SERQ_ERR_INVALID_ARG, "bad mode %d", (int)o->mode);
   if (o->saliency != SERQ_SALIENCY_SCALE && o->saliency != SERQ_SALIENCY_ROW_ABSMAX)
     return fail(SERQ_ERR_INVALID_ARG, "bad saliency metric %d", o->saliency);
+  if (o->quantizer != SERQ_QUANT_RTN && o->quantizer != SERQ_QUANT_GPTQ)
+    return fail(SERQ_ERR_INVALID_ARG, "bad quantizer %d", o->quantizer);
+  return SERQ_OK;
+}
+
+// Device buffers of one call, freed when the owner goes out of scope.
+struct Scratch {
+  std::vector<void*> bufs;
+  ~Scratch() {
+    for (void* b : bufs) cudaFree(b);
+  }
+  template <class T>
+  serq_status get(size_t count, T** out, const char* what) {
+    *out = nullptr;
+    void* d = nullptr;
+    cudaError_t e = cudaMalloc(&d, std::max<size_t>(count, 1) * sizeof(T));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(SERQ_ERR_ALLOC, "cudaMalloc of %zu bytes for %s failed: %s", count * sizeof(T), what,
+                  cudaGetErrorString(e));
+    }
+    bufs.push_back(d);
+    *out = static_cast<T*>(d);
+    return SERQ_OK;
+  }
+};
+
+template <typename TP, bool PT, bool QT, bool SUB>
+void launch_tile(const serq::gptq::TileArgs& a, cudaStream_t st) {
+  using namespace serq::gptq;
+  const int ti = (a.mi + kTile - 1) / kTile;
+  const int blocks = a.lower ? ti * (ti + 1) / 2 : ti * a.ntj;
+  if (blocks > 0) k_tile<TP, PT, QT, SUB><<<blocks, 256, 0, st>>>(a);
+}
+
+// In-place Cholesky of the lower triangle of A (K x K): 32-column panels,
+// each the diagonal block, the rows below it, then the trailing update.
+void chol_lower(double* A, int K, int* status, cudaStream_t st) {
+  using namespace serq::gptq;
+  for (int j0 = 0; j0 < K; j0 += kChunk) {
+    k_chol_diag<<<1, 32, 0, st>>>(A, K, j0, status);
+    const int rest = K - j0 - kChunk;
+    if (rest <= 0) break;
+    k_chol_trsm<<<(rest + 127) / 128, 128, 0, st>>>(A, K, j0);
+    TileArgs t{};
+    t.C = A; t.ldc = K; t.ci0 = t.cj0 = j0 + kChunk; t.mi = t.mj = rest;
+    t.P = A; t.ldp = K; t.pi0 = j0 + kChunk;
+    t.Q = A; t.ldq = K; t.qj0 = j0 + kChunk;
+    t.kb = j0; t.ke = j0 + kChunk; t.lower = 1;
+    launch_tile<double, true, true, true>(t, st);
+  }
+}
+
+// U (K x K upper; fp32 and/or fp64) with H^-1 = U^T U for the damped
+// Hessian of Xh (n x K fp32, device).  All pointers device.
+serq_status gptq_factor(const float* Xh, int n, int K, float* U32, double* U64, cudaStream_t st) {
+  using namespace serq::gptq;
+  Scratch sc;
+  double *A = nullptr, *B = nullptr;
+  int* status = nullptr;
+  serq_status s;
+  const size_t kk = (size_t)K * K;
+  if ((s = sc.get(kk, &A, "the GPTQ Hessian"))) return s;
+  if ((s = sc.get(kk, &B, "the GPTQ inverse"))) return s;
+  if ((s = sc.get(1, &status, "a status word"))) return s;
+  cudaMemsetAsync(status, 0, sizeof(int), st);
+  // H = Xh^T Xh (lower), damped
+  TileArgs g{};
+  g.C = A; g.ldc = K; g.mi = g.mj = K;
+  g.P = Xh; g.ldp = K; g.Q = Xh; g.ldq = K;
+  g.kb = 0; g.ke = n; g.lower = 1;
+  launch_tile<float, false, false, false>(g, st);
+  k_damp<<<1, 256, 0, st>>>(A, K);
+  chol_lower(A, K, status, st);
+  // V = L^-1 in B (forward substitution on the identity, 32-row panels)
+  const unsigned eb = (unsigned)((kk + 255) / 256);
+  k_identity<<<eb, 256, 0, st>>>(B, K);
+  for (int i0 = 0; i0 < K; i0 += kChunk) {
+    k_inv_panel<<<(i0 + kChunk + 127) / 128, 128, 0, st>>>(A, B, K, i0);
+    const int rest = K - i0 - kChunk;
+    if (rest <= 0) break;
+    TileArgs t{};
+    t.C = B; t.ldc = K; t.ci0 = i0 + kChunk; t.cj0 = 0; t.mi = rest; t.mj = i0 + kChunk;
+    t.P = A; t.ldp = K; t.pi0 = i0 + kChunk;
+    t.Q = B; t.ldq = K; t.qj0 = 0;
+    t.kb = i0; t.ke = i0 + kChunk; t.lower = 0; t.ntj = (t.mj + kTile - 1) / kTile;
+    launch_tile<double, true, false, true>(t, st);
+  }
+  // H^-1 = V^T V (lower; a tile's sum starts at its first row: V is lower)
+  TileArgs h{};
+  h.C = A; h.ldc = K; h.mi = h.mj = K;
+  h.P = B; h.ldp = K; h.Q = B; h.ldq = K;
+  h.kb = 0; h.ke = K; h.kb_row_tile = 1; h.lower = 1;
+  launch_tile<double, false, false, false>(h, st);
+  chol_lower(A, K, status, st);
+  k_upper_from_lower<<<eb, 256, 0, st>>>(A, K, U32, U64);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "GPTQ factor launch");
+  int flag = 0;
+  e = cudaMemcpyAsync(&flag, status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "GPTQ factor");
+  if (flag) return fail(SERQ_ERR_NUMERIC, "GPTQ: a Cholesky pivot was not positive (K = %d, %d calibration rows)", K, n);
   return SERQ_OK;
 }
 
@@ -795,6 +900,30 @@ serq_status prepare_impl(int n_weights, const float* const* W, const int* N, int
     cudaMemcpyAsync(layers[i]->smooth, L0->smooth, sizeof(float) * K, cudaMemcpyDeviceToDevice, st);
     cudaMemcpyAsync(layers[i]->perm, L0->perm, sizeof(int32_t) * K, cudaMemcpyDeviceToDevice, st);
   }
+  // 3 (GPTQ). the inverse-Hessian factor of the flattened, permuted
+  // calibration activations, shared by every weight of the group
+  Scratch gsc;
+  float* U32 = nullptr;
+  float* E = nullptr;
+  if (o.quantizer == SERQ_QUANT_GPTQ) {
+    int max_n = 0;
+    for (int i = 0; i < n_weights; ++i) max_n = std::max(max_n, N[i]);
+    float* Xh = nullptr;
+    if (!(s = gsc.get((size_t)n_calib * K, &Xh, "the flattened calibration activations")) &&
+        !(s = gsc.get((size_t)K * K, &U32, "the GPTQ factor")) &&
+        !(s = gsc.get((size_t)K * max_n, &E, "the GPTQ errors"))) {
+      const size_t ne = (size_t)n_calib * K;
+      serq::gptq::k_flatten<<<(unsigned)((ne + 255) / 256), 256, 0, st>>>(X_calib, L0->smooth, L0->perm, n_calib,
+                                                                        K, Xh);
+      s = gptq_factor(Xh, n_calib, K, U32, nullptr, st);
+    }
+    if (s) {
+      cudaStreamSynchronize(st);
+      cudaStreamDestroy(st);
+      cudaFree(key);
+      return cleanup(s);
+    }
+  }
   // 3-4. per weight: quantize W^ per output channel, compensator R
   for (int i = 0; i < n_weights; ++i) {
     serq_layer* Li = layers[i];
@@ -804,7 +933,11 @@ serq_status prepare_impl(int n_weights, const float* const* W, const int* N, int
     cudaMemsetAsync(Li->sw, 0, sizeof(float) * Ni, st);
     k_colmax_what<<<dim3((Ni + 255) / 256, (K + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(
         v, L0->smooth, L0->perm, K, rows_per_block, Li->sw);
-    k_quant_pack_w<<<dim3((Ni + 127) / 128, K / 32), 128, 0, st>>>(v, L0->smooth, L0->perm, K, Li->sw, Li->wq);
+    if (o.quantizer == SERQ_QUANT_GPTQ)
+      serq::gptq::k_gptq_pack_w<<<(Ni + 127) / 128, 128, 0, st>>>(v, L0->smooth, L0->perm, K, rank, Li->sw, U32, E,
+                                                                  Li->wq);
+    else
+      k_quant_pack_w<<<dim3((Ni + 127) / 128, K / 32), 128, 0, st>>>(v, L0->smooth, L0->perm, K, Li->sw, Li->wq);
     if (rank > 0) {
       k_colmax_resid<<<(Ni + 127) / 128, 128, 0, st>>>(v, L0->smooth, L0->perm, rank, Li->sw, Li->sr);
       k_quant_pack_r<<<dim3((Ni + 127) / 128, Li->rpad / 32), 128, 0, st>>>(v, L0->smooth, L0->perm, rank,
@@ -899,6 +1032,21 @@ serq_status serq_prepare_group(int n_weights, const float* const* W, const int* 
   serq_status s = check_group_args(n_weights, W, N, K, X_calib, n_calib, opts, out_perm, out_colscale, layers);
   if (s) return s;
   return prepare_impl(n_weights, W, N, K, X_calib, n_calib, *opts, out_perm, out_colscale, layers);
+}
+
+serq_status serq_gptq_factor(const float* Xh, int n_calib, int K, double* U) {
+  if (!Xh || !U) return fail(SERQ_ERR_INVALID_ARG, "null Xh or U");
+  if (K < 32 || K % 32) return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "K = %d must be a positive multiple of 32", K);
+  if (n_calib < 1) return fail(SERQ_ERR_INVALID_ARG, "n_calib = %d", n_calib);
+  serq_status s = check_device();
+  if (s) return s;
+  cudaStream_t st;
+  cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate");
+  s = gptq_factor(Xh, n_calib, K, nullptr, U, st);
+  cudaStreamSynchronize(st);
+  cudaStreamDestroy(st);
+  return s ? s : ok();
 }
 
 serq_status serq_prepare_shared(int n_weights, const float* const* W, const int* N, int K, const float* X_calib,

@@ -20,7 +20,7 @@ if not os.path.exists(LIB_PATH):
 lib = ctypes.CDLL(LIB_PATH)
 
 # enums
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_UNSUPPORTED_DEVICE, ERR_ALLOC, ERR_CUDA, ERR_TIMEOUT = range(7)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_UNSUPPORTED_DEVICE, ERR_ALLOC, ERR_CUDA, ERR_TIMEOUT, ERR_NUMERIC = range(8)
 W4A4, W4A8 = 0, 1
 F32, BF16 = 0, 1
 (ALGO_AUTO, ALGO_PREFILL, ALGO_DECODE, ALGO_PREFILL_N128, ALGO_PREFILL_N256, ALGO_PREFILL_PAIR_N256,
@@ -29,12 +29,13 @@ F32, BF16 = 0, 1
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
 SALIENCY_SCALE, SALIENCY_ROW_ABSMAX = 0, 1
+QUANT_RTN, QUANT_GPTQ = 0, 1
 
 
 class PrepareOpts(ctypes.Structure):
     """serq_prepare_opts."""
     _fields_ = [("alpha", ctypes.c_float), ("rank", _i), ("mode", _i), ("saliency", _i),
-                ("out_perm", _vp), ("out_colscale", _vp)]
+                ("out_perm", _vp), ("out_colscale", _vp), ("quantizer", _i)]
 
 
 EXPORTS = {
@@ -45,6 +46,7 @@ EXPORTS = {
                                  ctypes.POINTER(PrepareOpts), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                  ctypes.POINTER(_vp)]),
     "serq_prepare": (_i, [_vp, _i, _i, _vp, _i, ctypes.POINTER(PrepareOpts), ctypes.POINTER(_vp)]),
+    "serq_gptq_factor": (_i, [_vp, _i, _i, _vp]),
     "serq_layer_get_perm": (_i, [_vp, _vp]),
     "serq_layer_get_smooth": (_i, [_vp, _vp]),
     "serq_layer_destroy": (None, [_vp]),
@@ -178,20 +180,28 @@ class Layer:
                     sw=sw, sr=sr, perm=perm, smooth=smooth)
 
 
-def prepare_opts(rank: int = 128, mode="w4a4", alpha: float = 0.5, saliency: int = SALIENCY_SCALE) -> PrepareOpts:
+def _quantizer_code(q) -> int:
+    if isinstance(q, str):
+        return {"rtn": QUANT_RTN, "gptq": QUANT_GPTQ}[q.lower()]
+    return int(q)
+
+
+def prepare_opts(rank: int = 128, mode="w4a4", alpha: float = 0.5, saliency: int = SALIENCY_SCALE,
+                 quantizer="rtn") -> PrepareOpts:
     o = PrepareOpts()
     lib.serq_prepare_opts_init(ctypes.byref(o))
     o.rank, o.mode, o.alpha, o.saliency = rank, _mode_code(mode), alpha, saliency
+    o.quantizer = _quantizer_code(quantizer)
     return o
 
 
 def prepare_group(weights: Sequence[torch.Tensor], X_calib: torch.Tensor, rank: int, mode="w4a4",
                   out_perm: Optional[Sequence[Optional[torch.Tensor]]] = None,
                   out_div: Optional[Sequence[Optional[torch.Tensor]]] = None,
-                  alpha: float = 0.5, saliency: int = SALIENCY_SCALE) -> List[Layer]:
+                  alpha: float = 0.5, saliency: int = SALIENCY_SCALE, quantizer="rtn") -> List[Layer]:
     """serq_prepare_group: weights are CUDA fp32 K x N tensors sharing one
     input; out_perm / out_div are the next layer's order and smoothing scales
-    per weight (CUDA tensors or None)."""
+    per weight (CUDA tensors or None); quantizer "rtn" or "gptq"."""
     n = len(weights)
     K = weights[0].shape[0]
     for w in weights:
@@ -206,15 +216,28 @@ def prepare_group(weights: Sequence[torch.Tensor], X_calib: torch.Tensor, rank: 
     ps = (_vp * n)(*[(p.data_ptr() if p is not None else None) for p in (out_perm or [None] * n)])
     ds = (_vp * n)(*[(d.data_ptr() if d is not None else None) for d in (out_div or [None] * n)])
     outs = (_vp * n)()
-    o = prepare_opts(rank, mode, alpha, saliency)
+    o = prepare_opts(rank, mode, alpha, saliency, quantizer)
     _check(lib.serq_prepare_group(n, Ws, Ns, K, _ptr(X_calib), X_calib.shape[0], ctypes.byref(o), ps, ds, outs),
            "serq_prepare_group")
     return [Layer(_vp(outs[i])) for i in range(n)]
 
 
 def prepare(W: torch.Tensor, X_calib: torch.Tensor, rank: int, mode="w4a4", out_perm=None,
-            out_div=None, alpha: float = 0.5, saliency: int = SALIENCY_SCALE) -> Layer:
-    return prepare_group([W], X_calib, rank, mode, [out_perm], [out_div], alpha, saliency)[0]
+            out_div=None, alpha: float = 0.5, saliency: int = SALIENCY_SCALE, quantizer="rtn") -> Layer:
+    return prepare_group([W], X_calib, rank, mode, [out_perm], [out_div], alpha, saliency, quantizer)[0]
+
+
+def gptq_factor(Xh: torch.Tensor) -> torch.Tensor:
+    """serq_gptq_factor: Xh is the CUDA fp32 n x K flattened, permuted
+    calibration activations; returns the K x K fp64 upper factor U with
+    H^-1 = U^T U."""
+    _cuda2d(Xh, "Xh")
+    if Xh.dtype != torch.float32 or not Xh.is_contiguous():
+        raise ValueError("Xh must be contiguous fp32")
+    K = Xh.shape[1]
+    U = torch.empty((K, K), dtype=torch.float64, device=Xh.device)
+    _check(lib.serq_gptq_factor(_ptr(Xh), Xh.shape[0], K, _ptr(U)), "serq_gptq_factor")
+    return U
 
 
 def _host_f32(a, name):
@@ -226,13 +249,13 @@ def _host_f32(a, name):
 
 
 def prepare_host(W, X_calib, rank: int = 128, mode="w4a4", alpha: float = 0.5,
-                 saliency: int = SALIENCY_SCALE, out_perm=None, out_colscale=None) -> Layer:
+                 saliency: int = SALIENCY_SCALE, out_perm=None, out_colscale=None, quantizer="rtn") -> Layer:
     """serq_prepare: W (K x N) and X_calib (n x K) are host (numpy) arrays;
     the library uploads them."""
     import numpy as np
     W = _host_f32(W, "W")
     Xc = _host_f32(X_calib, "X_calib")
-    o = prepare_opts(rank, mode, alpha, saliency)
+    o = prepare_opts(rank, mode, alpha, saliency, quantizer)
     keep = []
     if out_perm is not None:
         keep.append(np.ascontiguousarray(out_perm, dtype=np.int32))
@@ -247,13 +270,14 @@ def prepare_host(W, X_calib, rank: int = 128, mode="w4a4", alpha: float = 0.5,
 
 
 def prepare_shared_host(weights, X_calib, rank: int = 128, mode="w4a4", alpha: float = 0.5,
-                        saliency: int = SALIENCY_SCALE, out_perm=None, out_colscale=None) -> List[Layer]:
+                        saliency: int = SALIENCY_SCALE, out_perm=None, out_colscale=None,
+                        quantizer="rtn") -> List[Layer]:
     """serq_prepare_shared: host (numpy) weights sharing one input."""
     import numpy as np
     Ws = [_host_f32(w, "W") for w in weights]
     n = len(Ws)
     Xc = _host_f32(X_calib, "X_calib")
-    o = prepare_opts(rank, mode, alpha, saliency)
+    o = prepare_opts(rank, mode, alpha, saliency, quantizer)
     keep = list(Ws)
     def arr(seq, dt):
         if seq is None:
