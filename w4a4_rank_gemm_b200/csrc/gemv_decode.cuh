@@ -218,8 +218,9 @@ __global__ void __launch_bounds__(kThreads, (!A8 && MT == 1) ? 2 : 1) k_decode(c
 
   if (warp == kComputeWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      bool ok = true;
+    bool ok = true;
+    int item = blockIdx.x, j = 0;
+    {
       auto issue = [&](int item, int j) -> bool {
         const int s = j % pl.stages;
         const uint32_t ph = (j / pl.stages) & 1;
@@ -236,15 +237,20 @@ __global__ void __launch_bounds__(kThreads, (!A8 && MT == 1) ? 2 : 1) k_decode(c
         bulk_load(sc + kRows * 4, lo.sr + n0, kRows * 4, &full[s]);
         return true;
       };
-      int item = blockIdx.x, j = 0;
       // weights first: no earlier kernel writes them
-      for (; ok && item < pl.items && j < pl.stages; item += gridDim.x, ++j) ok = issue(item, j);
+      if (lane == 0)
+        for (; ok && item < pl.items && j < pl.stages; item += gridDim.x, ++j) ok = issue(item, j);
       grid_dep_wait();
+      ok = __shfl_sync(0xffffffffu, ok, 0);
       if (ok && ACT_SMEM) {
-        mbar_arrive_expect_tx(act_full, (uint32_t)(p.M * pl.kb));
-        for (int m = 0; m < p.M; ++m) bulk_load(act + m * pl.act_pitch, p.Xq + (size_t)m * pl.kb, pl.kb, act_full);
+        // the token rows' copies go out side by side, one lane each
+        if (lane == 0) mbar_arrive_expect_tx(act_full, (uint32_t)(p.M * pl.kb));
+        __syncwarp();
+        for (int m = lane; m < p.M; m += 32)
+          bulk_load(act + m * pl.act_pitch, p.Xq + (size_t)m * pl.kb, pl.kb, act_full);
       }
-      for (; ok && item < pl.items; item += gridDim.x, ++j) ok = issue(item, j);
+      if (lane == 0)
+        for (; ok && item < pl.items; item += gridDim.x, ++j) ok = issue(item, j);
     }
   } else {
     // ------------------------------------------------------- compute warps

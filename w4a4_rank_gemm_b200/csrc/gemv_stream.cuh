@@ -6,16 +6,18 @@
 // of four channels, so every SM streams the same number of weight bytes
 // (o_proj at 4096 channels: 24 or 28 channels per SM instead of one or two
 // 16-channel items).  Inside a CTA the range is covered by 16-channel tiles
-// and every tile by "units" of 256 k: 16 rows x 128 bytes of packed weights
-// (2 KB), first the residual's units (R, k < r) and then the main
-// product's.  The CTA's unit list, tile by tile, is cut into one contiguous
+// and every tile by "units" of 512 k: 16 rows x 256 bytes of packed weights
+// (4 KB), first the residual's units (R, k < r) and then the main
+// product's.  (The copy engine streams 16 x 256-byte boxes at the full HBM
+// rate but 16 x 128-byte boxes at about two thirds of it.)  The CTA's unit list, tile by tile, is cut into one contiguous
 // run per warp, so a warp moves to another tile (and hands its partial sums
 // over) at most a few times.
 //
 // Each warp streams its run through a private ring of kDepth slots: one
-// lane issues a unit as up to four TMA boxes of 4 rows x 128 bytes (boxes
-// past the CTA's range are skipped; bytes past a row's end are zero-filled)
-// completing on the slot's mbarrier, so the copy engine, not the load/store
+// lane issues a unit as one TMA box of 16 rows x 256 bytes, or as up to four
+// boxes of 4 rows x 256 bytes where the tile leaves the CTA's range or a
+// layer (boxes past the range are skipped; bytes past a row's end are
+// zero-filled), completing on the slot's mbarrier, so the copy engine, not the load/store
 // unit, carries the stream.  The first kDepth units are requested before
 // the kernel waits for the grid it depends on, since no earlier kernel
 // writes the weights.  The activation codes of all tokens and the CTA's
@@ -38,21 +40,21 @@
 // salient channels).
 //
 // A warp adds its partial sums of a tile into the tile's shared
-// accumulators when it moves on to another tile, then adds the number of
-// units it covered to the tile's counter; the warp that completes the count
-// applies the epilogue sx * (sw * acc0 + sR * acc1) for the tile's channels
-// and every token.  No warp waits for another.
+// accumulators when it moves on to another tile.  After the loop (one CTA
+// barrier) the warps share the epilogues sx * (sw * acc0 + sR * acc1), a
+// tile at a time, so that no warp's loop is lengthened by them.
 #pragma once
 #include "common.cuh"
 
 namespace serq {
 namespace gs {
 
-constexpr int kDepth = 4;         // ring slots per warp
-constexpr int kUnitK = 256;       // k per unit
-constexpr int kUnitBytes = 2048;  // 16 rows x 128 bytes
+constexpr int kDepth = 2;         // ring slots per warp
+constexpr int kUnitK = 512;       // k per unit
+constexpr int kUnitRow = 256;     // bytes of one weight row in a unit (a TMA box's inner extent)
+constexpr int kUnitBytes = 16 * kUnitRow;
 constexpr int kBoxRows = 4;       // rows per TMA box (the channel granularity of the CTA ranges)
-constexpr int kBoxBytes = kBoxRows * 128;
+constexpr int kBoxBytes = kBoxRows * kUnitRow;
 #ifndef SERQ_GS_WARPS
 #define SERQ_GS_WARPS 16
 #endif
@@ -174,7 +176,7 @@ struct Cursor {
 __device__ __forceinline__ void issue_unit(const Args& p, const Maps& mp, const Plan& pl, uint8_t* slot,
                                            uint64_t* bar, const Cursor& c, int c0, int c1) {
   const bool res = c.ku < pl.units_res;
-  const int x = (res ? c.ku : c.ku - pl.units_res) * 128;
+  const int x = (res ? c.ku : c.ku - pl.units_res) * kUnitRow;
   const int r0 = c0 + c.tile * 16;
   const int l0 = layer_of(p, r0);
   if (r0 + 16 <= c1 && r0 + 16 <= p.lo[l0].base + p.lo[l0].N) {
@@ -197,11 +199,11 @@ template <int NTT, bool A8>
 __device__ __forceinline__ void unit_mma(const uint8_t* slot, const uint8_t* xs, int xpitch, int xc0, int nch, int g,
                                          int t, int (&acc)[NTT][4]) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < kUnitRow / 64; ++h) {
     if (h < nch) {
       const int xc = xc0 + h;
-      const uint4 wg = *reinterpret_cast<const uint4*>(slot + g * 128 + h * 64 + 16 * t);
-      const uint4 wg8 = *reinterpret_cast<const uint4*>(slot + (g + 8) * 128 + h * 64 + 16 * t);
+      const uint4 wg = *reinterpret_cast<const uint4*>(slot + g * kUnitRow + h * 64 + 16 * t);
+      const uint4 wg8 = *reinterpret_cast<const uint4*>(slot + (g + 8) * kUnitRow + h * 64 + 16 * t);
       uint4 xa[NTT], xb[NTT];
 #pragma unroll
       for (int nt = 0; nt < NTT; ++nt) {
@@ -275,8 +277,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   uint8_t* xs = ring + pl.warps * kDepth * kUnitBytes;                // [xrows][xpitch]
   uint8_t* xr = xs + pl.xrows * pl.xpitch;                            // [xrows][xrpitch] (comparator only)
   int* acc = reinterpret_cast<int*>(xr + pl.xrows * pl.xrpitch);      // [tile][AccLayout]
-  int* cnt = acc + pl.tmax * AccLayout<NTT>::kInts;                   // [tile] units added
-  float* ssw = reinterpret_cast<float*>(cnt + ((pl.tmax + 3) & ~3));  // [cmax] sw of the CTA's channels
+  float* ssw = reinterpret_cast<float*>(acc + pl.tmax * AccLayout<NTT>::kInts);  // [cmax] sw of the CTA's channels
   float* ssr = ssw + pl.cmax;                                         // [cmax] sR
   float* ssx = ssr + pl.cmax;                                         // [xrows] sx
   float* ssxr = ssx + pl.xrows;                                       // [xrows] residual scale (comparator)
@@ -335,16 +336,18 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       }
     }
   }
-  // Shared accumulators and counters.
+  // Shared accumulators.
   for (int i = threadIdx.x; i < tiles * AccLayout<NTT>::kInts; i += blockDim.x) acc[i] = 0;
-  for (int i = threadIdx.x; i < tiles; i += blockDim.x) cnt[i] = 0;
   __syncthreads();    // barriers initialised, accumulators zero
   grid_dep_launch();  // the next kernel in the stream may be scheduled
   grid_dep_wait();    // activations, sx and the outputs come after the grid this one depends on
-  if (threadIdx.x == 0 && !pl.withhold_x) {
-    for (int m = 0; m < p.M; ++m) bulk_load(xs + m * pl.xpitch, p.Xq + (size_t)m * pl.xbytes, pl.xbytes, xbar);
-    if (pl.xrpitch)
-      for (int m = 0; m < p.M; ++m) bulk_load(xr + m * pl.xrpitch, p.Xr + (size_t)m * rbytes, rbytes, xbar);
+  if (lane == 0 && !pl.withhold_x) {
+    // one token row per warp, so the copies are issued side by side (the
+    // expected byte count was registered before the barrier above)
+    for (int m = warp; m < p.M; m += pl.warps) {
+      bulk_load(xs + m * pl.xpitch, p.Xq + (size_t)m * pl.xbytes, pl.xbytes, xbar);
+      if (pl.xrpitch) bulk_load(xr + m * pl.xrpitch, p.Xr + (size_t)m * rbytes, rbytes, xbar);
+    }
   }
   if (!ACC) {
     for (int i = threadIdx.x; i < p.M; i += blockDim.x) {
@@ -362,7 +365,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     for (int nt = 0; nt < NTT; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc0[nt][q] = acc1[nt][q] = 0;
-    int cur = -1, cur_units = 0;
+    int cur = -1;
     bool had0 = false, had1 = false;
 
     auto flush = [&]() {
@@ -375,18 +378,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
           if (had1) atomicAdd(&a[((1 * NTT + nt) * 4 + q) * 32 + lane], acc1[nt][q]);
           acc0[nt][q] = acc1[nt][q] = 0;
         }
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        __threadfence_block();
-        last = (atomicAdd(&cnt[cur], cur_units) + cur_units == ut);
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence_block();
-        tile_epilogue<NTT, A8, ACC>(p, a, c0 + cur * 16, c0, c1, ssw, ssr, ssx, ssxr, lane);
-      }
-      cur_units = 0;
       had0 = had1 = false;
     };
 
@@ -406,18 +397,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       const bool res = cc.ku < pl.units_res;
       const int kunit = res ? cc.ku : cc.ku - pl.units_res;
       const int left = (res ? kl_res : kl_main) - kunit * kUnitK;
-      const int nch = left >= 256 ? 2 : (left + 127) >> 7;
+      const int nch = min(kUnitRow / 64, (left + 127) >> 7);  // 128-k chunks with codes
       if (res) {
         if (pl.xrpitch)
-          unit_mma<NTT, A8>(slot, xr, pl.xrpitch, kunit * 2, nch, g, t, acc1);
+          unit_mma<NTT, A8>(slot, xr, pl.xrpitch, kunit * (kUnitK / 128), nch, g, t, acc1);
         else
-          unit_mma<NTT, A8>(slot, xs, pl.xpitch, kunit * 2, nch, g, t, acc1);
+          unit_mma<NTT, A8>(slot, xs, pl.xpitch, kunit * (kUnitK / 128), nch, g, t, acc1);
         had1 = true;
       } else {
-        unit_mma<NTT, A8>(slot, xs, pl.xpitch, kunit * 2, nch, g, t, acc0);
+        unit_mma<NTT, A8>(slot, xs, pl.xpitch, kunit * (kUnitK / 128), nch, g, t, acc0);
         had0 = true;
       }
-      ++cur_units;
       // refill this slot with the unit kDepth ahead once every lane has read it
       __syncwarp();
       if (j + kDepth < nw && lane == 0) {
@@ -429,6 +419,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     if (live && cur >= 0) flush();
   }
   __syncthreads();
+  // Every tile's sums are complete: the warps share the epilogues (one tile
+  // each in turn), so no warp's loop carries them.
+  if (ok && !*abort_flag)
+    for (int tile = warp; tile < tiles; tile += pl.warps)
+      tile_epilogue<NTT, A8, ACC>(p, acc + tile * AccLayout<NTT>::kInts, c0 + tile * 16, c0, c1, ssw, ssr, ssx,
+                                  ssxr, lane);
   if (*abort_flag && threadIdx.x == 0) {
     // let the copies already issued land before shared memory is released
     const unsigned long long t0 = global_ns();
@@ -444,11 +440,11 @@ inline bool make_plan(const Args& p, int sms, int max_smem, Plan& pl) {
   pl.xbytes = A8 ? p.K : p.K / 2;
   pl.units_main = (p.K + kUnitK - 1) / kUnitK;
   pl.units_res = (p.rpad + kUnitK - 1) / kUnitK;
-  const int xrow = pl.units_main * (A8 ? 256 : 128);  // whole units (bytes past K meet zero weights)
+  const int xrow = pl.units_main * (A8 ? kUnitK : kUnitK / 2);  // whole units (bytes past K meet zero weights)
   pl.xpitch = xrow + (A8 ? 16 : 64);                   // rows g, g + 1 in opposite bank halves
   pl.xrows = 8 * NTT;
   // comparator's residual codes: whole units, rows g, g + 1 in opposite bank halves
-  pl.xrpitch = (p.Xr && !A8) ? pl.units_res * 128 + 64 : 0;
+  pl.xrpitch = (p.Xr && !A8) ? pl.units_res * (kUnitK / 2) + 64 : 0;
   if (p.C > (1 << 21)) return false;  // keeps chan_begin in 32-bit arithmetic
   int grid = (p.C + 15) / 16;
   if (grid > sms) grid = sms;
@@ -462,7 +458,7 @@ inline bool make_plan(const Args& p, int sms, int max_smem, Plan& pl) {
   pl.cmax = most;
   pl.tmax = (most + 15) / 16;
   const int fixed = 128 + pl.xrows * (pl.xpitch + pl.xrpitch) + pl.tmax * AccLayout<NTT>::kInts * 4 +
-                    ((pl.tmax + 3) & ~3) * 4 + pl.cmax * 8 + pl.xrows * 8 + 8 + 16;
+                    pl.cmax * 8 + pl.xrows * 8 + 8 + 16;
   for (int w = kMaxWarps; w >= 4; w -= 4) {
     const int bytes = fixed + w * (kDepth * kUnitBytes + kDepth * 8);
     if (bytes <= max_smem) {

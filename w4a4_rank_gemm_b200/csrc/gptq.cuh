@@ -258,68 +258,61 @@ __global__ void k_upper_from_lower(const double* __restrict__ L2, int K, float* 
   if (U64) U64[e] = v;
 }
 
-// GPTQ on one weight, one thread per output channel n (rows in blocks of
-// 32, registers): the row values W^[i, n] as the round-to-nearest path sees
-// them, then
-//   code_i = clamp(rint(w_i * (7 / amax)), -7, 7)
-//   for i >= r:  e_i = (w_i - code_i * sw) / u_ii,  w_j -= u_ij * e_i (j > i)
-// with every fp32 operation rounded once and each w_j receiving its
-// updates in increasing i (earlier blocks' errors are applied when the
-// block is loaded, then the block's own rows in order).  amax is the
-// column's maximum before any update (sw = amax / 7).  The scaled errors of
-// rows >= r go to E (K x N).
-constexpr int kUStage = 64;  // rows of U staged per shared-memory pass
-
-__global__ void __launch_bounds__(128) k_gptq_pack_w(prep::WeightView w, const float* __restrict__ s,
-                                                      const int32_t* __restrict__ perm, int K, int r,
-                                                      const float* __restrict__ amax_col,
-                                                      const float* __restrict__ U, float* __restrict__ E,
-                                                      uint8_t* __restrict__ wq) {
-  __shared__ float Us[kUStage][33];
-  __shared__ float Ub[32][33];
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+// GPTQ on one weight.  A CTA owns 32 output channels; in each block of 32
+// rows, thread (t, lane) holds row b0 + t of channel n = 32 * blockIdx.x +
+// lane, starting from W^[b0 + t, n] as the round-to-nearest path computes it:
+//   1. the errors of the earlier rows i = r .. b0 - 1, in order:
+//      w -= u_{i, b0+t} * e_i;
+//   2. the block's rows in order: row t2 takes its code
+//      code = clamp(rint(w * (7 / amax)), -7, 7) and, when b0 + t2 >= r, its
+//      scaled error e = (w - code * sw) / u_{t2, t2}; the later rows of the
+//      block then lose u_{t2, t} * e;
+//   3. the 32 codes of each channel are packed as in the RTN path.
+// Each entry therefore receives its updates in increasing row order, every
+// fp32 operation rounded once.  amax is the column's maximum before any
+// update (sw = amax / 7).  E (K x N) keeps the scaled errors of rows >= r.
+__global__ void __launch_bounds__(1024) k_gptq_pack_w(prep::WeightView w, const float* __restrict__ s,
+                                                       const int32_t* __restrict__ perm, int K, int r,
+                                                       const float* __restrict__ amax_col,
+                                                       const float* __restrict__ U, float* __restrict__ E,
+                                                       uint8_t* __restrict__ wq) {
+  __shared__ float ub[32][33];  // U over the block's rows and columns
+  __shared__ float es[32][33];  // the block's scaled errors [row][channel]
+  __shared__ int qs[32][33];    // the block's codes [row][channel]
+  const int t = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * 32 + lane;
   const bool live = n < w.N;
   const float amax = live ? amax_col[n] : 0.f;
   const float sw = __fdiv_rn(amax, 7.f);
   for (int b0 = 0; b0 < K; b0 += 32) {
-    float x[32];
-#pragma unroll
-    for (int t = 0; t < 32; ++t) x[t] = live ? prep::w_hat(w, s, perm, b0 + t, n) : 0.f;
-    // errors of the rows before this block (rows r .. b0 - 1, in order)
-    for (int i0 = r; i0 < b0; i0 += kUStage) {
-      const int ni = min(kUStage, b0 - i0);
-      __syncthreads();
-      for (int e = threadIdx.x; e < kUStage * 32; e += blockDim.x) {
-        const int ii = e / 32, c = e % 32;
-        Us[ii][c] = (ii < ni) ? U[(size_t)(i0 + ii) * K + b0 + c] : 0.f;
-      }
-      __syncthreads();
-      if (live) {
-        for (int ii = 0; ii < ni; ++ii) {
-          const float e = E[(size_t)(i0 + ii) * w.N + n];
-#pragma unroll
-          for (int t = 0; t < 32; ++t) x[t] = __fsub_rn(x[t], __fmul_rn(Us[ii][t], e));
+    float x = live ? prep::w_hat(w, s, perm, b0 + t, n) : 0.f;
+    if (live) {
+      const float* ucol = U + b0 + t;  // u_{i, b0+t}: the same for the whole warp
+#pragma unroll 8
+      for (int i = r; i < b0; ++i) x = __fsub_rn(x, __fmul_rn(ucol[(size_t)i * K], E[(size_t)i * w.N + n]));
+    }
+    ub[t][lane] = U[(size_t)(b0 + t) * K + b0 + lane];
+    __syncthreads();
+    for (int t2 = 0; t2 < 32; ++t2) {
+      if (t == t2) {
+        const int q = prep::code4(x, amax);
+        qs[t][lane] = q;
+        if (b0 + t >= r) {
+          const float err = __fdiv_rn(__fsub_rn(x, __fmul_rn((float)q, sw)), ub[t][t]);
+          es[t][lane] = err;
+          if (live) E[(size_t)(b0 + t) * w.N + n] = err;
         }
       }
+      __syncthreads();
+      if (t > t2 && b0 + t2 >= r) x = __fsub_rn(x, __fmul_rn(ub[t2][t], es[t2][lane]));
+    }
+    if (t == 0 && live) {
+      int q[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) q[k] = qs[k][lane];
+      *reinterpret_cast<uint4*>(wq + (size_t)n * (K / 2) + b0 / 2) = prep::pack_run32(q);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < 32 * 32; e += blockDim.x) {
-      const int rr = e / 32, c = e % 32;
-      Ub[rr][c] = U[(size_t)(b0 + rr) * K + b0 + c];
-    }
-    __syncthreads();
-    int q[32];
-#pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      q[t] = prep::code4(x[t], amax);
-      if (b0 + t >= r) {
-        const float err = __fdiv_rn(__fsub_rn(x[t], __fmul_rn((float)q[t], sw)), Ub[t][t]);
-        if (live) E[(size_t)(b0 + t) * w.N + n] = err;
-#pragma unroll
-        for (int t2 = t + 1; t2 < 32; ++t2) x[t2] = __fsub_rn(x[t2], __fmul_rn(Ub[t][t2], err));
-      }
-    }
-    if (live) *reinterpret_cast<uint4*>(wq + (size_t)n * (K / 2) + b0 / 2) = prep::pack_run32(q);
   }
 }
 

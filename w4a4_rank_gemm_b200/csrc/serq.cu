@@ -108,8 +108,8 @@ struct serq_layer {
   float* smooth;
   CUtensorMap tmB[3];  // box rows 128, 256, 96
   CUtensorMap tmR[3];
-  CUtensorMap tmW4, tmR4;    // 128-byte x 4-row boxes (streaming decode kernel)
-  CUtensorMap tmW16, tmR16;  // 128-byte x 16-row boxes (streaming decode kernel)
+  CUtensorMap tmW4, tmR4;    // 256-byte x 4-row boxes (streaming decode kernel)
+  CUtensorMap tmW16, tmR16;  // 256-byte x 16-row boxes (streaming decode kernel)
   int32_t* ws;         // split-K partial sums of the tensor-core decode, zero between calls
   int32_t* cnt;        // per 128-row tile: units done
 };
@@ -186,15 +186,15 @@ bool build_weight_maps(serq_layer* L) {
       L->tmR[i] = L->tmB[i];  // never read when r = 0
     }
   }
-  if (!make_map(&L->tmW4, L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 128, 4,
+  if (!make_map(&L->tmW4, L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 256, 4,
                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&L->tmW16, L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 128, 16,
+      !make_map(&L->tmW16, L->wq, (uint64_t)L->K / 2, (uint64_t)L->N, (uint64_t)L->K / 2, 256, 16,
                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   if (L->rpad) {
-    if (!make_map(&L->tmR4, L->rq, (uint64_t)L->rpad / 2, (uint64_t)L->N, (uint64_t)L->rpad / 2, 128, 4,
+    if (!make_map(&L->tmR4, L->rq, (uint64_t)L->rpad / 2, (uint64_t)L->N, (uint64_t)L->rpad / 2, 256, 4,
                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&L->tmR16, L->rq, (uint64_t)L->rpad / 2, (uint64_t)L->N, (uint64_t)L->rpad / 2, 128, 16,
+        !make_map(&L->tmR16, L->rq, (uint64_t)L->rpad / 2, (uint64_t)L->N, (uint64_t)L->rpad / 2, 256, 16,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
       return false;
   } else {
@@ -934,8 +934,8 @@ serq_status prepare_impl(int n_weights, const float* const* W, const int* N, int
     k_colmax_what<<<dim3((Ni + 255) / 256, (K + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(
         v, L0->smooth, L0->perm, K, rows_per_block, Li->sw);
     if (o.quantizer == SERQ_QUANT_GPTQ)
-      serq::gptq::k_gptq_pack_w<<<(Ni + 127) / 128, 128, 0, st>>>(v, L0->smooth, L0->perm, K, rank, Li->sw, U32, E,
-                                                                  Li->wq);
+      serq::gptq::k_gptq_pack_w<<<(Ni + 31) / 32, 1024, 0, st>>>(v, L0->smooth, L0->perm, K, rank, Li->sw, U32, E,
+                                                                 Li->wq);
     else
       k_quant_pack_w<<<dim3((Ni + 127) / 128, K / 32), 128, 0, st>>>(v, L0->smooth, L0->perm, K, Li->sw, Li->wq);
     if (rank > 0) {
