@@ -246,7 +246,8 @@ class LayerWorkload:
         self.gemm_bytes_step = sum(linear_bytes(M, K, N, r, self.a_bits) for _, K, N in self.gemms)
         self.decode = M <= S.decode_max_m()
         n_gemm_launches = len(self.grp) if self.grouped else len(self.gemms)
-        self.launches_per_step = len(self.grp) + n_gemm_launches
+        n_quant = sum(0 if self.fused(i, ps) else 1 for i, ps in self.grp)
+        self.launches_per_step = n_quant + n_gemm_launches
         self.weight_mb = sum(p.W.size for p in wl.projections) / 2 / 1e6
 
     def describe(self):
@@ -254,10 +255,22 @@ class LayerWorkload:
         return (f"{self.name}_{self.mode}_r{self.r}: one decoder layer's {len(self.gemms)} projections "
                 f"({shapes}), {len(self.grp)} shared-input quantizes, M = {self.M} tokens per GPU")
 
+    def fused(self, iname, projs):
+        """Whether the group runs as one serq_linear_group_act launch (M <= 8,
+        K <= 4096: the GEMV quantizes the tokens itself)."""
+        return self.decode and self.M <= 8 and self.grouped and self.wl.inputs[iname].K <= 4096
+
     def step(self, i, stream, events=None, gemm_only=False):
         S, torch = self.S, self.torch
         c, a = i % N_WEIGHT_COPIES, i % N_ACT_COPIES
         for iname, projs in self.grp:
+            if self.fused(iname, projs):
+                # one launch, quantize included (also in the GEMM-only graph:
+                # it is the GEMV launch of this group)
+                S.linear_group_act([self.layers[c][p.name] for p in projs], self.flat[iname][a],
+                                   Ys=[self.Y[p.name] for p in projs], Xq=self.Xq[iname], sx=self.sx[iname],
+                                   algo=self.algo, stream=stream)
+                continue
             if not gemm_only:
                 S.quantize_act(self.flat[iname][a], self.mode, Xq=self.Xq[iname], sx=self.sx[iname], stream=stream)
             for name, ps in self._launches(projs):
@@ -307,6 +320,11 @@ class LayerWorkload:
         self.Y = self.Ybuf[b]
         try:
             for iname, projs in self.grp:
+                if self.fused(iname, projs):
+                    S.linear_group_act([self.layers[c][p.name] for p in projs], self.flat[iname][b],
+                                       Ys=[self.Y[p.name] for p in projs], Xq=self.Xq[iname], sx=self.sx[iname],
+                                       algo=self.algo, stream=stream)
+                    continue
                 S.quantize_act(self.flat[iname][b], self.mode, Xq=self.Xq[iname], sx=self.sx[iname], stream=stream)
                 for _, ps in self._launches(projs):
                     self._linear(c, iname, ps, stream)
@@ -533,8 +551,9 @@ def run_gpu(args, rank, world, local_rank):
         peak = pk.get("hbm_gbs")
         achieved = W.gemm_bytes_step * roof_steps / (gemm_ms / 1e3) / 1e9
         res["roofline"] = {
-            "kernel": ("decode GEMVs, main + residual accumulators: serq::gs::k_gemv (streaming; q/k/v, gate/up, "
-                       "down) and serq::decode::k_decode (item ring; o_proj)"),
+            "kernel": ("decode GEMVs, main + residual accumulators: serq::gs::k_gemv (streaming; at M <= 8 and "
+                       "K <= 4096 (q/k/v, o, gate/up) one launch that also quantizes the tokens) and "
+                       "serq::decode::k_decode (item ring; o_proj at larger M)"),
             "bound": "hbm", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "traffic": recorded_traffic(f"{W.name}_M{W.M}", ["gemv_stream.cuh", "gemv_decode.cuh", "common.cuh"]),

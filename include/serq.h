@@ -332,6 +332,29 @@ serq_status serq_linear_group(int n, const serq_layer* const* layers, const void
                               int32_t* const* acc1, serq_algo algo, void* stream);
 
 /*
+ * serq_linear_group_act -- serq_quantize_act followed by serq_linear_group,
+ * from the flattened, permuted activations X^ (the token rows the layers
+ * consume).  For few tokens (the decode kernels chosen, bf16 input, M <= 8,
+ * K <= 4096) it is ONE launch: every CTA of the streaming decode kernel
+ * quantizes the M rows itself (the per-token symmetric quantizer of
+ * serq_quantize_act, same arithmetic, same codes) into the shared-memory
+ * rows its MMAs read, so the codes never go through HBM and the quantize
+ * launch and its dependency on the step before leave the critical path.
+ * Otherwise (where every CTA reading all M bf16 rows would cost more than
+ * the launch it saves) it runs the two calls one after the other.
+ *  X, dtype, ldx  DEVICE M x K activations (bf16 or fp32), row stride ldx,
+ *           rows 16-byte aligned.
+ *  Xq, sx   DEVICE scratch with the sizes serq_quantize_act writes (M x K/2
+ *           bytes for W4A4, M x K for W4A8; M floats); written when the call
+ *           quantizes in a launch of its own, contents unspecified after.
+ *  the rest as serq_linear_group.
+ * Asynchronous.  Errors: those of serq_quantize_act and serq_linear_group.
+ */
+serq_status serq_linear_group_act(int n, const serq_layer* const* layers, const void* X, serq_dtype dtype,
+                                  int ldx, int M, void* Xq, float* sx, void* const* Y, const int* ldy,
+                                  int32_t* const* acc0, int32_t* const* acc1, serq_algo algo, void* stream);
+
+/*
  * serq_linear_decode_static -- serq_linear (or, with acc0/acc1, the
  * accumulator hook) through the tensor-core decode kernel
  * (SERQ_ALGO_DECODE_TC) with its split-K partial sums and tile counters in a

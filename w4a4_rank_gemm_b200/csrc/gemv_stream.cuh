@@ -45,6 +45,7 @@
 // tile at a time, so that no warp's loop is lengthened by them.
 #pragma once
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace serq {
 namespace gs {
@@ -83,6 +84,12 @@ struct Args {
   // whose residual reuses the first r columns of Xq.
   const uint8_t* Xr;
   const float* sxr;
+  // Fused activation quantize (null: Xq and sx are given): the flattened,
+  // permuted bf16 activations, M x K at row stride ldxh, quantized per token
+  // by the CTA itself (every CTA, the same codes) into the staged rows; K <=
+  // 4096 (one warp holds a row in registers).
+  const __nv_bfloat16* Xh;
+  int ldxh;
   int M, K, rpad;
   int C;     // channels of the launch (all layers)
   int nlayers;
@@ -90,8 +97,8 @@ struct Args {
 };
 
 // Per layer: the weight and the compensator as 2-D byte tensors (rows =
-// output channels) read in 128-byte x 16-row boxes (a whole unit) and in
-// 128-byte x 4-row boxes (the last, partial tile of a CTA's range, or a
+// output channels) read in 256-byte x 16-row boxes (a whole unit) and in
+// 256-byte x 4-row boxes (the last, partial tile of a CTA's range, or a
 // tile across a layer boundary).
 struct Maps {
   CUtensorMap w[kMaxGroup];
@@ -190,6 +197,58 @@ __device__ __forceinline__ void issue_unit(const Args& p, const Maps& mp, const 
     const int ch = r0 + b * kBoxRows;
     const int l = layer_of(p, ch);
     tma_load_2d(slot + b * kBoxBytes, res ? &mp.r[l] : &mp.w[l], bar, x, ch - p.lo[l].base);
+  }
+}
+
+// Per-token quantize of one bf16 row by one warp into the staged layout
+// (packed INT4 runs of 16 bytes, or INT8 codes), with the arithmetic of the
+// standalone quantizer (quant::quantize_run): lane l owns the runs l, l + 32,
+// l + 64, l + 96 (K <= 4096) and holds them in registers between the
+// absolute maximum and the codes.
+template <int Q>
+__device__ __forceinline__ void quantize_row_warp(const __nv_bfloat16* row, int K, uint8_t* dst, float* sx_out,
+                                                  int lane) {
+  const int nrun = K >> 5;
+  uint4 raw[4][4];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int b = lane + 32 * i;
+    if (b < nrun)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) raw[i][c] = __ldg(reinterpret_cast<const uint4*>(row + b * 32 + c * 8));
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int b = lane + 32 * i;
+    if (b < nrun)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[8];
+        quant::LoadBF16::bf16x8(raw[i][c], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+      }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float qf = (float)Q;
+  const float inv = (amax > 0.f) ? __fdiv_rn(qf, amax) : 0.f;
+  if (lane == 0) *sx_out = __fdiv_rn(amax, qf);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int b = lane + 32 * i;
+    if (b < nrun) {
+      float v[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float u[8];
+        quant::LoadBF16::bf16x8(raw[i][c], u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[c * 8 + e] = u[e];
+      }
+      quant::quantize_run<Q>(v, inv, reinterpret_cast<uint4*>(dst + (Q == 7 ? 16 : 32) * b));
+    }
   }
 }
 
@@ -321,7 +380,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   }
   const uint32_t rbytes = (uint32_t)(p.rpad >> 1);
   if (threadIdx.x == 0 && !pl.withhold_x) {
-    uint32_t tx = (uint32_t)(p.M * pl.xbytes) + (pl.xrpitch ? (uint32_t)p.M * rbytes : 0u);
+    uint32_t tx = p.Xh ? 0u : (uint32_t)(p.M * pl.xbytes) + (pl.xrpitch ? (uint32_t)p.M * rbytes : 0u);
     if (!ACC) tx += 8u * (uint32_t)(c1 - c0);
     mbar_arrive_expect_tx(xbar, tx);
     if (!ACC) {
@@ -341,7 +400,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   __syncthreads();    // barriers initialised, accumulators zero
   grid_dep_launch();  // the next kernel in the stream may be scheduled
   grid_dep_wait();    // activations, sx and the outputs come after the grid this one depends on
-  if (lane == 0 && !pl.withhold_x) {
+  if (p.Xh) {
+    // the CTA quantizes the tokens itself, one warp per row
+    for (int m = warp; m < p.M; m += pl.warps)
+      quantize_row_warp<A8 ? 127 : 7>(p.Xh + (size_t)m * p.ldxh, p.K, xs + m * pl.xpitch, ssx + m, lane);
+  } else if (lane == 0 && !pl.withhold_x) {
     // one token row per warp, so the copies are issued side by side (the
     // expected byte count was registered before the barrier above)
     for (int m = warp; m < p.M; m += pl.warps) {
@@ -349,7 +412,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       if (pl.xrpitch) bulk_load(xr + m * pl.xrpitch, p.Xr + (size_t)m * rbytes, rbytes, xbar);
     }
   }
-  if (!ACC) {
+  if (!ACC && !p.Xh) {
     for (int i = threadIdx.x; i < p.M; i += blockDim.x) {
       ssx[i] = __ldg(p.sx + i);
       if (p.sxr) ssxr[i] = __ldg(p.sxr + i);

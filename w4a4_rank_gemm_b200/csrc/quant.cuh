@@ -112,15 +112,52 @@ struct LoadSiluMul {
   }
 };
 
+// ------------------------------------------------ codes of one 32-code run
+// code = clamp(rint(x * inv), -Q, Q).  |x| <= amax and inv = RN(Q/amax)
+// give |RN(x * inv)| <= Q (1 + 2^-23), which rounds to at most Q, so the
+// clamp never binds.  Adding 1.5 * 2^23 rounds to the nearest integer
+// (ties to even) exactly for |y| < 2^22, and the sum's low mantissa bits
+// are then the code in two's complement: a nibble or byte is a mask away.
+// (The product and the sum stay two roundings; a fused multiply-add would
+// round differently at ties.)
+//
+// Output, Q = 7: the packed INT4 format, every run of 32 codes is 16 bytes
+// (dst[0]) with byte j = code j (low nibble) | code j+16 (high nibble).
+// Q = 127: int8 codes in natural order (dst[0], dst[1]).
+template <int Q>
+__device__ __forceinline__ void quantize_run(const float (&v)[32], float inv, uint4* dst) {
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23
+  uint32_t t[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__fadd_rn(__fmul_rn(v[e], inv), kMagic));
+  if (Q == 7) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x |= ((t[4 * k + j] & 0xFu) | ((t[4 * k + j + 16] & 0xFu) << 4)) << (8 * j);
+      w[k] = x;
+    }
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    uint32_t w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      w[j] = __byte_perm(__byte_perm(t[4 * j], t[4 * j + 1], 0x0040), __byte_perm(t[4 * j + 2], t[4 * j + 3], 0x0040),
+                         0x5410);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
 // ------------------------------------------------------- quantize one row
 // One CTA per token row; lane l of warp w owns the 32-code runs
 // b = l + 32 (w + W i), i < RPL, and holds their raw input in registers, so
 // HBM sees the row once: load everything, reduce the absolute maximum
 // (shuffles, then shared memory across the W warps), quantize from registers.
 //
-// Output, Q = 7: the packed INT4 format, every run of 32 codes is 16 bytes
-// with byte j = code j (low nibble) | code j+16 (high nibble).  Q = 127: int8
-// codes in natural order.
+// Codes as quantize_run writes them.
 template <int Q, int RPL, class Loader>
 __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* __restrict__ Xq,
                                                     float* __restrict__ sx, int early_launch) {
@@ -173,49 +210,20 @@ __global__ void __launch_bounds__(256) k_quant_rows(Loader ld, int K, uint8_t* _
   const float inv = (amax > 0.f) ? __fdiv_rn(qf, amax) : 0.f;
   if (threadIdx.x == 0) sx[m] = __fdiv_rn(amax, qf);
 
-  // code = clamp(rint(x * inv), -Q, Q).  |x| <= amax and inv = RN(Q/amax)
-  // give |RN(x * inv)| <= Q (1 + 2^-23), which rounds to at most Q, so the
-  // clamp never binds.  Adding 1.5 * 2^23 rounds to the nearest integer
-  // (ties to even) exactly for |y| < 2^22, and the sum's low mantissa bits
-  // are then the code in two's complement: a nibble or byte is a mask away.
-  // (The product and the sum stay two roundings; a fused multiply-add would
-  // round differently at ties.)
-  const float kMagic = 12582912.0f;  // 1.5 * 2^23
 #pragma unroll
   for (int i = 0; i < RPL; ++i) {
     const int b = lane + 32 * (warp + nw * i);
     if (b >= nrun) continue;
-    uint32_t t[32];
+    float v[32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      float v[8];
-      ld.value(raw[i][c], v);
+      float u[8];
+      ld.value(raw[i][c], u);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        t[c * 8 + e] = __float_as_uint(__fadd_rn(__fmul_rn(v[e], inv), kMagic));
-      }
+      for (int e = 0; e < 8; ++e) v[c * 8 + e] = u[e];
     }
-    if (Q == 7) {
-      uint32_t w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t x = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          x |= ((t[4 * k + j] & 0xFu) | ((t[4 * k + j + 16] & 0xFu) << 4)) << (8 * j);
-        w[k] = x;
-      }
-      *reinterpret_cast<uint4*>(Xq + (size_t)m * (K >> 1) + b * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-      uint32_t w[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        w[j] = __byte_perm(__byte_perm(t[4 * j], t[4 * j + 1], 0x0040), __byte_perm(t[4 * j + 2], t[4 * j + 3], 0x0040),
-                           0x5410);
-      uint4* dst = reinterpret_cast<uint4*>(Xq + (size_t)m * K + b * 32);
-      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    }
+    uint8_t* dst = (Q == 7) ? Xq + (size_t)m * (K >> 1) + b * 16 : Xq + (size_t)m * K + b * 32;
+    quantize_run<Q>(v, inv, reinterpret_cast<uint4*>(dst));
   }
   if (!early_launch) grid_dep_launch();
 }

@@ -430,9 +430,15 @@ cudaError_t dispatch_tc(const LinearGroup& G, const void* Xq, const float* sx, i
 // else the item ring: for a share of one or two 16-channel items per SM its
 // simpler start-up is measured faster), 1 = item ring, 2 = streaming where
 // it fits.  fault_wait_ns is zero except in the failure-detection test hook.
+// Xh (bf16, K <= 4096, else null): the activations still to be quantized;
+// the streaming kernel quantizes them itself, the item ring after a
+// quantize launch into Xq / sx (then scratch the caller provided).
 cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const float* sx, int M, bool a8, bool accum,
-                                int kind, cudaStream_t st, unsigned long long fault_wait_ns = 0) {
-  if (kind == 0) {
+                                int kind, cudaStream_t st, unsigned long long fault_wait_ns = 0,
+                                const __nv_bfloat16* Xh = nullptr, int ldxh = 0) {
+  if (Xh && kind == 0) {
+    kind = 2;  // one launch: the quantize lives in the streaming kernel
+  } else if (kind == 0) {
     double bytes = 0;
     for (int l = 0; l < G.n; ++l) bytes += (double)G.L[l]->N * (G.L[l]->K / 2 + G.L[l]->rpad / 2);
     kind = (bytes >= 96.0 * 1024 * sm_count() || fault_wait_ns) ? 2 : 1;
@@ -442,6 +448,8 @@ cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const floa
     serq::gs::Maps mp;
     g.Xq = static_cast<const uint8_t*>(Xq);
     g.sx = sx;
+    g.Xh = Xh;
+    g.ldxh = ldxh;
     g.M = M;
     g.K = G.L[0]->K;
     g.rpad = G.L[0]->rpad;
@@ -468,6 +476,14 @@ cudaError_t launch_decode_group(const LinearGroup& G, const void* Xq, const floa
                    : serq::gs::launch<false, false>(g, mp, sm_count(), max_smem(), st, fault_wait_ns);
     }
     if (fault_wait_ns) return cudaErrorInvalidValue;
+  }
+  if (Xh) {
+    const serq::quant::LoadBF16 ld{Xh, ldxh};
+    uint8_t* q = static_cast<uint8_t*>(const_cast<void*>(Xq));
+    float* sq = const_cast<float*>(sx);
+    const cudaError_t e = a8 ? serq::quant::launch_quant_rows<127>(ld, M, G.L[0]->K, q, sq, st)
+                             : serq::quant::launch_quant_rows<7>(ld, M, G.L[0]->K, q, sq, st);
+    if (e != cudaSuccess) return e;
   }
   serq::decode::Args a = {};
   a.Xq = static_cast<const uint8_t*>(Xq);
@@ -578,7 +594,7 @@ serq_status linear_impl(const serq_layer* L, const void* Xq, const float* sx, in
 // variant run them one launch per layer.
 serq_status group_impl(int n, const serq_layer* const* Ls, const void* Xq, const float* sx, int M,
                        void* const* Y, const int* ldy, int32_t* const* acc0, int32_t* const* acc1, serq_algo algo,
-                       void* stream) {
+                       void* stream, const __nv_bfloat16* Xh = nullptr, int ldxh = 0) {
   serq_status s;
   if (n < 1 || n > serq::tc::kMaxGroup)
     return fail(SERQ_ERR_INVALID_ARG, "group of %d layers (1..%d)", n, serq::tc::kMaxGroup);
@@ -616,7 +632,7 @@ serq_status group_impl(int n, const serq_layer* const* Ls, const void* Xq, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (resolved == SERQ_ALGO_DECODE || resolved == SERQ_ALGO_DECODE_ITEMS || resolved == SERQ_ALGO_DECODE_STREAM) {
-    e = launch_decode_group(G, Xq, sx, M, Ls[0]->mode == SERQ_W4A8, accum, decode_kind(resolved), st);
+    e = launch_decode_group(G, Xq, sx, M, Ls[0]->mode == SERQ_W4A8, accum, decode_kind(resolved), st, 0, Xh, ldxh);
     if (e != cudaSuccess) return cuda_fail(e, "serq_linear_group launch");
     return ok();
   }
@@ -1207,6 +1223,30 @@ serq_status serq_linear_accum(const serq_layer* layer, const void* Xq, int M, in
 serq_status serq_linear_group(int n, const serq_layer* const* layers, const void* Xq, const float* sx, int M,
                               void* const* Y, const int* ldy, int32_t* const* acc0, int32_t* const* acc1,
                               serq_algo algo, void* stream) {
+  return group_impl(n, layers, Xq, sx, M, Y, ldy, acc0, acc1, algo, stream);
+}
+
+serq_status serq_linear_group_act(int n, const serq_layer* const* layers, const void* X, serq_dtype dtype, int ldx,
+                                  int M, void* Xq, float* sx, void* const* Y, const int* ldy, int32_t* const* acc0,
+                                  int32_t* const* acc1, serq_algo algo, void* stream) {
+  serq_status s;
+  if (n < 1 || n > serq::tc::kMaxGroup || !layers || !layers[0])
+    return fail(SERQ_ERR_INVALID_ARG, "null layer list or a group of %d layers", n);
+  if (dtype != SERQ_F32 && dtype != SERQ_BF16) return fail(SERQ_ERR_INVALID_ARG, "bad dtype");
+  const int K = layers[0]->K;
+  if ((s = check_rows(X, M, K, ldx, dtype == SERQ_F32 ? 4 : 2, "X"))) return s;
+  if (!Xq || !sx) return fail(SERQ_ERR_INVALID_ARG, "null Xq or sx (scratch)");
+  serq_algo a = algo;
+  if (a == SERQ_ALGO_AUTO) a = (M <= serq_decode_max_m()) ? SERQ_ALGO_DECODE : SERQ_ALGO_PREFILL;
+  const bool decode = a == SERQ_ALGO_DECODE || a == SERQ_ALGO_DECODE_STREAM || a == SERQ_ALGO_DECODE_ITEMS;
+  // One launch pays off for few tokens: every CTA reads all M bf16 rows
+  // (M x K x 2 bytes from L2) before its loop, which at M = 16 already costs
+  // more than the quantize launch it saves (measured on the 7B decode step:
+  // 1-3% faster for M <= 8, 2% slower at 16, 11% at 32).
+  if (dtype == SERQ_BF16 && K <= 4096 && M <= 8 && decode)
+    return group_impl(n, layers, Xq, sx, M, Y, ldy, acc0, acc1, algo, stream,
+                      static_cast<const __nv_bfloat16*>(X), ldx);
+  if ((s = serq_quantize_act(X, dtype, M, K, ldx, static_cast<serq_mode>(layers[0]->mode), Xq, sx, stream))) return s;
   return group_impl(n, layers, Xq, sx, M, Y, ldy, acc0, acc1, algo, stream);
 }
 

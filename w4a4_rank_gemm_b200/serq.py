@@ -60,6 +60,8 @@ EXPORTS = {
     "serq_linear_decode_static": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp]),
     "serq_linear_group": (_i, [_i, ctypes.POINTER(_vp), _vp, _vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_i),
                                ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp]),
+    "serq_linear_group_act": (_i, [_i, ctypes.POINTER(_vp), _vp, _i, _i, _i, _vp, _vp, ctypes.POINTER(_vp),
+                                   ctypes.POINTER(_i), ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp]),
     "serq_l2qer_prepare": (_i, [_vp, _vp, _vp, _i, ctypes.POINTER(_vp)]),
     "serq_l2qer_destroy": (None, [_vp]),
     "serq_l2qer_get_packed": (_i, [_vp, _vp, _vp, _vp, _vp]),
@@ -381,6 +383,39 @@ def linear_group(layers, Xq: torch.Tensor, sx: Optional[torch.Tensor] = None, Ys
     ld = (_i * n)(*[Y.stride(0) for Y in Ys])
     _check(lib.serq_linear_group(n, hl, _ptr(Xq), _ptr(sx), M, yp, ld, None, None, algo, _stream(stream)),
            "serq_linear_group")
+    return Ys
+
+
+def linear_group_act(layers, X: torch.Tensor, Ys=None, Xq: Optional[torch.Tensor] = None,
+                     sx: Optional[torch.Tensor] = None, algo: int = ALGO_AUTO, accum: bool = False, stream=None):
+    """serq_linear_group_act: quantize the flattened activations X (bf16 or
+    fp32, M x K) and run the group's products; one launch at decode sizes.
+    Xq / sx are scratch (allocated here when not given).  Returns the bf16
+    outputs, or (acc0, acc1) pairs when accum."""
+    n = len(layers)
+    M, K = X.shape
+    if X.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("X must be bf16 or fp32")
+    dt = BF16 if X.dtype == torch.bfloat16 else F32
+    if Xq is None:
+        Xq = torch.empty((M, K // 2 if layers[0].mode == W4A4 else K), dtype=torch.uint8, device=X.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=X.device)
+    hl = (_vp * n)(*[L.handle for L in layers])
+    if accum:
+        accs = [(torch.empty((M, L.N), dtype=torch.int32, device=X.device),
+                 torch.empty((M, L.N), dtype=torch.int32, device=X.device)) for L in layers]
+        a0 = (_vp * n)(*[_ptr(a[0]) for a in accs])
+        a1 = (_vp * n)(*[_ptr(a[1]) for a in accs])
+        _check(lib.serq_linear_group_act(n, hl, _ptr(X), dt, X.stride(0), M, _ptr(Xq), _ptr(sx), None, None, a0, a1,
+                                         algo, _stream(stream)), "serq_linear_group_act")
+        return accs
+    if Ys is None:
+        Ys = [torch.empty((M, L.N), dtype=torch.bfloat16, device=X.device) for L in layers]
+    yp = (_vp * n)(*[_ptr(Y) for Y in Ys])
+    ld = (_i * n)(*[Y.stride(0) for Y in Ys])
+    _check(lib.serq_linear_group_act(n, hl, _ptr(X), dt, X.stride(0), M, _ptr(Xq), _ptr(sx), yp, ld, None, None,
+                                     algo, _stream(stream)), "serq_linear_group_act")
     return Ys
 
 
