@@ -729,10 +729,15 @@ def run_compare(args):
         sum_main += t0
         sum_serq += t1 - t0
         sum_two += t2 - t0
-    ratio = sum_two / max(sum_serq, 1e-3)
+    # SERQ's residual rides in the main launch; where its added time is below
+    # the timings' noise (1% of the main products: run-to-run spread of
+    # these event timings) the ratio uses that floor, and says so.
+    floor = 0.01 * sum_main
+    ratio = sum_two / max(sum_serq, floor)
     return {
         "metric": "residual-path latency: two-factor comparator (L2QER) / SERQ, one Llama-2-7B layer",
         "value": round(ratio, 3), "unit": "x", "higher_is_better": True, "n_gpus": 1,
+        "serq_residual_at_noise_floor": sum_serq < floor,
         "steps": reps, "warmup": 3, "ms_per_step": round((sum_main + sum_serq) / 1e3, 4),
         "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 (W4A4 codes, int32 accumulate)",
