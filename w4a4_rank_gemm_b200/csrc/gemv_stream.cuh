@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     k_gemv(const __grid_constant__ Args p, const __grid_constant__ Maps mp, const Plan pl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  uint8_t* ring = sm;                                                 // [warp][slot][16 rows][128 B]
+  uint8_t* ring = sm;                                                 // [warp][slot][16 rows][256 B]
   uint8_t* xs = ring + pl.warps * kDepth * kUnitBytes;                // [xrows][xpitch]
   uint8_t* xr = xs + pl.xrows * pl.xpitch;                            // [xrows][xrpitch] (comparator only)
   int* acc = reinterpret_cast<int*>(xr + pl.xrows * pl.xrpitch);      // [tile][AccLayout]
