@@ -125,3 +125,16 @@ def test_linear_on_a_gptq_layer(S, M, mode):
     assert np.array_equal(g0.cpu().numpy(), acc0) and np.array_equal(g1.cpu().numpy(), acc1)
     assert_y_close(S.linear(L, Xq, sx), O.linear_epilogue(acc0, acc1, osx, ol))
     assert S.device_error() == 0
+
+
+def test_prepare_gptq_with_output_fold(S):
+    # the next layer's order and smoothing scales folded into the output
+    # columns (SERQ notes, key design 3) before GPTQ runs on the folded weight
+    rng = np.random.default_rng(12)
+    K, N, r = 256, 192, 32
+    Xc = _calib(rng, 64, K)
+    W = (0.05 * rng.standard_normal((K, N))).astype(np.float32)
+    P = rng.permutation(N).astype(np.int32)
+    d = rng.uniform(0.2, 5.0, N).astype(np.float32)
+    L = S.prepare_host(W, Xc, rank=r, out_perm=P, out_colscale=d, quantizer="gptq")
+    _check_prepared(L, G.prepare(O.fold_output_columns(W, P, d), Xc, r))

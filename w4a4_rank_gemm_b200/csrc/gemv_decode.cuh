@@ -237,9 +237,11 @@ __global__ void __launch_bounds__(kThreads, (!A8 && MT == 1) ? 2 : 1) k_decode(c
         bulk_load(sc + kRows * 4, lo.sr + n0, kRows * 4, &full[s]);
         return true;
       };
-      // weights first: no earlier kernel writes them
+      // weights first: no earlier kernel writes them.  One item before the
+      // dependency wait, the rest after the activation copies, which would
+      // otherwise queue behind every SM's whole prefetch.
       if (lane == 0)
-        for (; ok && item < pl.items && j < pl.stages; item += gridDim.x, ++j) ok = issue(item, j);
+        for (; ok && item < pl.items && j < 1; item += gridDim.x, ++j) ok = issue(item, j);
       grid_dep_wait();
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (ok && ACT_SMEM) {
