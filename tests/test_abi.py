@@ -141,6 +141,20 @@ def test_group_call_host_side_rejection(lib):
     layers[0] = None
     assert L.serq_linear_group(2, layers, fake, fake, 16, ys, ld, None, None, 0, None) == lib.ERR_INVALID_ARG
     assert b"null layer 0" in L.serq_last_error_string()
+    # the quantize-and-linear call: group size, null list or first layer, dtype
+    layers[0] = 0x1000
+    for n in (0, 5):
+        assert L.serq_linear_group_act(n, layers, fake, lib.BF16, 256, 8, fake, fake, ys, ld, None, None, 0,
+                                       None) == lib.ERR_INVALID_ARG
+    assert L.serq_linear_group_act(2, None, fake, lib.BF16, 256, 8, fake, fake, ys, ld, None, None, 0,
+                                   None) == lib.ERR_INVALID_ARG
+    layers[0] = None
+    assert L.serq_linear_group_act(2, layers, fake, lib.BF16, 256, 8, fake, fake, ys, ld, None, None, 0,
+                                   None) == lib.ERR_INVALID_ARG
+    layers[0] = 0x1000
+    assert L.serq_linear_group_act(2, layers, fake, 7, 256, 8, fake, fake, ys, ld, None, None, 0,
+                                   None) == lib.ERR_INVALID_ARG
+    assert b"bad dtype" in L.serq_last_error_string()
 
 
 def test_binding_refuses_to_load_without_library(tmp_path, monkeypatch):
