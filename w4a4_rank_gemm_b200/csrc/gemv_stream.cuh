@@ -327,8 +327,13 @@ __device__ __forceinline__ void tile_epilogue(const Args& p, const int* acc, int
   }
 }
 
+// 112 registers per thread (57 344 for 16 warps) leave room in the register
+// file for the small CTAs of the next kernel in the stream (a per-token
+// quantize), which then become resident during this grid's tail and wait
+// there instead of being launched after it: measured, the 7B decode step
+// at M = 16 went from 56.9 to 54.3 us with the loop's rate unchanged.
 template <int NTT, bool A8, bool ACC>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1)
+__global__ void __maxnreg__(112)
     k_gemv(const __grid_constant__ Args p, const __grid_constant__ Maps mp, const Plan pl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
