@@ -258,11 +258,15 @@ __global__ void k_upper_from_lower(const double* __restrict__ L2, int K, float* 
   if (U64) U64[e] = v;
 }
 
+constexpr int kUStage = 64;  // rows of U and E staged per shared-memory pass
+
 // GPTQ on one weight.  A CTA owns 32 output channels; in each block of 32
 // rows, thread (t, lane) holds row b0 + t of channel n = 32 * blockIdx.x +
 // lane, starting from W^[b0 + t, n] as the round-to-nearest path computes it:
 //   1. the errors of the earlier rows i = r .. b0 - 1, in order:
-//      w -= u_{i, b0+t} * e_i;
+//      w -= u_{i, b0+t} * e_i (staged 64 rows at a time through shared
+//      memory when U fits in L2: measured 2-3x faster at K = 4096, but 3x
+//      slower at K = 11008, where U streams from DRAM);
 //   2. the block's rows in order: row t2 takes its code
 //      code = clamp(rint(w * (7 / amax)), -7, 7) and, when b0 + t2 >= r, its
 //      scaled error e = (w - code * sw) / u_{t2, t2}; the later rows of the
@@ -271,6 +275,7 @@ __global__ void k_upper_from_lower(const double* __restrict__ L2, int K, float* 
 // Each entry therefore receives its updates in increasing row order, every
 // fp32 operation rounded once.  amax is the column's maximum before any
 // update (sw = amax / 7).  E (K x N) keeps the scaled errors of rows >= r.
+template <bool STAGE>
 __global__ void __launch_bounds__(1024) k_gptq_pack_w(prep::WeightView w, const float* __restrict__ s,
                                                        const int32_t* __restrict__ perm, int K, int r,
                                                        const float* __restrict__ amax_col,
@@ -279,6 +284,8 @@ __global__ void __launch_bounds__(1024) k_gptq_pack_w(prep::WeightView w, const 
   __shared__ float ub[32][33];  // U over the block's rows and columns
   __shared__ float es[32][33];  // the block's scaled errors [row][channel]
   __shared__ int qs[32][33];    // the block's codes [row][channel]
+  __shared__ float us[kUStage][33];  // U rows i of a stage, the block's columns
+  __shared__ float eh[kUStage][32];  // scaled errors of those rows, this CTA's channels
   const int t = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = blockIdx.x * 32 + lane;
   const bool live = n < w.N;
@@ -286,11 +293,28 @@ __global__ void __launch_bounds__(1024) k_gptq_pack_w(prep::WeightView w, const 
   const float sw = __fdiv_rn(amax, 7.f);
   for (int b0 = 0; b0 < K; b0 += 32) {
     float x = live ? prep::w_hat(w, s, perm, b0 + t, n) : 0.f;
-    if (live) {
+    // earlier rows' errors in order: staged kUStage rows at a time through
+    // shared memory (STAGE, U in L2), else read directly, every warp on its
+    // own (more loads in flight when U comes from DRAM)
+    if (STAGE) {
+      for (int i0 = r; i0 < b0; i0 += kUStage) {
+        const int ni = min(kUStage, b0 - i0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < kUStage * 32; e += blockDim.x) {
+          const int ii = e >> 5, c = e & 31;
+          const bool in = ii < ni;
+          us[ii][c] = in ? U[(size_t)(i0 + ii) * K + b0 + c] : 0.f;
+          eh[ii][c] = (in && blockIdx.x * 32 + c < w.N) ? E[(size_t)(i0 + ii) * w.N + blockIdx.x * 32 + c] : 0.f;
+        }
+        __syncthreads();
+        for (int ii = 0; ii < ni; ++ii) x = __fsub_rn(x, __fmul_rn(us[ii][t], eh[ii][lane]));
+      }
+    } else if (live) {
       const float* ucol = U + b0 + t;  // u_{i, b0+t}: the same for the whole warp
 #pragma unroll 8
       for (int i = r; i < b0; ++i) x = __fsub_rn(x, __fmul_rn(ucol[(size_t)i * K], E[(size_t)i * w.N + n]));
     }
+    __syncthreads();
     ub[t][lane] = U[(size_t)(b0 + t) * K + b0 + lane];
     __syncthreads();
     for (int t2 = 0; t2 < 32; ++t2) {

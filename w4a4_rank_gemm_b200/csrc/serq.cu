@@ -949,11 +949,20 @@ serq_status prepare_impl(int n_weights, const float* const* W, const int* N, int
     cudaMemsetAsync(Li->sw, 0, sizeof(float) * Ni, st);
     k_colmax_what<<<dim3((Ni + 255) / 256, (K + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(
         v, L0->smooth, L0->perm, K, rows_per_block, Li->sw);
-    if (o.quantizer == SERQ_QUANT_GPTQ)
-      serq::gptq::k_gptq_pack_w<<<(Ni + 31) / 32, 1024, 0, st>>>(v, L0->smooth, L0->perm, K, rank, Li->sw, U32, E,
-                                                                 Li->wq);
-    else
+    if (o.quantizer == SERQ_QUANT_GPTQ) {
+      // U and E staged through shared memory when U (K x K fp32) stays in L2;
+      // measured: 2-3x faster at K = 4096 (even with E at 180 MB), 3x slower
+      // at K = 11008, where U streams from DRAM
+      const bool stage = (size_t)K * K * sizeof(float) <= (size_t)64 << 20;
+      if (stage)
+        serq::gptq::k_gptq_pack_w<true><<<(Ni + 31) / 32, 1024, 0, st>>>(v, L0->smooth, L0->perm, K, rank, Li->sw,
+                                                                          U32, E, Li->wq);
+      else
+        serq::gptq::k_gptq_pack_w<false><<<(Ni + 31) / 32, 1024, 0, st>>>(v, L0->smooth, L0->perm, K, rank, Li->sw,
+                                                                           U32, E, Li->wq);
+    } else {
       k_quant_pack_w<<<dim3((Ni + 127) / 128, K / 32), 128, 0, st>>>(v, L0->smooth, L0->perm, K, Li->sw, Li->wq);
+    }
     if (rank > 0) {
       k_colmax_resid<<<(Ni + 127) / 128, 128, 0, st>>>(v, L0->smooth, L0->perm, rank, Li->sw, Li->sr);
       k_quant_pack_r<<<dim3((Ni + 127) / 128, Li->rpad / 32), 128, 0, st>>>(v, L0->smooth, L0->perm, rank,
