@@ -93,6 +93,35 @@ def linear_bytes(M, K, N, r, a_bits):
     return N * K / 2 + N * rpad / 2 + 8 * N + M * K * a_bits / 8 + 4 * M + 2 * M * N
 
 
+def fuses_act_quantize(decode, grouped, M, K):
+    """Whether a shared-input group runs as one serq_linear_group_act launch
+    whose GEMV CTAs quantize the tokens themselves (decode, grouped, M <= 8,
+    K <= 4096); otherwise the quantize is a launch of its own."""
+    return bool(decode and grouped and M <= 8 and K <= 4096)
+
+
+def residual_summary(times):
+    """times[(projection, v)] = us per call for v = 0 (main products only),
+    1 (SERQ: main + its rank-r compensator in the same launch), 2 (main, then
+    the two-factor comparator's products).  Returns the per-projection
+    figures, the summed residual times and the comparator / SERQ ratio.
+    SERQ's residual rides in the main launch; where its added time is below
+    the timings' noise (1% of the main products: run-to-run spread of these
+    event timings) the ratio divides by that floor and says so."""
+    per = {}
+    sum_serq = sum_two = sum_main = 0.0
+    for name in dict.fromkeys(n for n, _ in times):
+        t0, t1, t2 = (times[(name, v)] for v in range(3))
+        per[name] = {"main_us": round(t0, 2), "serq_us": round(t1, 2), "two_factor_us": round(t2, 2),
+                     "serq_residual_us": round(t1 - t0, 2), "two_factor_residual_us": round(t2 - t0, 2)}
+        sum_main += t0
+        sum_serq += t1 - t0
+        sum_two += t2 - t0
+    floor = 0.01 * sum_main
+    return {"per": per, "sum_main": sum_main, "sum_serq": sum_serq, "sum_two": sum_two,
+            "ratio": sum_two / max(sum_serq, floor), "at_floor": sum_serq < floor}
+
+
 def max_over_ranks(x: float, world: int, device=None) -> float:
     """Max of a per-rank float over the process group (the step time of a
     weak-scaling job is its slowest rank's)."""
@@ -256,9 +285,7 @@ class LayerWorkload:
                 f"({shapes}), {len(self.grp)} shared-input quantizes, M = {self.M} tokens per GPU")
 
     def fused(self, iname, projs):
-        """Whether the group runs as one serq_linear_group_act launch (M <= 8,
-        K <= 4096: the GEMV quantizes the tokens itself)."""
-        return self.decode and self.M <= 8 and self.grouped and self.wl.inputs[iname].K <= 4096
+        return fuses_act_quantize(self.decode, self.grouped, self.M, self.wl.inputs[iname].K)
 
     def step(self, i, stream, events=None, gemm_only=False):
         S, torch = self.S, self.torch
@@ -720,24 +747,12 @@ def run_compare(args):
                 del gs
     if S.device_error() != 0:
         raise RuntimeError("a kernel reported a timed-out wait")
-    per = {}
-    sum_serq = sum_two = sum_main = 0.0
-    for pr in projs:
-        t0, t1, t2 = (times[(pr["name"], v)] for v in range(3))
-        per[pr["name"]] = {"main_us": round(t0, 2), "serq_us": round(t1, 2), "two_factor_us": round(t2, 2),
-                           "serq_residual_us": round(t1 - t0, 2), "two_factor_residual_us": round(t2 - t0, 2)}
-        sum_main += t0
-        sum_serq += t1 - t0
-        sum_two += t2 - t0
-    # SERQ's residual rides in the main launch; where its added time is below
-    # the timings' noise (1% of the main products: run-to-run spread of
-    # these event timings) the ratio uses that floor, and says so.
-    floor = 0.01 * sum_main
-    ratio = sum_two / max(sum_serq, floor)
+    rs = residual_summary(times)
+    per, sum_main, sum_serq, sum_two, ratio = rs["per"], rs["sum_main"], rs["sum_serq"], rs["sum_two"], rs["ratio"]
     return {
         "metric": "residual-path latency: two-factor comparator (L2QER) / SERQ, one Llama-2-7B layer",
         "value": round(ratio, 3), "unit": "x", "higher_is_better": True, "n_gpus": 1,
-        "serq_residual_at_noise_floor": sum_serq < floor,
+        "serq_residual_at_noise_floor": rs["at_floor"],
         "steps": reps, "warmup": 3, "ms_per_step": round((sum_main + sum_serq) / 1e3, 4),
         "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 (W4A4 codes, int32 accumulate)",
