@@ -505,6 +505,102 @@ serq_status serq_test_decode_timeout(const serq_layer* layer, const void* Xq, co
 /* Library version string. */
 const char* serq_version(void);
 
+/*
+ * ---------------------------------------------------------------------------
+ * SERQ with MXFP4 codes.  The SERQ pages name MXFP4 beside INT4 as a data
+ * format the method supports and quote their Blackwell latency on it
+ * (gist.science (de) sections 3 "Kompatibilität" and 4 "Performance &
+ * Latenz", about 1% over plain MXFP4; gist.science (ja) section 2: with R in
+ * 4 bits the linear is 4-bit integer or MXFP4 arithmetic).  The format is
+ * the OCP Microscaling (MX) one: blocks of 32 consecutive elements along K
+ * share a power-of-two scale stored as an E8M0 byte (2^(byte - 127)), every
+ * element is FP4 E2M1 (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; sign in bit
+ * 3).  A block's exponent is floor(log2(max|v|)) - 2 clamped to [-127, 127]
+ * (-127 for an all-zero block); an element is v / 2^e rounded to the
+ * nearest E2M1 value, ties to the even code, beyond 6 to 6, zero as +0.
+ *
+ * The steps of serq_prepare stay as they are (the smoothing scales s and
+ * the saliency order P are taken from a prepared INT4 layer); W^, R and the
+ * per-token activations are MXFP4 instead of INT4, and the GEMM multiplies
+ * the codes on the tensor core with the block scales applied inside it, the
+ * residual product X~_{s,q} Q(R) accumulating into the same fp32 sums:
+ *     Y = deq(X_q) deq(W^_q) + deq(X_q[:, 0:r]) deq(R_q)     (rounded to bf16).
+ *
+ * Storage: codes two per byte in K order (element 2i in the low nibble),
+ * rows of K/2 bytes.  Scales of the GEMM's operands are TILED: 1 KB tiles of
+ * 128 rows x 8 blocks (256 elements of K), row-major over (row / 128,
+ * block / 8), 8 bytes per row inside a tile; the byte of (row m, block b) is
+ * at ((m / 128) * (K / 256) + b / 8) * 1024 + (m % 128) * 8 + b % 8.
+ * Shapes: K a multiple of 256, N a multiple of 128, r a multiple of 32.
+ * ---------------------------------------------------------------------------
+ */
+typedef struct serq_mx_layer serq_mx_layer;
+
+/*
+ * serq_mx_prepare -- the offline stage with MXFP4 codes.
+ *  base  a prepared layer (not owned; may be destroyed afterwards) whose
+ *        smoothing scales s, saliency order P and rank r are used; prepared
+ *        without an output fold, from the same W.
+ *  W     DEVICE, K x N fp32 row-major, the weight base was prepared from.
+ *  out   receives the handle (NULL on failure; nothing leaks).
+ * W^ = P diag(s) W (one fp32 multiply per element, as serq_prepare) is
+ * quantized per output channel in blocks of 32 along K; R = W^[0:r] -
+ * deq(W^_q)[0:r] (one fp32 subtraction, the dequantized value being exact)
+ * is quantized the same way.
+ * Errors: SERQ_ERR_INVALID_ARG (null pointers, layer of another device),
+ * SERQ_ERR_UNSUPPORTED_SHAPE (K not a multiple of 256, N not of 128, r not
+ * of 32), SERQ_ERR_ALLOC, SERQ_ERR_CUDA, SERQ_ERR_UNSUPPORTED_DEVICE.
+ * Synchronous.
+ */
+serq_status serq_mx_prepare(const serq_layer* base, const float* W, serq_mx_layer** out);
+
+/* Frees the layer's device memory.  NULL accepted. */
+void serq_mx_destroy(serq_mx_layer* q);
+
+/* Synchronous copies to HOST buffers (any may be NULL), scales UNTILED:
+ * wq N x K/2 bytes, we N x K/32 E8M0 bytes, rq N x r/2 bytes, re N x r/32
+ * E8M0 bytes (rq and re untouched when r = 0). */
+serq_status serq_mx_get_packed(const serq_mx_layer* q, uint8_t* wq, uint8_t* we, uint8_t* rq, uint8_t* re);
+
+/* Bytes of the tiled activation scales for M tokens of K channels:
+ * ceil(M / 128) * 128 * K / 32 (rows past M hold zero bytes); 0 for an
+ * invalid shape. */
+size_t serq_mx_act_scale_bytes(int M, int K);
+
+/*
+ * serq_mx_quantize_act -- per-token MXFP4 of the flattened, permuted
+ * activations X^ (serq_flatten_permute's output), blocks of 32 along K.
+ *  Xh    DEVICE M x K (row stride ldxh elements, rows 16-byte aligned), bf16
+ *        or fp32.
+ *  Xq    DEVICE M x K/2 bytes (written).
+ *  xe    DEVICE serq_mx_act_scale_bytes(M, K) bytes, tiled (written).
+ * The residual product reads the first r/32 blocks of the same codes and
+ * scales.  Inputs must be finite.  Errors: SERQ_ERR_INVALID_ARG (null or
+ * misaligned pointers, bad dtype or M), SERQ_ERR_UNSUPPORTED_SHAPE (K not a
+ * positive multiple of 256), SERQ_ERR_CUDA.  Asynchronous on `stream`.
+ */
+serq_status serq_mx_quantize_act(const void* Xh, serq_dtype dtype, int M, int K, int ldxh, void* Xq, void* xe,
+                                 void* stream);
+
+/*
+ * serq_mx_linear -- Y = deq(X_q) deq(W^_q) + deq(X_q[:, 0:r]) deq(R_q) for
+ * codes and tiled scales from serq_mx_quantize_act.  One launch: 128 x 128
+ * output tiles, tcgen05.mma kind::mxf4 with E8M0 block scales, fp32
+ * accumulation in tensor memory (summation order within the tensor core
+ * unspecified), bf16 output by round-to-nearest-even.
+ *  Y, ldy  DEVICE bf16 M x N output, row stride ldy elements (a multiple of
+ *          8, >= N).
+ * Errors: SERQ_ERR_INVALID_ARG (null or misaligned pointers, M outside
+ * [1, 65535 * 128], bad ldy), SERQ_ERR_CUDA.  A wait that gives up is
+ * reported by serq_device_error.  Asynchronous on `stream`.
+ * Validation: the codes and scales of serq_mx_prepare and
+ * serq_mx_quantize_act are bit-exact against the CPU oracle on a B200; this
+ * product's parity with the replicated scale-word layout is not yet
+ * confirmed on a B200.
+ */
+serq_status serq_mx_linear(const serq_mx_layer* q, const void* Xq, const void* xe, int M, void* Y, int ldy,
+                           void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -182,3 +182,28 @@ def test_comparator_host_side_rejection(lib):
     assert b"null comparator" in L.serq_last_error_string()
     assert L.serq_l2qer_accum(None, fake, fake, 4, fake, fake, 0, None) == lib.ERR_INVALID_ARG
     L.serq_l2qer_destroy(None)
+
+
+def test_mxfp4_host_side_rejection(lib):
+    """The MXFP4 calls check their arguments on the host; the scale-size
+    helper is pure host arithmetic."""
+    L = lib.lib
+    out = ctypes.c_void_p()
+    fake = ctypes.c_void_p(0x1000)
+    assert L.serq_mx_prepare(None, fake, ctypes.byref(out)) == lib.ERR_INVALID_ARG
+    assert L.serq_mx_prepare(fake, None, ctypes.byref(out)) == lib.ERR_INVALID_ARG
+    assert out.value is None
+    assert L.serq_mx_linear(None, fake, fake, 4, fake, 256, None) == lib.ERR_INVALID_ARG
+    assert b"null MXFP4 layer" in L.serq_last_error_string()
+    assert L.serq_mx_get_packed(None, None, None, None, None) == lib.ERR_INVALID_ARG
+    # K must be a positive multiple of 256; rows 16-byte aligned; M in range
+    assert L.serq_mx_quantize_act(fake, lib.BF16, 4, 384, 384, fake, fake, None) == lib.ERR_UNSUPPORTED_SHAPE
+    assert L.serq_mx_quantize_act(fake, lib.BF16, 4, 256, 260, fake, fake, None) == lib.ERR_INVALID_ARG
+    assert L.serq_mx_quantize_act(fake, lib.F32, 0, 256, 256, fake, fake, None) == lib.ERR_INVALID_ARG
+    assert L.serq_mx_quantize_act(None, lib.F32, 4, 256, 256, fake, fake, None) == lib.ERR_INVALID_ARG
+    assert L.serq_mx_quantize_act(fake, 7, 4, 256, 256, fake, fake, None) == lib.ERR_INVALID_ARG
+    # scales of M tokens: rows padded to 128, K / 32 bytes each
+    assert lib.mx_act_scale_bytes(1, 256) == 128 * 8
+    assert lib.mx_act_scale_bytes(130, 4096) == 256 * 128
+    assert lib.mx_act_scale_bytes(4, 100) == 0 and lib.mx_act_scale_bytes(0, 256) == 0
+    L.serq_mx_destroy(None)

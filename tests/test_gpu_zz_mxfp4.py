@@ -1,0 +1,188 @@
+"""GPU parity of SERQ with MXFP4 codes (serq_mx_*) against the CPU oracle
+(oracle/mxfp4_oracle.py):
+
+* the offline codes and E8M0 scales of W^ and R, and the per-token
+  activation codes and tiled scales, bit for bit (both sides take every
+  rounding decision on exactly scaled fp32 values);
+* the product Y against the oracle's fp64 value of the same codes within
+  |y - y_ref| <= 1e-2 * max(|y_ref|, 1e-3) + (64 + (K + rpad) / 64) * 2^-20 * S,
+  S = sum_k |x_k w_k| over both products: the first term is the bf16 output
+  rounding with the usual margin; the second bounds the accumulation -- each
+  instruction's 64-term sum inside the tensor core and each of the
+  (K + rpad) / 64 additions into the fp32 accumulator errs by at most 2^-20
+  (8 fp32 ulps: the tensor core's internal alignment is not documented, and
+  one ulp per addition was exceeded once in 16384 outputs) of a partial sum
+  no larger than S.  A wrong scale, block or operand moves an output by a
+  block's contribution, orders of magnitude above this.
+
+Collected after the other GPU parity files.  The GEMM tests are non-strict
+expected failures until the block-scaled GEMM's parity is confirmed on a
+B200; the quantizers' tests are plain.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import mxfp4_oracle as X
+from oracle import serq_oracle as O
+from tests.gpu_support import dev
+
+pytestmark = pytest.mark.gpu
+
+# Each tensor-core sub-partition reads the scale words from its own TMEM lane
+# quarter, so B's scales are replicated in all four quarters; this layout
+# has not yet run on a B200.
+GEMM_UNCONFIRMED = pytest.mark.xfail(
+    strict=False, reason="block-scaled GEMM: parity with the replicated scale-word layout not yet confirmed on a B200")
+
+
+@pytest.fixture(scope="module")
+def S():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from w4a4_rank_gemm_b200 import serq
+    assert serq.lib.serq_check_device() == serq.OK, serq.lib.serq_last_error_string()
+    return serq
+
+
+def _bf16_dev(a):
+    """bf16 CUDA tensor holding the bf16-representable fp32 array a, built
+    from its bits (no conversion arithmetic)."""
+    bits = (np.ascontiguousarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16).view(np.int16)
+    return torch.from_numpy(bits).view(torch.bfloat16).cuda()
+
+
+def _calib(rng, n, K):
+    Xc = rng.standard_normal((n, K)).astype(np.float32)
+    Xc[:, rng.choice(K, 4, replace=False)] *= 25.0
+    return Xc
+
+
+def _layer(S, K, N, r, seed):
+    rng = np.random.default_rng(seed)
+    W = (0.02 * rng.standard_normal((K, N))).astype(np.float32)
+    W[rng.choice(K, 3, replace=False)] *= 6.0
+    Xc = _calib(rng, 64, K)
+    base = S.prepare_host(W, Xc, rank=r)
+    q = S.MXLayer(base, dev(W))
+    return q, base, X.prepare(W, Xc, r), rng
+
+
+def _check_packed(q, ol):
+    got = q.get_packed()
+    assert np.array_equal(got["wq"], X.pack_fp4_rows(ol.q_w)), "W^ codes differ"
+    assert np.array_equal(got["we"], X.e8m0_bytes(ol.e_w)), "W^ scales differ"
+    if ol.r:
+        assert np.array_equal(got["rq"], X.pack_fp4_rows(ol.q_r)), "R codes differ"
+        assert np.array_equal(got["re"], X.e8m0_bytes(ol.e_r)), "R scales differ"
+
+
+def _tolerance(y_ref, Sabs, K, r):
+    rpad = (r + 255) // 256 * 256
+    return 1e-2 * np.maximum(np.abs(y_ref), 1e-3) + (64 + (K + rpad) / 64) * 2.0 ** -20 * Sabs
+
+
+# smallest first: one tile, one step, no compensator
+LINEAR = [
+    (128, 256, 128, 0),
+    (128, 256, 128, 32),
+    (200, 512, 256, 64),
+    (77, 1024, 384, 128),
+    (300, 2048, 256, 256),
+    (5, 4096, 128, 128),
+    (260, 1280, 128, 288),
+]
+
+
+def test_prepare_bit_exact(S):
+    for K, N, r in [(256, 128, 0), (512, 256, 64), (1024, 128, 288)]:
+        q, _, ol, _ = _layer(S, K, N, r, seed=K + r)
+        _check_packed(q, ol)
+
+
+@pytest.mark.parametrize("M,K", [(1, 256), (130, 512), (300, 4096)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quantize_act_bit_exact(S, M, K, dtype):
+    rng = np.random.default_rng(M + K)
+    Xh = (rng.standard_normal((M, K)) * np.exp(rng.uniform(-6, 6, (M, 1)))).astype(np.float32)
+    Xh[0, 32:64] = 0.0                                  # an all-zero block
+    Xh[-1, :32] = np.float32(3.0e-39)                   # subnormal block maximum
+    if dtype == torch.bfloat16:
+        Xh = O.to_bf16(Xh)
+        Xq, xe = S.mx_quantize_act(_bf16_dev(Xh))
+    else:
+        Xq, xe = S.mx_quantize_act(dev(Xh))
+    torch.cuda.synchronize()
+    c, e = X.quantize_act(Xh)
+    assert np.array_equal(Xq.cpu().numpy(), X.pack_fp4_rows(c)), "activation codes differ"
+    assert np.array_equal(xe.cpu().numpy(), X.tile_scales(e)), "activation scales differ"
+
+
+@GEMM_UNCONFIRMED
+@pytest.mark.parametrize("M,K,N,r", LINEAR)
+def test_linear_parity(S, M, K, N, r):
+    q, base, ol, rng = _layer(S, K, N, r, seed=M + K + N + r)
+    _check_packed(q, ol)
+    Xraw = rng.standard_normal((M, K)).astype(np.float32)
+    Xraw[:, rng.choice(K, 3, replace=False)] *= 20.0
+    Xraw = O.to_bf16(Xraw)                              # bf16 activations
+    Xh = S.flatten_permute(base, _bf16_dev(Xraw), out_dtype=torch.bfloat16)
+    xh = O.flatten_permute(Xraw, ol.s, ol.pi, out_bf16=True)
+    Xq, xe = S.mx_quantize_act(Xh)
+    Y = S.mx_linear(q, Xq, xe)
+    torch.cuda.synchronize()
+    xq, xs = X.quantize_act(xh)
+    assert np.array_equal(Xq.cpu().numpy(), X.pack_fp4_rows(xq)), "activation codes differ"
+    y_ref = X.linear_codes(xq, xs, ol)
+    tol = _tolerance(y_ref, X.abs_products(xq, xs, ol), K, r)
+    got = Y.float().cpu().numpy().astype(np.float64)
+    bad = np.abs(got - y_ref) > tol
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} outputs outside tolerance; worst "
+                           f"{np.max(np.abs(got - y_ref) / np.maximum(np.abs(y_ref), 1e-3)):.3g} relative")
+    assert S.device_error() == 0
+
+
+@GEMM_UNCONFIRMED
+def test_residual_moves_the_output_towards_full_precision(S):
+    # the compensator is live in the kernel: with r > 0 the output is closer
+    # to the unquantized-weight product than the same kernel at r = 0
+    K, N, M = 1024, 256, 64
+    rng = np.random.default_rng(5)
+    W = (0.02 * rng.standard_normal((K, N))).astype(np.float32)
+    Xc = _calib(rng, 64, K)
+    Xraw = O.to_bf16(Xc[:M])
+    errs = []
+    for r in (0, 256):
+        base = S.prepare_host(W, Xc, rank=r)
+        q = S.MXLayer(base, dev(W))
+        Xh = S.flatten_permute(base, _bf16_dev(Xraw), out_dtype=torch.bfloat16)
+        Xq, xe = S.mx_quantize_act(Xh)
+        Y = S.mx_linear(q, Xq, xe).float().cpu().numpy()
+        ol = X.prepare(W, Xc, r)
+        xh = O.flatten_permute(Xraw, ol.s, ol.pi, out_bf16=True)
+        Yfull = xh.astype(np.float64) @ ol.W_hat.astype(np.float64)
+        errs.append(np.linalg.norm(Y - Yfull) / np.linalg.norm(Yfull))
+    assert errs[1] < errs[0]
+
+
+@GEMM_UNCONFIRMED
+def test_outputs_into_a_wider_buffer_and_rejections(S):
+    q, base, ol, rng = _layer(S, 512, 256, 64, seed=9)
+    M = 40
+    Xh = _bf16_dev(O.to_bf16(rng.standard_normal((M, 512)).astype(np.float32)))
+    Xq, xe = S.mx_quantize_act(Xh)
+    Ybig = torch.full((M, 384), 7.0, dtype=torch.bfloat16, device="cuda")
+    S.mx_linear(q, Xq, xe, Y=Ybig[:, 64:320])
+    Y = S.mx_linear(q, Xq, xe)
+    torch.cuda.synchronize()
+    assert torch.equal(Ybig[:, 64:320], Y)
+    assert torch.all(Ybig[:, :64] == 7.0) and torch.all(Ybig[:, 320:] == 7.0)
+    with pytest.raises(RuntimeError):
+        S.mx_linear(q, Xq, xe, Y=torch.empty((M, 250), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(RuntimeError):                   # K not a multiple of 256
+        S.mx_quantize_act(torch.zeros((4, 96), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(RuntimeError):                   # r not a multiple of 32
+        rng2 = np.random.default_rng(1)
+        W = rng2.standard_normal((256, 128)).astype(np.float32)
+        S.MXLayer(S.prepare_host(W, _calib(rng2, 8, 256), rank=40), dev(W))
+    assert S.device_error() == 0

@@ -21,6 +21,7 @@
 #include "prepare.cuh"
 #include "gptq.cuh"
 #include "quant.cuh"
+#include "mxfp4.cuh"
 
 namespace {
 
@@ -1534,6 +1535,208 @@ serq_status serq_l2qer_accum(const serq_l2qer* q, const void* Xq, const void* Zq
   if (!aligned16(Xq) || !aligned16(acc0) || !aligned16(acc1))
     return fail(SERQ_ERR_INVALID_ARG, "Xq, acc0, acc1 must be 16-byte aligned");
   return l2qer_final(q, Xq, nullptr, M, Zq, nullptr, nullptr, 0, acc0, acc1, algo, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------
+// SERQ with MXFP4 codes: the base layer's smoothing scales and saliency
+// order, W^ and R in OCP MX blocks of 32 along K, the block-scaled
+// tcgen05 GEMM (mxfp4.cuh).
+// ------------------------------------------------------------------------
+struct serq_mx_layer {
+  int K, N, r, rpad, device;
+  void* block;
+  uint8_t* wq;  // N x K/2 codes
+  uint8_t* we;  // tiled scales of W^ (N x K/32)
+  uint8_t* rq;  // N x rpad/2 codes (zero past r)
+  uint8_t* re;  // tiled scales of R (N x rpad/32)
+  CUtensorMap tmW, tmR;
+};
+
+namespace {
+
+void free_mx(serq_mx_layer* q) {
+  if (!q) return;
+  if (q->block) cudaFree(q->block);
+  delete q;
+}
+
+serq_status check_mx(const serq_mx_layer* q) {
+  if (!q) return fail(SERQ_ERR_INVALID_ARG, "null MXFP4 layer");
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != q->device)
+    return fail(SERQ_ERR_INVALID_ARG, "layer was prepared on device %d, current device is %d", q->device, dev);
+  return check_device();
+}
+
+// Tiled scales -> plain rows x n_blocks bytes on the host.
+void untile_scales(const uint8_t* tiled, int rows, int n_blocks, uint8_t* out) {
+  for (int i = 0; i < rows; ++i)
+    for (int b = 0; b < n_blocks; ++b) out[(size_t)i * n_blocks + b] = tiled[serq::mx::scale_offset(i, b, n_blocks)];
+}
+
+}  // namespace
+
+extern "C" {
+
+serq_status serq_mx_prepare(const serq_layer* base, const float* W, serq_mx_layer** out) {
+  if (!out) return fail(SERQ_ERR_INVALID_ARG, "null out");
+  *out = nullptr;
+  if (!base || !W) return fail(SERQ_ERR_INVALID_ARG, "null base layer or W");
+  serq_status s;
+  if ((s = check_device())) return s;
+  if ((s = check_layer(base))) return s;
+  const int K = base->K, N = base->N, r = base->rank;
+  if (K % serq::mx::kTileK || N % 128)
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "MXFP4 needs K a multiple of 256 and N of 128 (K = %d, N = %d)", K, N);
+  if (r % serq::mx::kBlock)
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "MXFP4 needs the rank to be a multiple of 32 (r = %d)", r);
+  serq_mx_layer* q = new (std::nothrow) serq_mx_layer();
+  if (!q) return fail(SERQ_ERR_ALLOC, "host allocation failed");
+  std::memset(q, 0, sizeof(*q));
+  q->K = K;
+  q->N = N;
+  q->r = r;
+  q->rpad = (r + serq::mx::kTileK - 1) / serq::mx::kTileK * serq::mx::kTileK;
+  q->device = base->device;
+  const size_t s_wq = up256((size_t)N * K / 2), s_we = up256((size_t)N * K / 32);
+  const size_t s_rq = up256((size_t)N * q->rpad / 2), s_re = up256((size_t)N * q->rpad / 32);
+  cudaError_t e = cudaMalloc(&q->block, s_wq + s_we + s_rq + s_re + 256);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    free_mx(q);
+    return fail(SERQ_ERR_ALLOC, "cudaMalloc for the MXFP4 layer failed: %s", cudaGetErrorString(e));
+  }
+  uint8_t* b = static_cast<uint8_t*>(q->block);
+  q->wq = b;
+  q->we = b + s_wq;
+  q->rq = b + s_wq + s_we;
+  q->re = b + s_wq + s_we + s_rq;
+  cudaStream_t st;
+  e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    free_mx(q);
+    return cuda_fail(e, "cudaStreamCreate");
+  }
+  const serq::prep::WeightView v{W, N, nullptr, nullptr};
+  serq::mx::k_quant_w<<<dim3(N / 128, K / serq::mx::kBlock), 128, 0, st>>>(v, base->smooth, base->perm, K, r, q->rpad,
+                                                                          q->wq, q->we, q->rq, q->re);
+  e = cudaGetLastError();
+  const cudaError_t e2 = cudaStreamSynchronize(st);
+  cudaStreamDestroy(st);
+  if (e == cudaSuccess) e = e2;
+  if (e != cudaSuccess) {
+    free_mx(q);
+    return cuda_fail(e, "serq_mx_prepare");
+  }
+  const bool okw = make_map(&q->tmW, q->wq, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+  const bool okr = q->rpad == 0 ? true
+                                : make_map(&q->tmR, q->rq, (uint64_t)q->rpad / 2, (uint64_t)N, (uint64_t)q->rpad / 2,
+                                           128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!okw || !okr) {
+    free_mx(q);
+    return fail(SERQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the MXFP4 layer");
+  }
+  if (q->rpad == 0) q->tmR = q->tmW;  // never read when r = 0
+  *out = q;
+  return ok();
+}
+
+void serq_mx_destroy(serq_mx_layer* q) { free_mx(q); }
+
+serq_status serq_mx_get_packed(const serq_mx_layer* q, uint8_t* wq, uint8_t* we, uint8_t* rq, uint8_t* re) {
+  serq_status s;
+  if ((s = check_mx(q))) return s;
+  const int nb = q->K / 32, nbr = q->rpad / 32;
+  cudaError_t e = cudaSuccess;
+  if (wq) e = cudaMemcpy(wq, q->wq, (size_t)q->N * q->K / 2, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && we) {
+    std::vector<uint8_t> t((size_t)q->N * nb);
+    e = cudaMemcpy(t.data(), q->we, t.size(), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) untile_scales(t.data(), q->N, nb, we);
+  }
+  if (e == cudaSuccess && q->r > 0 && (rq || re)) {
+    std::vector<uint8_t> c((size_t)q->N * q->rpad / 2), t((size_t)q->N * nbr);
+    e = cudaMemcpy(c.data(), q->rq, c.size(), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(t.data(), q->re, t.size(), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) {
+      std::vector<uint8_t> plain((size_t)q->N * nbr);
+      untile_scales(t.data(), q->N, nbr, plain.data());
+      for (int n = 0; n < q->N; ++n) {
+        if (rq) std::memcpy(rq + (size_t)n * q->r / 2, c.data() + (size_t)n * q->rpad / 2, (size_t)q->r / 2);
+        if (re) std::memcpy(re + (size_t)n * q->r / 32, plain.data() + (size_t)n * nbr, (size_t)q->r / 32);
+      }
+    }
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "serq_mx_get_packed");
+  return ok();
+}
+
+size_t serq_mx_act_scale_bytes(int M, int K) {
+  if (M < 1 || K < serq::mx::kTileK || K % serq::mx::kTileK) return 0;
+  return (size_t)((M + 127) / 128 * 128) * (size_t)(K / 32);
+}
+
+serq_status serq_mx_quantize_act(const void* Xh, serq_dtype dtype, int M, int K, int ldxh, void* Xq, void* xe,
+                                 void* stream) {
+  if (!Xh || !Xq || !xe) return fail(SERQ_ERR_INVALID_ARG, "null pointer argument");
+  if (dtype != SERQ_F32 && dtype != SERQ_BF16) return fail(SERQ_ERR_INVALID_ARG, "bad dtype %d", (int)dtype);
+  if (M < 1 || M > 65535 * 128) return fail(SERQ_ERR_INVALID_ARG, "M = %d out of range", M);
+  if (K < serq::mx::kTileK || K % serq::mx::kTileK)
+    return fail(SERQ_ERR_UNSUPPORTED_SHAPE, "MXFP4 needs K a positive multiple of 256 (got %d)", K);
+  const int esz = dtype == SERQ_F32 ? 4 : 2;
+  if (ldxh < K || ((size_t)ldxh * esz) % 16 || !aligned16(Xh) || !aligned16(Xq) || !aligned16(xe))
+    return fail(SERQ_ERR_INVALID_ARG, "Xh, Xq, xe must be 16-byte aligned and ldxh >= K with 16-byte rows");
+  serq_status s;
+  if ((s = check_device())) return s;
+  const int Mpad = (M + 127) / 128 * 128;
+  const long n = (long)Mpad * (K / 32);
+  const int threads = 256;
+  const unsigned blocks = (unsigned)((n + threads - 1) / threads);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == SERQ_BF16)
+    serq::mx::k_quant_act<uint16_t><<<blocks, threads, 0, st>>>(static_cast<const uint16_t*>(Xh), M, K, ldxh, Mpad,
+                                                                static_cast<uint8_t*>(Xq), static_cast<uint8_t*>(xe));
+  else
+    serq::mx::k_quant_act<float><<<blocks, threads, 0, st>>>(static_cast<const float*>(Xh), M, K, ldxh, Mpad,
+                                                             static_cast<uint8_t*>(Xq), static_cast<uint8_t*>(xe));
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "serq_mx_quantize_act launch");
+  return ok();
+}
+
+serq_status serq_mx_linear(const serq_mx_layer* q, const void* Xq, const void* xe, int M, void* Y, int ldy,
+                           void* stream) {
+  serq_status s;
+  if ((s = check_mx(q))) return s;
+  if (!Xq || !xe || !Y) return fail(SERQ_ERR_INVALID_ARG, "null pointer argument");
+  if (M < 1 || M > 65535 * 128) return fail(SERQ_ERR_INVALID_ARG, "M = %d out of range", M);
+  if (!aligned16(Xq) || !aligned16(xe) || !aligned16(Y) || ldy < q->N || ldy % 8)
+    return fail(SERQ_ERR_INVALID_ARG, "Xq, xe, Y must be 16-byte aligned, ldy >= N and a multiple of 8");
+  CUtensorMap tmA;
+  if (!make_map(&tmA, Xq, (uint64_t)q->K / 2, (uint64_t)M, (uint64_t)q->K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(SERQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for Xq");
+  serq::mx::Args a;
+  a.xe = static_cast<const uint8_t*>(xe);
+  a.we = q->we;
+  a.re = q->re;
+  a.Y = static_cast<__nv_bfloat16*>(Y);
+  a.ldy = ldy;
+  a.M = M;
+  a.N = q->N;
+  a.K = q->K;
+  a.rpad = q->rpad;
+  cudaError_t e = serq::smem_limit(reinterpret_cast<const void*>(serq::mx::k_gemm), serq::mx::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (MXFP4 GEMM)");
+  const dim3 grid(q->N / 128, (M + 127) / 128);
+  serq::mx::k_gemm<<<grid, serq::mx::kThreads, serq::mx::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+      tmA, q->tmW, q->tmR, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "serq_mx_linear launch");
+  return ok();
 }
 
 }  // extern "C"

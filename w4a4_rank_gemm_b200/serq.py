@@ -67,6 +67,12 @@ EXPORTS = {
     "serq_l2qer_get_packed": (_i, [_vp, _vp, _vp, _vp, _vp]),
     "serq_l2qer_linear": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp]),
     "serq_l2qer_accum": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp]),
+    "serq_mx_prepare": (_i, [_vp, _vp, ctypes.POINTER(_vp)]),
+    "serq_mx_destroy": (None, [_vp]),
+    "serq_mx_get_packed": (_i, [_vp, _vp, _vp, _vp, _vp]),
+    "serq_mx_act_scale_bytes": (ctypes.c_size_t, [_i, _i]),
+    "serq_mx_quantize_act": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "serq_mx_linear": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp]),
     "serq_silu_mul_quantize": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "serq_flatten_permute": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _i, _vp]),
     "serq_test_decode_timeout": (_i, [_vp, _vp, _vp, _i, _vp, _i, _i, _vp]),
@@ -496,6 +502,74 @@ class L2QER:
         _check(lib.serq_l2qer_accum(self._h, _ptr(Xq), _ptr(Zq), M, _ptr(acc0), _ptr(acc1), algo, _stream(stream)),
                "serq_l2qer_accum")
         return acc0, acc1
+
+
+class MXLayer:
+    """Owner of a SERQ layer with MXFP4 codes (serq_mx_prepare): the smoothing
+    scales, saliency order and rank of a prepared INT4 layer, W^ and R in OCP
+    MX blocks of 32 along K."""
+
+    def __init__(self, base: Layer, W: torch.Tensor):
+        if not W.is_cuda or W.dtype != torch.float32 or not W.is_contiguous() or W.shape != (base.K, base.N):
+            raise ValueError("W must be the base layer's contiguous K x N fp32 CUDA weight")
+        self.K, self.N, self.r = base.K, base.N, base.rank
+        h = _vp()
+        _check(lib.serq_mx_prepare(base.handle, _ptr(W), ctypes.byref(h)), "serq_mx_prepare")
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h:
+            lib.serq_mx_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def get_packed(self) -> dict:
+        """Codes (N x K/2, N x r/2 bytes) and untiled E8M0 scale bytes
+        (N x K/32, N x r/32)."""
+        import numpy as np
+        wq = np.empty((self.N, self.K // 2), np.uint8)
+        we = np.empty((self.N, self.K // 32), np.uint8)
+        rq = np.empty((self.N, self.r // 2), np.uint8)
+        re = np.empty((self.N, self.r // 32), np.uint8)
+        c = lambda a: a.ctypes.data_as(_vp)
+        _check(lib.serq_mx_get_packed(self._h, c(wq), c(we), c(rq), c(re)), "serq_mx_get_packed")
+        return dict(wq=wq, we=we, rq=rq, re=re)
+
+
+def mx_act_scale_bytes(M: int, K: int) -> int:
+    return int(lib.serq_mx_act_scale_bytes(M, K))
+
+
+def mx_quantize_act(Xh: torch.Tensor, Xq: Optional[torch.Tensor] = None, xe: Optional[torch.Tensor] = None,
+                    stream=None):
+    """Per-token MXFP4 codes (M x K/2 bytes) and tiled E8M0 scales."""
+    _cuda2d(Xh, "Xh")
+    M, K = Xh.shape
+    if Xq is None:
+        Xq = torch.empty((M, K // 2), dtype=torch.uint8, device=Xh.device)
+    if xe is None:
+        xe = torch.empty(max(1, mx_act_scale_bytes(M, K)), dtype=torch.uint8, device=Xh.device)
+    _check(lib.serq_mx_quantize_act(_ptr(Xh), _dtype_code(Xh), M, K, Xh.stride(0), _ptr(Xq), _ptr(xe),
+                                    _stream(stream)), "serq_mx_quantize_act")
+    return Xq, xe
+
+
+def mx_linear(layer: MXLayer, Xq: torch.Tensor, xe: torch.Tensor, Y: Optional[torch.Tensor] = None, stream=None):
+    M = Xq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=Xq.device)
+    _check(lib.serq_mx_linear(layer.handle, _ptr(Xq), _ptr(xe), M, _ptr(Y), Y.stride(0), _stream(stream)),
+           "serq_mx_linear")
+    return Y
 
 
 def device_error() -> int:
