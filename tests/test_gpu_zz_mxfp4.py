@@ -30,8 +30,8 @@ from tests.gpu_support import dev
 pytestmark = pytest.mark.gpu
 
 # Each tensor-core sub-partition reads the scale words from its own TMEM lane
-# quarter, so B's scales are replicated in all four quarters; this layout
-# has not yet run on a B200.
+# quarter, so B's scales are replicated in all four quarters; the GEMM with
+# that layout has not yet run on a B200.
 GEMM_UNCONFIRMED = pytest.mark.xfail(
     strict=False, reason="block-scaled GEMM: parity with the replicated scale-word layout not yet confirmed on a B200")
 

@@ -219,21 +219,25 @@ __device__ __forceinline__ void umma_mxf4(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
-// Scale words of one stage for the 32 TMEM lanes of one warp quarter.  The
+// Scale words of one stage for the 32 TMEM lanes of warp quarter q.  The
 // block-scaled MMA's sub-partition q (output rows 32q..32q+31) reads its
-// scale factors from its own lane quarter only: A's row m = 32q + i from
-// lane m at column m / 32 of the slot, and B's row n (every n) from lane
-// 32q + n % 32 at column n / 32.  So every quarter holds the same 32 x 4
-// words: lane 32q + i, column c = the scales of row i + 32c.  For MMA k
-// (elements 64k..64k+63 of the stage) each operand has one such 4-column
-// slot; bytes 0-1 of a word are the row's scales of blocks 2k and 2k+1
-// (scale-factor id 0), repeated in bytes 2-3.
-__device__ __forceinline__ void stage_scale_words(const uint8_t* sf, int lane, uint32_t* w) {
+// scale factors from its own lane quarter only.  B's row n is read, for
+// every q, from lane 32q + n % 32 at column n / 32 of the operand's slot, so
+// B's words are the same in every quarter: column c holds row lane + 32c.
+// A's row m = 32q + lane is read from lane m, at the slot's column m / 32
+// (or its first column): A's column 0 holds the lane's own row and column
+// c >= 1 row lane + 32c, which serves both.  For MMA k (elements
+// 64k..64k+63 of the stage) each operand has one 4-column slot; bytes 0-1 of
+// a word are the row's scales of blocks 2k and 2k+1 (scale-factor id 0),
+// repeated in bytes 2-3.
+template <bool A_OPERAND>
+__device__ __forceinline__ void stage_scale_words(const uint8_t* sf, int q, int lane, uint32_t* w) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const uint32_t b = *reinterpret_cast<const uint16_t*>(sf + (lane + 32 * c) * 8 + 2 * k);
+      const int row = (A_OPERAND && c == 0) ? 32 * q + lane : lane + 32 * c;
+      const uint32_t b = *reinterpret_cast<const uint16_t*>(sf + row * 8 + 2 * k);
       w[4 * k + c] = b | (b << 16);
     }
   }
@@ -350,8 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       uint32_t words[32];
-      stage_scale_words(smem + oSFA + s * kSfTile, lane, words);
-      stage_scale_words(smem + oSFB + s * kSfTile, lane, words + 16);
+      stage_scale_words<true>(smem + oSFA + s * kSfTile, q, lane, words);
+      stage_scale_words<false>(smem + oSFB + s * kSfTile, q, lane, words + 16);
       tmem_st_32x32b_x32(tmem + lane_base + kSfCol + 32u * (uint32_t)s, words);
       tmem_st_wait();
       tc_fence_before();
