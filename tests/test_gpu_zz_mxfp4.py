@@ -11,7 +11,8 @@
   instruction's 64-term sum inside the tensor core and each of the
   (K + rpad) / 64 additions into the fp32 accumulator errs by at most 2^-20
   (8 fp32 ulps: the tensor core's internal alignment is not documented, and
-  one ulp per addition was exceeded once in 16384 outputs) of a partial sum
+  the one-ulp form failed one output on a B200 that no scale error explains)
+  of a partial sum
   no larger than S.  A wrong scale, block or operand moves an output by a
   block's contribution, orders of magnitude above this.
 
